@@ -1,0 +1,484 @@
+// C ABI of the group-wise fully quantized int8 Winograd convolution library.
+// Argument checking, workspace layout and kernel orchestration; all
+// arithmetic of the convolution runs in the CUDA kernels.
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <new>
+#include <vector>
+
+#include "../../include/wino.h"
+#include "kernels.h"
+#include "plan.h"
+
+struct wino_plan_s {
+    wino::Matrices mat;
+    wino::TransformArgs tf;
+    wino::WeightArgs wa;
+    int G = 0;
+    bool bt_masked = false, at_masked = false;
+    wino_opts opts;
+    int last_cuda = 0;
+    // per-kernel timing (wino_profile_begin / wino_profile_end)
+    std::vector<cudaEvent_t> prof_events;
+    int prof_max_calls = 0, prof_calls = 0, prof_launches = 0;
+};
+
+namespace {
+
+using namespace wino;
+
+constexpr size_t kAlign = 256;
+size_t up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+struct Layout {
+    int TH = 0, TW = 0, n2 = 0, ng = 0, ngo = 0;
+    long T = 0, T_pad = 0;
+    int y_path = 0, gemm = 0;
+    bool dbg_yq = false, dbg_acc = false;
+    size_t off_vq = 0, off_sv = 0, off_amax = 0, off_yq = 0, off_y32 = 0, off_sy = 0, off_acc = 0, off_err = 0;
+    size_t total = 0;
+};
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int num_sms() {
+    static int sms = 0;
+    if (!sms) {
+        int dev = 0;
+        cudaGetDevice(&dev);
+        if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0) sms = 148;
+    }
+    return sms;
+}
+
+// Byte / ALU cost model choosing how Y reaches the output transform.
+int choose_y_path(const wino_plan_s* p, long T, int Cin, int Cout, int n2) {
+    const double hbm = 6.5e12;          // bytes/s
+    const double alu = 148.0 * 128 * 1.6e9;  // fp32 lane-ops/s
+    const double ng = (double)Cin / p->G;
+    const double tpad = (double)((T + 127) / 128 * 128);
+    const double v = (double)T * n2 * Cin * (1.0 + 4.0 / p->G);
+    const double u = (double)n2 * Cout * Cin * (1.0 + 4.0 / p->G);
+    const double y = (double)T * n2 * Cout;
+    const double epi = tpad * n2 * Cout * ng * 4.0 / alu;  // dequant epilogue of one GEMM pass
+    const double t_rec = std::max((v + u) / hbm, epi) + std::max((v + u + y) / hbm, epi) + (y) / hbm;
+    const double t_y32 = std::max((v + u + 4 * y) / hbm, epi) + 4 * y / hbm;
+    return t_rec < t_y32 ? WINO_YPATH_RECOMPUTE : WINO_YPATH_Y32;
+}
+
+int check_shape(const wino_plan_s* p, int N, int H, int W, int Cin, int Cout) {
+    if (!p || N <= 0 || H <= 0 || W <= 0 || Cin <= 0 || Cout <= 0) return WINO_ERR_INVALID_ARG;
+    if (Cin % p->G != 0 || Cout % p->G != 0 || Cin % 32 != 0 || Cout % 32 != 0) return WINO_ERR_INVALID_ARG;
+    return WINO_OK;
+}
+
+Layout make_layout(const wino_plan_s* p, int N, int H, int W, int Cin, int Cout) {
+    Layout L;
+    const int m = p->mat.m, n = p->mat.n;
+    L.TH = (H + m - 1) / m;
+    L.TW = (W + m - 1) / m;
+    L.n2 = n * n;
+    L.T = (long)N * L.TH * L.TW;
+    L.T_pad = (L.T + 127) / 128 * 128;
+    L.ng = Cin / p->G;
+    L.ngo = Cout / p->G;
+    L.gemm = p->opts.gemm == WINO_GEMM_AUTO ? WINO_GEMM_TCGEN05 : p->opts.gemm;
+    if (L.gemm == WINO_GEMM_TCGEN05 && tc_block_n(Cout, p->G) == 0) L.gemm = WINO_GEMM_SIMT;
+    L.y_path = p->opts.y_path == WINO_YPATH_AUTO ? choose_y_path(p, L.T, Cin, Cout, L.n2) : p->opts.y_path;
+    L.dbg_yq = (p->opts.debug & WINO_DEBUG_YQ) != 0;
+    L.dbg_acc = (p->opts.debug & WINO_DEBUG_ACC32) != 0;
+    size_t off = 0;
+    L.off_vq = off;
+    off = up(off + (size_t)L.T_pad * L.n2 * Cin, kAlign);
+    L.off_sv = off;
+    off = up(off + sizeof(float) * (size_t)L.n2 * L.ng * L.T_pad, kAlign);
+    L.off_amax = off;
+    off = up(off + sizeof(unsigned) * (size_t)L.T_pad * L.ngo, kAlign);
+    if (L.y_path == WINO_YPATH_RECOMPUTE || L.dbg_yq) {
+        L.off_yq = off;
+        off = up(off + (size_t)L.T * L.n2 * Cout, kAlign);
+    }
+    if (L.y_path == WINO_YPATH_Y32) {
+        L.off_y32 = off;
+        off = up(off + sizeof(float) * (size_t)L.T * L.n2 * Cout, kAlign);
+    }
+    if (L.dbg_yq) {
+        L.off_sy = off;
+        off = up(off + sizeof(float) * (size_t)L.T * L.ngo, kAlign);
+    }
+    if (L.dbg_acc) {
+        L.off_acc = off;
+        off = up(off + sizeof(int) * (size_t)L.n2 * L.T * Cout * L.ng, kAlign);
+    }
+    L.off_err = off;
+    off = up(off + 16, kAlign);
+    L.total = off;
+    return L;
+}
+
+int cuda_status(wino_plan_s* p, cudaError_t e) {
+    if (e == cudaSuccess) return WINO_OK;
+    p->last_cuda = (int)e;
+    return WINO_ERR_CUDA;
+}
+
+constexpr int kMaxLaunches = 4;
+
+// Records profiling event `slot` of the current call (no-op unless profiling).
+void prof_mark(wino_plan_s* p, int slot, cudaStream_t st) {
+    if (p->prof_calls >= p->prof_max_calls) return;
+    cudaEventRecord(p->prof_events[(size_t)p->prof_calls * (kMaxLaunches + 1) + slot], st);
+}
+
+int run_conv(wino_plan_s* p, const void* x, int x_dtype, int N, int H, int W, int Cin, const void* wt, int Cout,
+             void* y, int y_dtype, void* ws, size_t ws_bytes, cudaStream_t st) {
+    int rc = check_shape(p, N, H, W, Cin, Cout);
+    if (rc) return rc;
+    if (!x || !wt || !y || !ws || !aligned16(x) || !aligned16(wt) || !aligned16(y) || !aligned16(ws))
+        return WINO_ERR_INVALID_ARG;
+    if ((x_dtype != WINO_BF16 && x_dtype != WINO_F32) || (y_dtype != WINO_BF16 && y_dtype != WINO_F32))
+        return WINO_ERR_INVALID_ARG;
+    const Layout L = make_layout(p, N, H, W, Cin, Cout);
+    if (ws_bytes < L.total) return WINO_ERR_WORKSPACE;
+    unsigned char* base = static_cast<unsigned char*>(ws);
+    int8_t* Vq = reinterpret_cast<int8_t*>(base + L.off_vq);
+    float* sV = reinterpret_cast<float*>(base + L.off_sv);
+    unsigned* amax = reinterpret_cast<unsigned*>(base + L.off_amax);
+    int8_t* Yq = L.off_yq ? reinterpret_cast<int8_t*>(base + L.off_yq) : nullptr;
+    float* Y32 = L.off_y32 ? reinterpret_cast<float*>(base + L.off_y32) : nullptr;
+    float* sYd = L.dbg_yq ? reinterpret_cast<float*>(base + L.off_sy) : nullptr;
+    int* acc = L.dbg_acc ? reinterpret_cast<int*>(base + L.off_acc) : nullptr;
+    int* err = reinterpret_cast<int*>(base + L.off_err);
+    const int8_t* Uq = static_cast<const int8_t*>(wt);
+    const float* sU = reinterpret_cast<const float*>(static_cast<const unsigned char*>(wt) +
+                                                     up((size_t)L.n2 * Cout * Cin, kAlign));
+
+    InputArgs ia;
+    ia.x = x;
+    ia.N = N;
+    ia.H = H;
+    ia.W = W;
+    ia.Cin = Cin;
+    ia.TH = L.TH;
+    ia.TW = L.TW;
+    ia.T = L.T;
+    ia.T_pad = L.T_pad;
+    ia.G = p->G;
+    ia.ngo = L.ngo;
+    ia.Vq = Vq;
+    ia.sV = sV;
+    ia.amax = amax;
+    ia.err = err;
+    int slot = 0;
+    prof_mark(p, slot++, st);
+    cudaError_t e = launch_input_transform(ia, p->tf, p->mat.m, p->bt_masked, x_dtype == WINO_BF16, st);
+    if (e != cudaSuccess) return cuda_status(p, e);
+
+    GemmArgs ga;
+    std::memset(&ga, 0, sizeof(ga));
+    ga.T = (int)L.T;
+    ga.T_pad = (int)L.T_pad;
+    ga.Cin = Cin;
+    ga.Cout = Cout;
+    ga.n2 = L.n2;
+    ga.G = p->G;
+    ga.ng = L.ng;
+    ga.ngo = L.ngo;
+    ga.sV = sV;
+    ga.sU = sU;
+    ga.amax = amax;
+    ga.Yq = Yq;
+    ga.Y32 = Y32;
+    ga.acc = acc;
+    ga.err = err;
+    auto gemm = [&](int mode) -> cudaError_t {
+        prof_mark(p, slot++, st);
+        if (L.gemm == WINO_GEMM_SIMT) return launch_hadamard_simt(ga, Vq, Uq, mode, st);
+        return launch_hadamard_tc(ga, Vq, Uq, mode, num_sms(), st, nullptr);
+    };
+    if (L.y_path == WINO_YPATH_RECOMPUTE) {
+        if ((e = gemm(kModeAbsmax)) != cudaSuccess) return cuda_status(p, e);
+        ga.acc = nullptr;
+        if ((e = gemm(kModeQuant)) != cudaSuccess) return cuda_status(p, e);
+    } else {
+        if ((e = gemm(kModeY32)) != cudaSuccess) return cuda_status(p, e);
+    }
+
+    OutputArgs oa;
+    oa.N = N;
+    oa.H = H;
+    oa.W = W;
+    oa.Cout = Cout;
+    oa.TH = L.TH;
+    oa.TW = L.TW;
+    oa.T = L.T;
+    oa.n2 = L.n2;
+    oa.G = p->G;
+    oa.ngo = L.ngo;
+    oa.Yq = Yq;
+    oa.Y32 = Y32;
+    oa.amax = amax;
+    oa.Yq_dbg = (L.y_path == WINO_YPATH_Y32 && L.dbg_yq) ? Yq : nullptr;
+    oa.sY_dbg = sYd;
+    oa.out = y;
+    prof_mark(p, slot++, st);
+    e = launch_output_transform(oa, p->tf, p->mat.m, p->at_masked, L.y_path == WINO_YPATH_Y32, y_dtype == WINO_BF16,
+                                st);
+    prof_mark(p, slot, st);
+    if (p->prof_calls < p->prof_max_calls) {
+        p->prof_launches = slot;
+        ++p->prof_calls;
+    }
+    return cuda_status(p, e);
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* wino_status_string(int s) {
+    switch (s) {
+        case WINO_OK: return "ok";
+        case WINO_ERR_INVALID_ARG: return "invalid argument";
+        case WINO_ERR_UNSUPPORTED: return "unsupported";
+        case WINO_ERR_WORKSPACE: return "workspace or weight buffer too small";
+        case WINO_ERR_CUDA: return "CUDA error";
+        case WINO_ERR_DEVICE_TIMEOUT: return "bounded device wait expired";
+        case WINO_ERR_NOT_EXACT: return "transform not exactly representable";
+        default: return "unknown status";
+    }
+}
+
+int wino_plan(wino_plan_t* out, int m, const double* points, const float* S_B, const float* S_G, int group,
+              const wino_opts* opts) {
+    if (!out) return WINO_ERR_INVALID_ARG;
+    *out = nullptr;
+    if (group != 32 && group != 64 && group != 256) return WINO_ERR_INVALID_ARG;
+    wino_plan_s* p = new (std::nothrow) wino_plan_s();
+    if (!p) return WINO_ERR_INVALID_ARG;
+    int rc = build_matrices(m, points, S_B, S_G, &p->mat);
+    if (rc != WINO_OK) {
+        delete p;
+        return rc;
+    }
+    p->G = group;
+    std::memset(&p->opts, 0, sizeof(p->opts));
+    if (opts) p->opts = *opts;
+    if (p->opts.y_path < 0 || p->opts.y_path > 2 || p->opts.gemm < 0 || p->opts.gemm > 2) {
+        delete p;
+        return WINO_ERR_INVALID_ARG;
+    }
+    const int n = p->mat.n;
+    std::memset(&p->tf, 0, sizeof(p->tf));
+    std::memcpy(p->tf.BT, p->mat.BT, sizeof(float) * n * n);
+    std::memcpy(p->tf.AT, p->mat.AT, sizeof(float) * m * n);
+    std::memcpy(p->wa.G, p->mat.G, sizeof(double) * n * 3);
+    const uint64_t bt_mask = m == 4 ? kMaskBT_F4 : kMaskBT_F6;
+    const uint64_t at_mask = m == 4 ? kMaskAT_F4 : kMaskAT_F6;
+    p->bt_masked = (p->mat.bt_nonzero & ~bt_mask) == 0;
+    p->at_masked = (p->mat.at_nonzero & ~at_mask) == 0;
+    *out = p;
+    return WINO_OK;
+}
+
+int wino_plan_destroy(wino_plan_t p) {
+    if (p)
+        for (cudaEvent_t ev : p->prof_events) cudaEventDestroy(ev);
+    delete p;
+    return WINO_OK;
+}
+
+int wino_plan_matrices(wino_plan_t p, float* BT, double* G, float* AT) {
+    if (!p) return WINO_ERR_INVALID_ARG;
+    const int m = p->mat.m, n = p->mat.n;
+    if (BT) std::memcpy(BT, p->mat.BT, sizeof(float) * n * n);
+    if (G) std::memcpy(G, p->mat.G, sizeof(double) * n * 3);
+    if (AT) std::memcpy(AT, p->mat.AT, sizeof(float) * m * n);
+    return WINO_OK;
+}
+
+int wino_plan_info(wino_plan_t p, int* m, int* n, int* group) {
+    if (!p) return WINO_ERR_INVALID_ARG;
+    if (m) *m = p->mat.m;
+    if (n) *n = p->mat.n;
+    if (group) *group = p->G;
+    return WINO_OK;
+}
+
+size_t wino_weight_bytes(wino_plan_t p, int Cin, int Cout) {
+    if (!p || Cin <= 0 || Cout <= 0 || Cin % p->G || Cout % p->G) return 0;
+    const size_t n2 = (size_t)p->mat.n * p->mat.n;
+    return up(n2 * Cout * Cin, kAlign) + up(sizeof(float) * n2 * (Cin / p->G) * Cout, kAlign);
+}
+
+int wino_transform_weights(wino_plan_t p, const float* w, int Cin, int Cout, void* wt, size_t wt_bytes, void* stream) {
+    if (!p || !w || !wt || !aligned16(w) || !aligned16(wt)) return WINO_ERR_INVALID_ARG;
+    if (check_shape(p, 1, 1, 1, Cin, Cout)) return WINO_ERR_INVALID_ARG;
+    if (wt_bytes < wino_weight_bytes(p, Cin, Cout)) return WINO_ERR_WORKSPACE;
+    const size_t n2 = (size_t)p->mat.n * p->mat.n;
+    int8_t* Uq = static_cast<int8_t*>(wt);
+    float* sU = reinterpret_cast<float*>(static_cast<unsigned char*>(wt) + up(n2 * Cout * Cin, kAlign));
+    return cuda_status(p, launch_weight_transform(p->wa, p->mat.m, w, Cin, Cout, p->G, Uq, sU,
+                                                  static_cast<cudaStream_t>(stream)));
+}
+
+size_t wino_workspace_bytes(wino_plan_t p, int N, int H, int W, int Cin, int Cout) {
+    if (check_shape(p, N, H, W, Cin, Cout)) return 0;
+    return make_layout(p, N, H, W, Cin, Cout).total;
+}
+
+int wino_conv2d_int8(wino_plan_t p, const void* x, int x_dtype, int N, int H, int W, int Cin, const void* wt,
+                      int Cout, void* y, int y_dtype, void* ws, size_t ws_bytes, void* stream) {
+    if (!p) return WINO_ERR_INVALID_ARG;
+    return run_conv(p, x, x_dtype, N, H, W, Cin, wt, Cout, y, y_dtype, ws, ws_bytes,
+                    static_cast<cudaStream_t>(stream));
+}
+
+size_t wino_host_staging_bytes(wino_plan_t p, int N, int H, int W, int Cin, int Cout, int x_dtype, int y_dtype) {
+    if (check_shape(p, N, H, W, Cin, Cout)) return 0;
+    const size_t xs = x_dtype == WINO_BF16 ? 2 : 4, ys = y_dtype == WINO_BF16 ? 2 : 4;
+    return up(xs * N * H * W * Cin, kAlign) + up(ys * N * H * W * Cout, kAlign);
+}
+
+int wino_conv2d_int8_host(wino_plan_t p, const void* x_host, int x_dtype, int N, int H, int W, int Cin,
+                           const void* wt, int Cout, void* y_host, int y_dtype, void* ws, size_t ws_bytes,
+                           void* stream) {
+    if (!p || !x_host || !y_host || !ws) return WINO_ERR_INVALID_ARG;
+    int rc = check_shape(p, N, H, W, Cin, Cout);
+    if (rc) return rc;
+    const size_t need = make_layout(p, N, H, W, Cin, Cout).total;
+    const size_t stage = wino_host_staging_bytes(p, N, H, W, Cin, Cout, x_dtype, y_dtype);
+    if (ws_bytes < need + stage) return WINO_ERR_WORKSPACE;
+    const size_t xs = x_dtype == WINO_BF16 ? 2 : 4, ys = y_dtype == WINO_BF16 ? 2 : 4;
+    const size_t xbytes = xs * N * H * W * Cin, ybytes = ys * N * H * W * Cout;
+    unsigned char* xd = static_cast<unsigned char*>(ws) + need;
+    unsigned char* yd = xd + up(xbytes, kAlign);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    cudaError_t e = cudaMemcpyAsync(xd, x_host, xbytes, cudaMemcpyHostToDevice, st);
+    if (e != cudaSuccess) return cuda_status(p, e);
+    rc = run_conv(p, xd, x_dtype, N, H, W, Cin, wt, Cout, yd, y_dtype, ws, need, st);
+    if (rc) return rc;
+    return cuda_status(p, cudaMemcpyAsync(y_host, yd, ybytes, cudaMemcpyDeviceToHost, st));
+}
+
+int wino_check_device_error(wino_plan_t p, const void* ws, int N, int H, int W, int Cin, int Cout, void* stream) {
+    int rc = check_shape(p, N, H, W, Cin, Cout);
+    if (rc) return rc;
+    if (!ws) return WINO_ERR_INVALID_ARG;
+    const Layout L = make_layout(p, N, H, W, Cin, Cout);
+    cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_status(p, e);
+    int v = 0;
+    e = cudaMemcpy(&v, static_cast<const unsigned char*>(ws) + L.off_err, sizeof(int), cudaMemcpyDeviceToHost);
+    if (e != cudaSuccess) return cuda_status(p, e);
+    return v ? WINO_ERR_DEVICE_TIMEOUT : WINO_OK;
+}
+
+int wino_debug_dump(wino_plan_t p, const void* ws, int N, int H, int W, int Cin, int Cout, int what, void* dst,
+                    size_t bytes) {
+    int rc = check_shape(p, N, H, W, Cin, Cout);
+    if (rc) return rc;
+    if (!ws || !dst) return WINO_ERR_INVALID_ARG;
+    const Layout L = make_layout(p, N, H, W, Cin, Cout);
+    const unsigned char* base = static_cast<const unsigned char*>(ws);
+    size_t need = 0, off = 0;
+    switch (what) {
+        case WINO_DUMP_VQ: need = (size_t)L.T * L.n2 * Cin; off = L.off_vq; break;
+        case WINO_DUMP_SV: need = sizeof(float) * (size_t)L.T * L.n2 * L.ng; off = L.off_sv; break;
+        case WINO_DUMP_YQ:
+            if (!L.off_yq || (L.y_path == WINO_YPATH_Y32 && !L.dbg_yq)) return WINO_ERR_UNSUPPORTED;
+            need = (size_t)L.T * L.n2 * Cout; off = L.off_yq; break;
+        case WINO_DUMP_SY:
+            if (!L.dbg_yq) return WINO_ERR_UNSUPPORTED;
+            need = sizeof(float) * (size_t)L.T * L.ngo; off = L.off_sy; break;
+        case WINO_DUMP_Y32:
+            if (!L.off_y32) return WINO_ERR_UNSUPPORTED;
+            need = sizeof(float) * (size_t)L.T * L.n2 * Cout; off = L.off_y32; break;
+        case WINO_DUMP_ACC32:
+            if (!L.dbg_acc) return WINO_ERR_UNSUPPORTED;
+            need = sizeof(int) * (size_t)L.n2 * L.T * Cout * L.ng; off = L.off_acc; break;
+        default: return WINO_ERR_INVALID_ARG;
+    }
+    if (bytes < need) return WINO_ERR_WORKSPACE;
+    cudaError_t e = cudaDeviceSynchronize();
+    if (e != cudaSuccess) return cuda_status(p, e);
+    if (what != WINO_DUMP_SV) return cuda_status(p, cudaMemcpy(dst, base + off, need, cudaMemcpyDeviceToHost));
+    // scales are stored [n2][ng][T_pad] for coalesced GEMM-epilogue reads; hand them out as [T][n2][ng]
+    std::vector<float> raw((size_t)L.n2 * L.ng * L.T_pad);
+    e = cudaMemcpy(raw.data(), base + off, raw.size() * sizeof(float), cudaMemcpyDeviceToHost);
+    if (e != cudaSuccess) return cuda_status(p, e);
+    float* o = static_cast<float*>(dst);
+    for (long t = 0; t < L.T; ++t)
+        for (int k = 0; k < L.n2; ++k)
+            for (int j = 0; j < L.ng; ++j) o[((size_t)t * L.n2 + k) * L.ng + j] = raw[((size_t)k * L.ng + j) * L.T_pad + t];
+    return WINO_OK;
+}
+
+int wino_resolved_config(wino_plan_t p, int N, int H, int W, int Cin, int Cout, int* y_path, int* gemm) {
+    int rc = check_shape(p, N, H, W, Cin, Cout);
+    if (rc) return rc;
+    const Layout L = make_layout(p, N, H, W, Cin, Cout);
+    if (y_path) *y_path = L.y_path;
+    if (gemm) *gemm = L.gemm;
+    return WINO_OK;
+}
+
+int wino_launches_per_call(wino_plan_t p, int N, int H, int W, int Cin, int Cout) {
+    if (check_shape(p, N, H, W, Cin, Cout)) return 0;
+    const Layout L = make_layout(p, N, H, W, Cin, Cout);
+    return L.y_path == WINO_YPATH_RECOMPUTE ? 4 : 3;
+}
+
+int wino_profile_begin(wino_plan_t p, int max_calls) {
+    if (!p || max_calls <= 0 || max_calls > (1 << 20)) return WINO_ERR_INVALID_ARG;
+    for (cudaEvent_t ev : p->prof_events) cudaEventDestroy(ev);
+    p->prof_events.assign((size_t)max_calls * (kMaxLaunches + 1), nullptr);
+    for (cudaEvent_t& ev : p->prof_events) {
+        cudaError_t e = cudaEventCreate(&ev);
+        if (e != cudaSuccess) {
+            p->prof_max_calls = 0;
+            return cuda_status(p, e);
+        }
+    }
+    p->prof_max_calls = max_calls;
+    p->prof_calls = 0;
+    p->prof_launches = 0;
+    return WINO_OK;
+}
+
+int wino_profile_end(wino_plan_t p, float* ms, int max_launches, int* launches_per_call, int* calls) {
+    if (!p) return WINO_ERR_INVALID_ARG;
+    int rc = WINO_OK;
+    const int nl = p->prof_launches;
+    if (ms)
+        for (int i = 0; i < max_launches; ++i) ms[i] = 0.0f;
+    if (p->prof_calls > 0) {
+        cudaError_t e = cudaEventSynchronize(p->prof_events[(size_t)(p->prof_calls - 1) * (kMaxLaunches + 1) + nl]);
+        if (e != cudaSuccess) rc = cuda_status(p, e);
+        for (int c = 0; rc == WINO_OK && c < p->prof_calls; ++c)
+            for (int i = 0; i < nl && i < max_launches; ++i) {
+                float t = 0.0f;
+                e = cudaEventElapsedTime(&t, p->prof_events[(size_t)c * (kMaxLaunches + 1) + i],
+                                         p->prof_events[(size_t)c * (kMaxLaunches + 1) + i + 1]);
+                if (e != cudaSuccess) {
+                    rc = cuda_status(p, e);
+                    break;
+                }
+                if (ms) ms[i] += t;
+            }
+    }
+    if (launches_per_call) *launches_per_call = nl;
+    if (calls) *calls = p->prof_calls;
+    for (cudaEvent_t ev : p->prof_events) cudaEventDestroy(ev);
+    p->prof_events.clear();
+    p->prof_max_calls = p->prof_calls = p->prof_launches = 0;
+    return rc;
+}
+
+int wino_last_cuda_error(wino_plan_t p) { return p ? p->last_cuda : 0; }
+
+}  // extern "C"

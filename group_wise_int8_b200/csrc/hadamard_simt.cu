@@ -1,0 +1,70 @@
+// Hadamard stage on CUDA cores (cross-check kernel for the tensor-core one).
+// Per tap, tile and output channel: acc_j = exact int32 dot product of the
+// G int8 pairs of K-group j (dp4a), y = fma((float)acc_j, sV_j * sU_j, y) in
+// fp32 for ascending j -- the same arithmetic as the tcgen05 kernel, one
+// thread per output.  Epilogue modes as in the tcgen05 kernel: Y absmax
+// (per tile and G-cout group, over taps, via atomicMax on the float bits),
+// requantisation to int8 with sY = absmax/127, or fp32 Y.
+#include "kernels.h"
+
+namespace wino {
+namespace {
+
+template <int MODE, bool DUMP>
+__global__ void __launch_bounds__(256) hadamard_simt_kernel(GemmArgs p, const int8_t* __restrict__ Vq,
+                                                            const int8_t* __restrict__ Uq) {
+    const int tap = blockIdx.y;
+    const long i = (long)blockIdx.x * blockDim.x + threadIdx.x;
+    const long t = i / p.Cout;
+    const int co = (int)(i - t * p.Cout);
+    if (t >= p.T) return;  // Cout % 32 == 0: uniform per warp
+    const int4* v = reinterpret_cast<const int4*>(Vq + ((size_t)t * p.n2 + tap) * p.Cin);
+    const int4* u = reinterpret_cast<const int4*>(Uq + ((size_t)tap * p.Cout + co) * p.Cin);
+    float y = 0.0f;
+    for (int j = 0; j < p.ng; ++j) {
+        int acc = 0;
+        for (int c = 0; c < p.G / 16; ++c) {
+            const int4 a = v[j * (p.G / 16) + c], b = __ldg(&u[j * (p.G / 16) + c]);
+            acc = __dp4a(a.x, b.x, acc);
+            acc = __dp4a(a.y, b.y, acc);
+            acc = __dp4a(a.z, b.z, acc);
+            acc = __dp4a(a.w, b.w, acc);
+        }
+        if (DUMP) p.acc[(((size_t)tap * p.T + t) * p.Cout + co) * p.ng + j] = acc;
+        const float pr = __fmul_rn(p.sV[((size_t)tap * p.ng + j) * p.T_pad + t], p.sU[((size_t)tap * p.ng + j) * p.Cout + co]);
+        y = __fmaf_rn((float)acc, pr, y);
+    }
+    const size_t o = ((size_t)t * p.n2 + tap) * p.Cout + co;
+    unsigned* am = p.amax + (size_t)t * p.ngo + co / p.G;
+    if (MODE == kModeQuant) {
+        p.Yq[o] = (int8_t)quant_code(y, group_scale(__uint_as_float(*am)));
+    } else {
+        if (MODE == kModeY32) p.Y32[o] = y;
+        const unsigned m = __reduce_max_sync(0xffffffffu, __float_as_uint(fabsf(y)));
+        if ((threadIdx.x & 31) == 0) atomicMax(am, m);  // a warp's 32 couts lie in one group (G >= 32)
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_hadamard_simt(const GemmArgs& a, const int8_t* Vq, const int8_t* Uq, int mode, cudaStream_t st) {
+    const long threads = (long)a.T * a.Cout;
+    const dim3 grid((unsigned)((threads + 255) / 256), a.n2);
+    const bool dump = a.acc != nullptr && mode != kModeQuant;
+    switch (mode) {
+        case kModeAbsmax:
+            if (dump) hadamard_simt_kernel<kModeAbsmax, true><<<grid, 256, 0, st>>>(a, Vq, Uq);
+            else hadamard_simt_kernel<kModeAbsmax, false><<<grid, 256, 0, st>>>(a, Vq, Uq);
+            break;
+        case kModeQuant:
+            hadamard_simt_kernel<kModeQuant, false><<<grid, 256, 0, st>>>(a, Vq, Uq);
+            break;
+        default:
+            if (dump) hadamard_simt_kernel<kModeY32, true><<<grid, 256, 0, st>>>(a, Vq, Uq);
+            else hadamard_simt_kernel<kModeY32, false><<<grid, 256, 0, st>>>(a, Vq, Uq);
+            break;
+    }
+    return cudaGetLastError();
+}
+
+}  // namespace wino

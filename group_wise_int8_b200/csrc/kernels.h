@@ -1,0 +1,69 @@
+// Launchers of the Winograd library's CUDA kernels (internal header).
+#pragma once
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cstdint>
+
+#include "common.cuh"
+
+namespace wino {
+
+// ----------------------------------------------------------- weight transform
+cudaError_t launch_weight_transform(const WeightArgs& wa, int m, const float* w, int Cin, int Cout, int G,
+                                    int8_t* Uq, float* sU, cudaStream_t st);
+
+// ------------------------------------------------------------ input transform
+struct InputArgs {
+    const void* x;   // [N][H][W][Cin] bf16 or fp32
+    int N, H, W, Cin;
+    int TH, TW;      // tiles per column / row
+    long T;          // N * TH * TW
+    long T_pad;      // T rounded up to 128
+    int G;
+    int ngo;         // Cout / G (rows of the Y absmax table to clear)
+    int8_t* Vq;      // [T][n*n][Cin]
+    float* sV;       // [n*n][Cin/G][T_pad]
+    unsigned* amax;  // [T_pad][Cout/G], cleared here
+    int* err;        // device error word, cleared here
+};
+cudaError_t launch_input_transform(const InputArgs& a, const TransformArgs& tf, int m, bool masked, bool bf16_in,
+                                   cudaStream_t st);
+
+// ------------------------------------------------------------ Hadamard GEMM
+enum GemmMode { kModeAbsmax = 0, kModeQuant = 1, kModeY32 = 2 };
+
+struct GemmArgs {
+    int T, T_pad, Cin, Cout, n2, G, ng, ngo;
+    int BK, stages, tpu, num_tc, num_mb, num_nb, num_units;
+    const float* sV;   // [n2][ng][T_pad]
+    const float* sU;   // [n2][ng][Cout]
+    unsigned* amax;    // [T_pad][ngo] fp32 bits of |Y| maxima
+    int8_t* Yq;        // [T][n2][Cout]   (quant mode)
+    float* Y32;        // [T][n2][Cout]   (Y32 mode)
+    int* acc;          // [n2][T][Cout][ng] (debug dump) or null
+    int* err;
+};
+
+// Tensor maps and launch of the tcgen05 kernel; `Vq` is [T_pad][n2][Cin], `Uq` [n2][Cout][Cin].
+cudaError_t launch_hadamard_tc(GemmArgs a, const int8_t* Vq, const int8_t* Uq, int mode, int num_sms,
+                               cudaStream_t st, int* launches);
+int tc_block_n(int Cout, int G);  // 0 if unsupported
+
+cudaError_t launch_hadamard_simt(const GemmArgs& a, const int8_t* Vq, const int8_t* Uq, int mode, cudaStream_t st);
+
+// ----------------------------------------------------------- output transform
+struct OutputArgs {
+    int N, H, W, Cout, TH, TW;
+    long T;
+    int n2, G, ngo;
+    const int8_t* Yq;      // [T][n2][Cout] (Yq source) or written (debug)
+    const float* Y32;      // [T][n2][Cout] (Y32 source)
+    const unsigned* amax;  // [T_pad][ngo]
+    int8_t* Yq_dbg;        // debug copy of Yq (Y32 source), or null
+    float* sY_dbg;         // debug copy of sY [T][ngo], or null
+    void* out;             // [N][H][W][Cout] fp32 or bf16
+};
+cudaError_t launch_output_transform(const OutputArgs& a, const TransformArgs& tf, int m, bool masked, bool src_y32,
+                                    bool bf16_out, cudaStream_t st);
+
+}  // namespace wino

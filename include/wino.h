@@ -1,0 +1,218 @@
+/*
+ * wino.h -- C ABI of the B200 (sm_100a) group-wise fully quantized int8
+ * Winograd convolution library.
+ *
+ * The method: "Data-Free Group-Wise Fully Quantized Winograd Convolution via
+ * Learnable Scales" (arXiv 2412.19867).  A 3x3, stride-1, pad-1 convolution is
+ * computed as F(m,3), m in {4,6}, with transforms built from the Vandermonde
+ * factorisation B^T = S_B V^{-T}, G = S_G V, A^T = V^T S_A, S_A = (S_B S_G)^{-1}
+ * (review page, "What carries the argument"; Sec. 7.1 "Standard Winograd
+ * transforms" for V), and every Winograd stage -- input transform, Hadamard
+ * product, output transform -- group-wise quantised to int8 (Fig. 2).
+ *
+ * Pipeline per call of wino_conv2d_int8 (all stages are CUDA kernels):
+ *   input transform   x -> V = B^T d B per tile and channel, int8 Vq with one
+ *                     fp32 scale per (tile, tap, G input channels);
+ *   Hadamard product  per tap an int8 tensor-core GEMM [tiles x Cin].[Cin x Cout],
+ *                     exact int32 per K-group, y = fma(acc_j, sV_j*sU_j, y) in
+ *                     fp32, ascending j;
+ *   Y requantisation  one fp32 scale per (tile, G output channels) over all
+ *                     n*n taps (the cross-shaped per-tap spread of Y, Fig. 3);
+ *   output transform  out = A^T (sY Yq) A, cropped, NHWC fp32 or bf16.
+ * Quantiser Q everywhere: s = absmax/127, q = clamp(rne(v/s), -127, 127),
+ * s = q = 0 for an all-zero group.
+ *
+ * Conventions
+ *  - Status: every function returning int returns WINO_OK (0) or a negative
+ *    WINO_ERR_* code.  Nothing aborts, throws or traps; no device trap is used.
+ *  - Memory: the caller owns every device buffer and the stream.  The library
+ *    owns only the plan (a host object).  Pointers marked _dev are device
+ *    pointers, _host are host pointers.  Device pointers must be 16-byte
+ *    aligned (WINO_ERR_INVALID_ARG otherwise).
+ *  - Streams: `stream` is a cudaStream_t passed as void* (NULL = legacy
+ *    default stream).  Launching calls are asynchronous on it; the plan and
+ *    query calls are synchronous host calls.
+ *  - Layouts: activations NHWC, weights [Cout][3][3][Cin] fp32 (row-major, C
+ *    order).  Cin and Cout must be multiples of the group size G.
+ *  - Threading: a plan may be used from several host threads as long as the
+ *    calls do not share a workspace concurrently.
+ */
+#ifndef WINO_H_
+#define WINO_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* ---------------------------------------------------------------- status */
+#define WINO_OK 0
+#define WINO_ERR_INVALID_ARG (-1)    /* null/misaligned pointer, bad m, G, shape or points */
+#define WINO_ERR_UNSUPPORTED (-2)    /* valid request this build does not implement */
+#define WINO_ERR_WORKSPACE (-3)      /* workspace or weight buffer smaller than required */
+#define WINO_ERR_CUDA (-4)           /* CUDA runtime/driver error; see wino_last_cuda_error */
+#define WINO_ERR_DEVICE_TIMEOUT (-5) /* a bounded device wait expired; the kernel returned early */
+#define WINO_ERR_NOT_EXACT (-6)      /* transform entries not exactly representable (plan) */
+
+/* ----------------------------------------------------------------- dtypes */
+#define WINO_F32 0
+#define WINO_BF16 1
+
+/* ----------------------------------------------------------------- options */
+/* How Y travels from the Hadamard GEMM to the output transform. */
+#define WINO_YPATH_AUTO 0      /* per layer, by a byte/ALU cost model */
+#define WINO_YPATH_RECOMPUTE 1 /* GEMM pass 1: absmax only; pass 2: recompute, quantise, write int8 Yq */
+#define WINO_YPATH_Y32 2       /* one GEMM pass writes fp32 Y; the output transform requantises it */
+
+/* Which kernel runs the Hadamard GEMM. */
+#define WINO_GEMM_AUTO 0
+#define WINO_GEMM_TCGEN05 1 /* TMA + tcgen05.mma kind::i8, TMEM accumulators (default) */
+#define WINO_GEMM_SIMT 2    /* CUDA-core integer dot-product kernel, for cross-checks */
+
+typedef struct wino_opts {
+    int y_path;    /* WINO_YPATH_* */
+    int gemm;      /* WINO_GEMM_* */
+    int debug;     /* bit 0: materialise Yq and sY in the workspace on every path;
+                      bit 1: dump the int32 per-K-group accumulators (needs the
+                             larger workspace wino_workspace_bytes reports) */
+    int reserved[5];
+} wino_opts;
+
+#define WINO_DEBUG_YQ 1
+#define WINO_DEBUG_ACC32 2
+
+/* Debug dump selectors for wino_debug_dump (logical layouts of the copy). */
+#define WINO_DUMP_VQ 0    /* int8  [T][n*n][Cin]        quantised input transform */
+#define WINO_DUMP_SV 1    /* fp32  [T][n*n][Cin/G]      its scales */
+#define WINO_DUMP_YQ 2    /* int8  [T][n*n][Cout]       requantised Y (needs WINO_DEBUG_YQ on the Y32 path) */
+#define WINO_DUMP_SY 3    /* fp32  [T][Cout/G]          Y scales (needs WINO_DEBUG_YQ) */
+#define WINO_DUMP_Y32 4   /* fp32  [T][n*n][Cout]       dequantised Y (Y32 path only) */
+#define WINO_DUMP_ACC32 5 /* int32 [n*n][T][Cout][Cin/G] per-K-group accumulators (WINO_DEBUG_ACC32) */
+
+typedef struct wino_plan_s* wino_plan_t;
+
+/*
+ * wino_plan -- build the transforms of F(m,3) on the host.
+ *   m       4 or 6 (n = m + 2 interpolation points).
+ *   points  n doubles, the points in tap order; INFINITY is the point at
+ *           infinity (homogeneous (1,0)); finite points must be exact
+ *           dyadic-friendly doubles and pairwise distinct.
+ *   S_B,S_G n fp32 diagonal scales each, nonzero; NULL = identity.
+ *   group   int8 group size G: 32, 64 or 256 (the paper's Sec. 1 sizes).
+ *   opts    NULL = defaults (all zero).
+ * The Vandermonde inverse is computed in exact rational arithmetic; each
+ * entry is rounded once to double, multiplied by the double scale, then
+ * rounded to fp32 (B^T, A^T) or kept in double (G).  A^T uses
+ * S_A[j] = 1/((double)S_B[j] * (double)S_G[j]).
+ * Errors: INVALID_ARG (bad m, group, duplicate or non-finite points, zero
+ * scale), NOT_EXACT (a rational does not fit the exact-rounding rule).
+ * The plan owns no device memory.  Free with wino_plan_destroy.
+ */
+int wino_plan(wino_plan_t* out, int m, const double* points, const float* S_B, const float* S_G, int group,
+              const wino_opts* opts);
+int wino_plan_destroy(wino_plan_t plan);
+
+/* Host copies of the fp32 transforms the kernels use: BT [n][n], AT [m][n],
+ * and the fp64 G [n][3] of the weight transform.  Any pointer may be NULL. */
+int wino_plan_matrices(wino_plan_t plan, float* BT_host, double* G_host, float* AT_host);
+
+/* m, n, G of a plan; any pointer may be NULL. */
+int wino_plan_info(wino_plan_t plan, int* m, int* n, int* group);
+
+/* Bytes of the transformed-weight buffer: int8 Uq [n*n][Cout][Cin] followed
+ * (at a 256-byte boundary) by fp32 sU [n*n][Cin/G][Cout].  0 on bad args. */
+size_t wino_weight_bytes(wino_plan_t plan, int Cin, int Cout);
+
+/*
+ * wino_transform_weights -- offline, once per layer.  U = G g G^T per
+ * (cout, cin) in fp64 (fma chains in ascending index from +0), rounded to
+ * fp32, then Q over G consecutive input channels at fixed (tap, cout).
+ *   w_dev   fp32 [Cout][3][3][Cin] (device).
+ *   wt_dev  caller-owned device buffer of wt_bytes >= wino_weight_bytes().
+ * Asynchronous on stream.  Errors: INVALID_ARG, WORKSPACE, CUDA.
+ */
+int wino_transform_weights(wino_plan_t plan, const float* w_dev, int Cin, int Cout, void* wt_dev, size_t wt_bytes,
+                           void* stream);
+
+/* Bytes of device workspace wino_conv2d_int8 needs for this shape under the
+ * plan's options (includes the debug buffers if the plan enables them). */
+size_t wino_workspace_bytes(wino_plan_t plan, int N, int H, int W, int Cin, int Cout);
+
+/*
+ * wino_conv2d_int8 -- the hot path: one 3x3 stride-1 pad-1 convolution.
+ *   x_dev    [N][H][W][Cin] in x_dtype (WINO_BF16 or WINO_F32), device.
+ *   wt_dev   transformed weights from wino_transform_weights (same plan,
+ *            Cin, Cout).
+ *   y_dev    [N][H][W][Cout] in y_dtype (WINO_F32 or WINO_BF16, RNE), device.
+ *   ws_dev   device workspace of ws_bytes >= wino_workspace_bytes().
+ * Launches the input transform, the Hadamard GEMM (one or two passes) and the
+ * output transform on stream; returns after the launches (asynchronous).
+ * A bounded device wait that expires makes a later call on the same
+ * workspace return WINO_ERR_DEVICE_TIMEOUT (see wino_check_device_error).
+ * Errors: INVALID_ARG, UNSUPPORTED, WORKSPACE, CUDA, DEVICE_TIMEOUT.
+ */
+int wino_conv2d_int8(wino_plan_t plan, const void* x_dev, int x_dtype, int N, int H, int W, int Cin,
+                      const void* wt_dev, int Cout, void* y_dev, int y_dtype, void* ws_dev, size_t ws_bytes,
+                      void* stream);
+
+/* Extra device bytes wino_conv2d_int8_host needs beyond wino_workspace_bytes
+ * (device staging for x and y). */
+size_t wino_host_staging_bytes(wino_plan_t plan, int N, int H, int W, int Cin, int Cout, int x_dtype,
+                               int y_dtype);
+
+/*
+ * wino_conv2d_int8_host -- same convolution with HOST input and output
+ * buffers: copies x_host to the device, runs wino_conv2d_int8, copies the
+ * result to y_host, all asynchronously on stream (pinned host memory gives
+ * truly asynchronous copies).  ws_dev must hold wino_workspace_bytes() +
+ * wino_host_staging_bytes().  The caller synchronises the stream before
+ * reading y_host.
+ */
+int wino_conv2d_int8_host(wino_plan_t plan, const void* x_host, int x_dtype, int N, int H, int W, int Cin,
+                           const void* wt_dev, int Cout, void* y_host, int y_dtype, void* ws_dev, size_t ws_bytes,
+                           void* stream);
+
+/* Synchronises stream and reads the workspace's device error word: WINO_OK,
+ * or WINO_ERR_DEVICE_TIMEOUT if a bounded wait in a kernel expired. */
+int wino_check_device_error(wino_plan_t plan, const void* ws_dev, int N, int H, int W, int Cin, int Cout,
+                            void* stream);
+
+/* Synchronous copy of one intermediate tensor of the last call on ws_dev
+ * into host_dst (logical layout per WINO_DUMP_*).  Errors: INVALID_ARG,
+ * UNSUPPORTED (tensor not materialised under these options), WORKSPACE. */
+int wino_debug_dump(wino_plan_t plan, const void* ws_dev, int N, int H, int W, int Cin, int Cout, int what,
+                    void* host_dst, size_t host_bytes);
+
+/* The Y path and GEMM kernel a call of this shape will use (after AUTO). */
+int wino_resolved_config(wino_plan_t plan, int N, int H, int W, int Cin, int Cout, int* y_path, int* gemm);
+
+/* Number of kernels one wino_conv2d_int8 call of this shape launches. */
+int wino_launches_per_call(wino_plan_t plan, int N, int H, int W, int Cin, int Cout);
+
+/*
+ * Per-kernel device timing.  wino_profile_begin(plan, max_calls) makes the
+ * next max_calls calls of wino_conv2d_int8 on this plan record a CUDA event on
+ * their stream before each kernel launch and after the last one (the events
+ * are owned by the plan).  wino_profile_end synchronises on the last event
+ * and returns, per launch index (input transform, GEMM pass(es), output
+ * transform), the summed elapsed milliseconds over the recorded calls, the
+ * number of launches per call and the number of calls recorded; it then
+ * releases the events.  Errors: INVALID_ARG, CUDA.
+ */
+int wino_profile_begin(wino_plan_t plan, int max_calls);
+int wino_profile_end(wino_plan_t plan, float* ms_per_launch, int max_launches, int* launches_per_call,
+                     int* calls);
+
+/* Last CUDA error code seen by this plan (cudaError_t as int), 0 if none. */
+int wino_last_cuda_error(wino_plan_t plan);
+
+/* Static description of a status code. */
+const char* wino_status_string(int status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* WINO_H_ */

@@ -1,0 +1,107 @@
+"""Host-side checks of the C ABI that need no GPU: the library loads, exports
+every entry point include/wino.h declares, and its host plan (transform
+construction, argument checks, workspace sizing) behaves as specified."""
+import ctypes
+import math
+import os
+import re
+
+import numpy as np
+import pytest
+
+import oracle
+from group_wise_int8_b200 import build, synth, wino
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return wino.load_library()
+
+
+def declared_functions():
+    src = open(os.path.join(ROOT, "include", "wino.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(wino_[a-z0-9_]+)\s*\(", src)))
+
+
+def test_header_declares_the_binding_entry_points():
+    assert declared_functions() == sorted(wino.EXPORTED)
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+    out = os.popen("nm -D --defined-only %s" % wino.LIB_PATH).read()
+    for name in declared_functions():
+        assert re.search(r"\bT %s\b" % name, out), name
+
+
+@pytest.mark.parametrize("m,pts", [(4, synth.POINTS_F4), (6, synth.POINTS_F6)])
+@pytest.mark.parametrize("scales", ["identity", "loguniform", "rownorm"])
+def test_plan_matches_oracle_bit_exactly(lib, m, pts, scales):
+    """The library builds V^{-1} from Lagrange basis polynomials, the oracle by
+    Gauss-Jordan elimination; both round the same exact rationals once."""
+    n = m + 2
+    sb = sg = None
+    if scales == "loguniform":
+        r = np.random.default_rng(m)
+        sb = np.exp(r.uniform(math.log(0.5), math.log(2), n)).astype(np.float32)
+        sg = np.exp(r.uniform(math.log(0.5), math.log(2), n)).astype(np.float32)
+    elif scales == "rownorm":
+        p0 = oracle.Plan(m, pts)
+        sb = (1.0 / np.linalg.norm(p0.BT_d, axis=1)).astype(np.float32)
+        sg = (1.0 / np.linalg.norm(p0.G_d, axis=1)).astype(np.float32)
+    op = oracle.Plan(m, pts, sb, sg)
+    BT, G, AT = wino.Plan(m, pts, sb, sg, 32).matrices()
+    assert np.array_equal(BT.view(np.uint32), op.BT_f.view(np.uint32))
+    assert np.array_equal(G.view(np.uint64), op.G_d.view(np.uint64))
+    assert np.array_equal(AT.view(np.uint32), op.AT_f.view(np.uint32))
+
+
+def test_plan_other_point_orders_match_oracle(lib):
+    pts = (math.inf, 0.5, -2.0, 1.0, 0.0, -1.0)   # permuted F(4,3) points: generic (unmasked) kernels
+    op = oracle.Plan(4, pts)
+    BT, G, AT = wino.Plan(4, pts, None, None, 64).matrices()
+    assert np.array_equal(BT, op.BT_f) and np.array_equal(G, op.G_d) and np.array_equal(AT, op.AT_f)
+
+
+@pytest.mark.parametrize("bad", [
+    dict(m=5), dict(group=48), dict(points=(0.0, 1.0, 1.0, 2.0, -2.0, math.inf)),
+    dict(points=(0.0, 1.0, -1.0, math.inf, -2.0, math.inf)), dict(points=(0.0, 1.0, -1.0, 2.0, float("nan"), math.inf)),
+    dict(S_B=[1, 1, 0, 1, 1, 1]),
+])
+def test_plan_rejects_invalid_arguments(lib, bad):
+    kw = dict(m=4, points=synth.POINTS_F4, S_B=None, S_G=None, group=32)
+    kw.update(bad)
+    if kw["m"] != 4:
+        kw["points"] = kw["points"] + (0.5,) * (kw["m"] - 4)
+    with pytest.raises(wino.WinoError) as e:
+        wino.Plan(kw["m"], kw["points"], kw["S_B"], kw["S_G"], kw["group"])
+    assert e.value.status == wino.ERR_INVALID_ARG
+
+
+def test_workspace_and_weight_sizes(lib):
+    p = wino.Plan(6, synth.POINTS_F6, None, None, 32)
+    N, H, W, C = 32, 56, 56, 64
+    T = N * 10 * 10
+    ws = p.workspace_bytes(N, H, W, C, C)
+    Tpad = (T + 127) // 128 * 128
+    assert ws >= Tpad * 64 * C + 4 * 64 * (C // 32) * Tpad + 4 * Tpad * (C // 32) + T * 64 * C
+    assert p.weight_bytes(C, C) >= 64 * C * C + 4 * 64 * (C // 32) * C
+    assert p.workspace_bytes(N, H, W, 48, C) == 0       # Cin not a multiple of G
+    assert p.weight_bytes(C, 40) == 0
+
+
+def test_resolved_config_cost_model(lib):
+    p = wino.Plan(6, synth.POINTS_F6, None, None, 64)
+    # many tiles, few channels: recompute the GEMM rather than round-trip fp32 Y
+    assert p.resolved_config(32, 56, 56, 64, 64)[0] in (wino.YPATH_RECOMPUTE, wino.YPATH_Y32)
+    # few tiles, many channels: re-reading the transformed weights dominates -> fp32 Y
+    assert p.resolved_config(2, 8, 8, 1280, 1280)[0] == wino.YPATH_Y32
+    assert p.resolved_config(2, 8, 8, 1280, 1280)[1] == wino.GEMM_TCGEN05
+    forced = wino.Plan(6, synth.POINTS_F6, None, None, 64, y_path=wino.YPATH_RECOMPUTE, gemm=wino.GEMM_SIMT)
+    assert forced.resolved_config(2, 8, 8, 1280, 1280) == (wino.YPATH_RECOMPUTE, wino.GEMM_SIMT)
+    assert forced.launches_per_call(2, 8, 8, 1280, 1280) == 4

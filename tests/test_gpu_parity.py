@@ -1,0 +1,141 @@
+"""GPU parity: the CUDA path through the C ABI against the CPU oracle on the
+same seeded inputs.
+
+Bar (from the method's specification of this library): every int8 tensor
+(Uq, Vq, Yq), every scale (sU, sV, sY), the int32 per-K-group accumulators and
+the fp32 Y are bit-exact; fp32 outputs agree within 1e-5 relative L2; the
+SQNR against the fp64 direct convolution equals the oracle's to 0.01 dB.
+Zero-coefficient skipping in the transforms can change only the sign of a
+zero, which the quantiser maps to the same code, so value equality is the
+bit-exactness criterion for the fp32 tensors.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from group_wise_int8_b200 import synth, wino
+from tests.gpu_util import assert_bits_equal, bf16_round, rel_l2, run_gpu, run_oracle
+
+pytestmark = pytest.mark.gpu
+
+P4, P6 = synth.POINTS_F4, synth.POINTS_F6
+
+# name: (m, points, N, H, W, Cin, Cout, G, dtype, act, scales)
+CASES = {
+    "tiny_f4": (4, P4, 1, 16, 16, 32, 32, 32, "f32", "normal", "identity"),
+    "ragged_f6_cout96": (6, P6, 2, 13, 11, 64, 96, 32, "bf16", "relu_normal", "loguniform"),
+    "f4_g64_outliers": (4, P4, 1, 20, 20, 128, 64, 64, "bf16", "student_t_outliers", "loguniform"),
+    "f6_g64_cout128": (6, P6, 1, 12, 12, 64, 128, 64, "bf16", "student_t_outliers", "loguniform"),
+    "f6_g256": (6, P6, 1, 8, 8, 256, 256, 256, "bf16", "relu_normal", "loguniform"),
+    "f6_wide_k": (6, P6, 1, 8, 8, 1280, 128, 64, "bf16", "student_t_outliers", "loguniform"),
+    "f4_two_row_blocks": (4, P4, 2, 40, 38, 64, 64, 32, "bf16", "relu_normal", "loguniform"),
+    "f6_single_partial_tile": (6, P6, 1, 3, 5, 32, 32, 32, "f32", "normal", "loguniform"),
+    "f6_one_pixel": (6, P6, 3, 1, 1, 64, 32, 32, "bf16", "relu_normal", "identity"),
+    "f4_permuted_points": (4, (math.inf, 0.5, -2.0, 1.0, 0.0, -1.0), 1, 10, 9, 64, 64, 64, "bf16",
+                           "relu_normal", "loguniform"),
+}
+
+
+def make_case(name, seed=0):
+    m, pts, N, H, W, Cin, Cout, G, dtype, act, scales = CASES[name]
+    layer = synth.random_layer(seed, m, N, H, W, Cin, Cout, G, dtype=dtype, act=act, scales=scales,
+                               w_var_num=2.0, workload="parity_" + name)
+    x_f32, x_bits = synth.make_input(layer)
+    w = synth.make_weights(layer)
+    sb, sg = synth.make_scales(layer)
+    return m, pts, G, x_f32, x_bits, w, sb, sg
+
+
+_oracle_cache = {}
+
+
+def oracle_for(name):
+    if name not in _oracle_cache:
+        m, pts, G, x_f32, x_bits, w, sb, sg = make_case(name)
+        _oracle_cache[name] = run_oracle(m, pts, sb, sg, G, x_f32, w, want_acc=True)
+    return _oracle_cache[name]
+
+
+@pytest.mark.parametrize("gemm", [wino.GEMM_TCGEN05, wino.GEMM_SIMT])
+@pytest.mark.parametrize("y_path", [wino.YPATH_RECOMPUTE, wino.YPATH_Y32])
+@pytest.mark.parametrize("name", list(CASES))
+def test_stagewise_bit_exact(cuda_dev, name, y_path, gemm):
+    m, pts, G, x_f32, x_bits, w, sb, sg = make_case(name)
+    ref = oracle_for(name)
+    got = run_gpu(m, pts, sb, sg, G, x_f32, x_bits, w, out_dtype=torch.float32, y_path=y_path, gemm=gemm,
+                  debug=wino.DEBUG_YQ | wino.DEBUG_ACC32)
+    assert got["gemm"] == gemm and got["y_path"] == y_path
+    for k in ("Uq", "sU", "Vq", "sV", "acc", "Yq", "sY"):
+        assert_bits_equal(k, got[k], ref[k])
+    if y_path == wino.YPATH_Y32:
+        assert_bits_equal("Y", got["Y"], ref["Y"])
+    assert rel_l2(got["out"], ref["out"]) <= 1e-5
+    s_gpu, s_orc = oracle.sqnr_db(ref["ref"], got["out"]), oracle.sqnr_db(ref["ref"], ref["out"])
+    assert abs(s_gpu - s_orc) <= 0.01
+
+
+@pytest.mark.parametrize("name", ["ragged_f6_cout96", "f6_g64_cout128", "f4_two_row_blocks"])
+def test_default_path_bf16_output(cuda_dev, name):
+    """Default options (AUTO path and kernel) with bf16 output, as the benchmark runs them."""
+    m, pts, G, x_f32, x_bits, w, sb, sg = make_case(name)
+    ref = oracle_for(name)
+    got = run_gpu(m, pts, sb, sg, G, x_f32, x_bits, w, out_dtype=torch.bfloat16)
+    assert got["gemm"] == wino.GEMM_TCGEN05
+    want = bf16_round(ref["out"])
+    assert np.array_equal(got["out"], want) or rel_l2(got["out"], want) <= 1e-5
+    assert abs(oracle.sqnr_db(ref["ref"], got["out"]) - oracle.sqnr_db(ref["ref"], want)) <= 0.01
+
+
+def test_host_entry_point_matches_device_call(cuda_dev):
+    m, pts, G, x_f32, x_bits, w, sb, sg = make_case("ragged_f6_cout96")
+    N, H, W, Cin = x_f32.shape
+    Cout = w.shape[0]
+    plan = wino.Plan(m, pts, sb, sg, G)
+    wt = plan.transform_weights(torch.from_numpy(w).cuda())
+    x_host = torch.from_numpy(x_bits.view(np.int16).copy()).view(torch.bfloat16).pin_memory()
+    y_host = torch.empty((N, H, W, Cout), dtype=torch.bfloat16).pin_memory()
+    ws = torch.empty(plan.workspace_bytes(N, H, W, Cin, Cout) + plan.host_staging_bytes(N, H, W, Cin, Cout),
+                     dtype=torch.uint8, device="cuda")
+    plan.conv2d_host(x_host, wt, Cout, y_host, ws)
+    torch.cuda.synchronize()
+    y_dev = plan.conv2d(x_host.cuda(), wt, Cout, out_dtype=torch.bfloat16)
+    torch.cuda.synchronize()
+    assert torch.equal(y_host, y_dev.cpu())
+
+
+def test_repeated_calls_reuse_workspace(cuda_dev):
+    """The workspace carries nothing between calls: a second call on a dirty
+    workspace gives the same bits."""
+    m, pts, G, x_f32, x_bits, w, sb, sg = make_case("f4_two_row_blocks")
+    N, H, W, Cin = x_f32.shape
+    Cout = w.shape[0]
+    plan = wino.Plan(m, pts, sb, sg, G)
+    x = torch.from_numpy(x_bits.view(np.int16).copy()).view(torch.bfloat16).cuda()
+    wt = plan.transform_weights(torch.from_numpy(w).cuda())
+    ws = torch.full((plan.workspace_bytes(N, H, W, Cin, Cout),), 0x7f, dtype=torch.uint8, device="cuda")
+    a = plan.conv2d(x, wt, Cout, out_dtype=torch.float32, workspace=ws).clone()
+    b = plan.conv2d(x, wt, Cout, out_dtype=torch.float32, workspace=ws)
+    torch.cuda.synchronize()
+    assert torch.equal(a, b)
+
+
+def test_argument_errors_are_status_codes(cuda_dev):
+    plan = wino.Plan(4, P4, None, None, 32)
+    x = torch.zeros((1, 8, 8, 32), dtype=torch.bfloat16, device="cuda")
+    w = torch.zeros((32, 3, 3, 32), dtype=torch.float32, device="cuda")
+    wt = plan.transform_weights(w)
+    small = torch.empty(16, dtype=torch.uint8, device="cuda")
+    with pytest.raises(wino.WinoError) as e:
+        plan.conv2d(x, wt, 32, workspace=small)
+    assert e.value.status == wino.ERR_WORKSPACE
+    with pytest.raises(wino.WinoError) as e:
+        plan.conv2d(x, wt, 48)                       # Cout not a multiple of G
+    assert e.value.status == wino.ERR_INVALID_ARG
+    buf = torch.empty(plan.workspace_bytes(1, 8, 8, 32, 32) + 64, dtype=torch.uint8, device="cuda")
+    lib = wino.load_library()
+    rc = lib.wino_conv2d_int8(plan._h, x.data_ptr() + 2, wino.BF16, 1, 8, 8, 32, wt.data_ptr(), 32,
+                              buf.data_ptr(), wino.F32, buf.data_ptr(), buf.numel(), None)
+    assert rc == wino.ERR_INVALID_ARG                # misaligned input pointer

@@ -1,0 +1,66 @@
+"""Full-size sampled parity on every configured layer.
+
+The GPU runs the whole layer in the launch configuration the benchmark times
+(default options: automatic Y path, tcgen05 GEMM, bf16 output).  Every output
+pixel of image i depends only on image i and the weights, so the CPU oracle
+recomputes sampled images one at a time and the matching output slices must
+agree (bf16 of the oracle's fp32 output within 1e-5 relative L2, SQNR equal to
+0.01 dB).  The transformed weights are compared in full, bit for bit.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from group_wise_int8_b200 import synth, wino
+from tests.gpu_util import assert_bits_equal, bf16_round, rel_l2, to_device_input, weight_dumps
+
+pytestmark = pytest.mark.gpu
+
+
+def _layers():
+    out = []
+    for name in ("resnet18", "resnet34", "sd15"):
+        for layer in synth.workload(name):
+            out.append(layer)
+    seen = set()
+    for layer in synth.workload("sd15_stack"):
+        key = (layer.Cin, layer.Cout, layer.H)
+        if key not in seen:
+            seen.add(key)
+            out.append(layer)
+    return out
+
+
+LAYERS = _layers()
+
+
+@pytest.mark.parametrize("layer", LAYERS, ids=[f"{l.workload}{l.index}-{l.describe().replace(' ', '_')}" for l in LAYERS])
+def test_full_size_layer_sampled(cuda_dev, layer):
+    x_f32, x_bits = synth.make_input(layer)
+    w = synth.make_weights(layer)
+    sb, sg = synth.make_scales(layer)
+    plan = wino.Plan(layer.m, layer.points, sb, sg, layer.group)
+    N, H, W, Cin, Cout = layer.N, layer.H, layer.W, layer.Cin, layer.Cout
+    x = to_device_input(x_f32, x_bits)
+    wt = plan.transform_weights(torch.from_numpy(w).cuda())
+    ws = torch.empty(plan.workspace_bytes(N, H, W, Cin, Cout), dtype=torch.uint8, device="cuda")
+    y = plan.conv2d(x, wt, Cout, out_dtype=torch.bfloat16, workspace=ws)
+    torch.cuda.synchronize()
+    assert plan.check_device_error(ws, N, H, W, Cin, Cout) == wino.OK
+    y = y.float().cpu().numpy()
+
+    op = oracle.Plan(layer.m, layer.points, sb, sg)
+    Uq, sU, _ = oracle.weight_transform(op, w, layer.group)
+    gUq, gsU = weight_dumps(plan, wt, Cin, Cout)
+    assert_bits_equal("Uq", gUq, Uq)
+    assert_bits_equal("sU", gsU, sU)
+    images = [0, N - 1] if layer.workload != "sd15_stack" else [N - 1]
+    for i in sorted(set(images)):
+        xi = np.ascontiguousarray(x_f32[i:i + 1])
+        res = oracle.run_pipeline(op, xi, w, layer.group)
+        want = bf16_round(res["out"])
+        got = y[i:i + 1]
+        assert rel_l2(got, want) <= 1e-5, (i, rel_l2(got, want))
+        ref = oracle.conv_direct_f64(xi, w)
+        assert abs(oracle.sqnr_db(ref, got) - oracle.sqnr_db(ref, want)) <= 0.01
