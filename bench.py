@@ -46,7 +46,10 @@ UNIT = "TFLOP/s"
 # (dram__bytes_read.sum + dram__bytes_write.sum); the summary with its command
 # line is the named file under profiles/.  None until a capture of the
 # current kernel exists.
-NCU_TRAFFIC = {}
+NCU_TRAFFIC = {
+    # profiles/resnet18_f63_g32_launches_and_full.md (input transform, CC=64 TX=4 kernel)
+    ("resnet18", 0, "input_transform"): 12904448,
+}
 
 
 def parse():
@@ -112,7 +115,7 @@ class ClockSampler:
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
     def __init__(self, bus_id: str | None):
-        self.bus_id = (bus_id or "").lower()
+        self.bus_id = str(bus_id or "").lower()
         self.proc = None
         self.file = None
 
@@ -193,7 +196,8 @@ def run_ours(args, layer, rank, world):
     ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     bus = None
     try:
-        bus = torch.cuda.get_device_properties(dev).pci_bus_id
+        pr = torch.cuda.get_device_properties(dev)
+        bus = "%08X:%02X:%02X.0" % (int(pr.pci_domain_id), int(pr.pci_bus_id), int(pr.pci_device_id))
     except Exception:
         pass
     sampler = ClockSampler(bus)
