@@ -35,7 +35,8 @@ DUMP_VQ, DUMP_SV, DUMP_YQ, DUMP_SY, DUMP_Y32, DUMP_ACC32 = range(6)
 
 EXPORTED = [
     "wino_plan", "wino_plan_destroy", "wino_plan_matrices", "wino_plan_info", "wino_weight_bytes",
-    "wino_transform_weights", "wino_workspace_bytes", "wino_conv2d_int8", "wino_host_staging_bytes",
+    "wino_transform_weights", "wino_workspace_bytes", "wino_conv2d_int8", "wino_conv2d_int8_noalloc",
+    "wino_host_staging_bytes",
     "wino_conv2d_int8_host", "wino_check_device_error", "wino_debug_dump", "wino_resolved_config",
     "wino_launches_per_call", "wino_profile_begin", "wino_profile_end", "wino_last_cuda_error",
     "wino_status_string",
@@ -80,6 +81,7 @@ def load_library(path: str = LIB_PATH):
     L.wino_workspace_bytes.argtypes = [_vp, _i, _i, _i, _i, _i]
     L.wino_workspace_bytes.restype = _sz
     L.wino_conv2d_int8.argtypes = [_vp, _vp, _i, _i, _i, _i, _i, _vp, _i, _vp, _i, _vp, _sz, _vp]
+    L.wino_conv2d_int8_noalloc.argtypes = [_vp, _vp, _i, _i, _i, _i, _i, _vp, _i, _vp, _i, _vp]
     L.wino_host_staging_bytes.argtypes = [_vp, _i, _i, _i, _i, _i, _i, _i]
     L.wino_host_staging_bytes.restype = _sz
     L.wino_conv2d_int8_host.argtypes = [_vp, _vp, _i, _i, _i, _i, _i, _vp, _i, _vp, _i, _vp, _sz, _vp]
@@ -206,6 +208,15 @@ class Plan:
         self._check(_lib.wino_conv2d_int8(self._h, x.data_ptr(), _dtype_code(x.dtype), N, H, W, Cin, wt.data_ptr(),
                                           Cout, out.data_ptr(), _dtype_code(out.dtype), workspace.data_ptr(),
                                           workspace.numel(), _stream_handle(stream)), "wino_conv2d_int8")
+        return out
+
+    def conv2d_noalloc(self, x: torch.Tensor, wt: torch.Tensor, Cout: int, out: torch.Tensor, stream=None):
+        """wino_conv2d_int8_noalloc: no workspace argument; the library's fixed
+        device scratch array is used instead (see include/wino.h)."""
+        N, H, W, Cin = x.shape
+        self._check(_lib.wino_conv2d_int8_noalloc(self._h, x.data_ptr(), _dtype_code(x.dtype), N, H, W, Cin,
+                                                  wt.data_ptr(), Cout, out.data_ptr(), _dtype_code(out.dtype),
+                                                  _stream_handle(stream)), "wino_conv2d_int8_noalloc")
         return out
 
     def conv2d_host(self, x_host: torch.Tensor, wt: torch.Tensor, Cout: int, y_host: torch.Tensor,

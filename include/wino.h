@@ -157,6 +157,29 @@ int wino_conv2d_int8(wino_plan_t plan, const void* x_dev, int x_dtype, int N, in
                       const void* wt_dev, int Cout, void* y_dev, int y_dtype, void* ws_dev, size_t ws_bytes,
                       void* stream);
 
+/*
+ * wino_conv2d_int8_noalloc -- the same convolution as wino_conv2d_int8 for
+ * callers that cannot allocate device memory (no cudaMalloc available or
+ * allowed where they run, or no way to pass a workspace through their own
+ * interface).  It takes the same inputs and output but no workspace: its
+ * scratch is a fixed array of WINO_NOALLOC_SCRATCH_BYTES inside the library,
+ * which every GPU that loads the library holds until the process exits.  The
+ * call allocates nothing.  (The paper has no counterpart; this is an
+ * interface convenience of this library.)
+ *   - Shapes whose wino_workspace_bytes() exceeds WINO_NOALLOC_SCRATCH_BYTES
+ *     are rejected with WINO_ERR_WORKSPACE before anything is launched.
+ *   - The first call on each device looks up the array's device address
+ *     (cudaGetSymbolAddress) with that device current; make that first call
+ *     before any stream capture.
+ *   - All calls share the array, which keeps the previous call's contents;
+ *     the convolution clears what must start at zero itself.  Calls whose
+ *     kernels overlap on the GPU race on the array: order them.
+ * Errors: INVALID_ARG, WORKSPACE, CUDA, plus those of wino_conv2d_int8.
+ */
+#define WINO_NOALLOC_SCRATCH_BYTES (64u << 20)
+int wino_conv2d_int8_noalloc(wino_plan_t plan, const void* x_dev, int x_dtype, int N, int H, int W, int Cin,
+                             const void* wt_dev, int Cout, void* y_dev, int y_dtype, void* stream);
+
 /* Extra device bytes wino_conv2d_int8_host needs beyond wino_workspace_bytes
  * (device staging for x and y). */
 size_t wino_host_staging_bytes(wino_plan_t plan, int N, int H, int W, int Cin, int Cout, int x_dtype,
