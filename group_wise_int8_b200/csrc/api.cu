@@ -406,15 +406,28 @@ int wino_debug_dump(wino_plan_t p, const void* ws, int N, int H, int W, int Cin,
     if (bytes < need) return WINO_ERR_WORKSPACE;
     cudaError_t e = cudaDeviceSynchronize();
     if (e != cudaSuccess) return cuda_status(p, e);
-    if (what != WINO_DUMP_SV) return cuda_status(p, cudaMemcpy(dst, base + off, need, cudaMemcpyDeviceToHost));
-    // scales are stored [n2][ng][T_pad] for coalesced GEMM-epilogue reads; hand them out as [T][n2][ng]
-    std::vector<float> raw((size_t)L.n2 * L.ng * L.T_pad);
-    e = cudaMemcpy(raw.data(), base + off, raw.size() * sizeof(float), cudaMemcpyDeviceToHost);
+    if (what == WINO_DUMP_SY || what == WINO_DUMP_ACC32)
+        return cuda_status(p, cudaMemcpy(dst, base + off, need, cudaMemcpyDeviceToHost));
+    // The kernels keep these tensors tap-major (Vq [n2][T_pad][Cin]; Yq, Y32 [n2][T][Cout];
+    // sV [n2][ng][T_pad]); the dump hands them out tile-major as documented in wino.h.
+    size_t esz = 1, inner = 0, rows = 0;  // element size, inner extent, stored rows per tap
+    switch (what) {
+        case WINO_DUMP_VQ: esz = 1; inner = Cin; rows = L.T_pad; break;
+        case WINO_DUMP_SV: esz = 4; inner = L.ng; rows = L.T_pad; break;
+        case WINO_DUMP_YQ: esz = 1; inner = Cout; rows = L.T; break;
+        default: esz = 4; inner = Cout; rows = L.T; break;  // Y32
+    }
+    std::vector<unsigned char> raw(esz * inner * rows * L.n2);
+    e = cudaMemcpy(raw.data(), base + off, raw.size(), cudaMemcpyDeviceToHost);
     if (e != cudaSuccess) return cuda_status(p, e);
-    float* o = static_cast<float*>(dst);
+    unsigned char* o = static_cast<unsigned char*>(dst);
     for (long t = 0; t < L.T; ++t)
         for (int k = 0; k < L.n2; ++k)
-            for (int j = 0; j < L.ng; ++j) o[((size_t)t * L.n2 + k) * L.ng + j] = raw[((size_t)k * L.ng + j) * L.T_pad + t];
+            for (size_t c = 0; c < inner; ++c) {
+                const size_t src = what == WINO_DUMP_SV ? ((size_t)k * L.ng + c) * L.T_pad + t
+                                                        : ((size_t)k * rows + t) * inner + c;
+                std::memcpy(o + (((size_t)t * L.n2 + k) * inner + c) * esz, raw.data() + src * esz, esz);
+            }
     return WINO_OK;
 }
 

@@ -48,6 +48,35 @@ __device__ __forceinline__ int quant_code(float v, float s) {
 // Group scale from an absmax.
 __device__ __forceinline__ float group_scale(float amax) { return __fdiv_rn(amax, 127.0f); }
 
+// A group scale with the fp64 reciprocal of its value, for quant_code_fast.
+struct QScale {
+    float s;
+    double rd;  // RN53(1 / s); 0 when s == 0
+};
+
+__device__ __forceinline__ QScale make_qscale(float amax) {
+    QScale q;
+    q.s = group_scale(amax);
+    q.rd = q.s != 0.0f ? __drcp_rn((double)q.s) : 0.0;
+    return q;
+}
+
+// The same code as quant_code(v, s) without a division or a branch.
+// RN24(v/s) = (float)((double)v * RN53(1/s)) for fp32 v and s > 0: the exact
+// quotient of two 24-bit numbers is never an fp32 rounding midpoint and lies at
+// least 2^-49 (relative) away from every midpoint (write v - s*mid as a
+// multiple of the lowest set bit of s*mid), while the fp64 product carries a
+// relative error below 2^-51 (one rounding in the reciprocal, one in the
+// product), so both round to the same fp32 value -- the argument by which
+// double rounding through 53 bits is innocuous for a 24-bit quotient.  The
+// integer step and the clamp then match quant_code exactly.
+__device__ __forceinline__ int quant_code_fast(float v, QScale q) {
+    const float r = __double2float_rn(__dmul_rn((double)v, q.rd));   // RN24(v / s); 0 when s == 0
+    int c = __float_as_int(__fadd_rn(r, kRoundMagic)) - kRoundMagicBits;
+    c = c > 127 ? 127 : c;
+    return c < -127 ? -127 : c;
+}
+
 // Recursive-halving max over the 32 lanes of a warp for 64 values per lane.
 // a[0..63] holds this lane's values; on return a[0], a[1] hold the maxima
 // over all lanes of entries 2*lane and 2*lane + 1.

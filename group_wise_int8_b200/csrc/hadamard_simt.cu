@@ -18,7 +18,7 @@ __global__ void __launch_bounds__(256) hadamard_simt_kernel(GemmArgs p, const in
     const long t = i / p.Cout;
     const int co = (int)(i - t * p.Cout);
     if (t >= p.T) return;  // Cout % 32 == 0: uniform per warp
-    const int4* v = reinterpret_cast<const int4*>(Vq + ((size_t)t * p.n2 + tap) * p.Cin);
+    const int4* v = reinterpret_cast<const int4*>(Vq + ((size_t)tap * p.T_pad + t) * p.Cin);
     const int4* u = reinterpret_cast<const int4*>(Uq + ((size_t)tap * p.Cout + co) * p.Cin);
     float y = 0.0f;
     for (int j = 0; j < p.ng; ++j) {
@@ -34,7 +34,7 @@ __global__ void __launch_bounds__(256) hadamard_simt_kernel(GemmArgs p, const in
         const float pr = __fmul_rn(p.sV[((size_t)tap * p.ng + j) * p.T_pad + t], p.sU[((size_t)tap * p.ng + j) * p.Cout + co]);
         y = __fmaf_rn((float)acc, pr, y);
     }
-    const size_t o = ((size_t)t * p.n2 + tap) * p.Cout + co;
+    const size_t o = ((size_t)tap * p.T + t) * p.Cout + co;
     unsigned* am = p.amax + (size_t)t * p.ngo + co / p.G;
     if (MODE == kModeQuant) {
         p.Yq[o] = (int8_t)quant_code(y, group_scale(__uint_as_float(*am)));

@@ -10,16 +10,25 @@
 //
 // Kernel structure (one CTA per SM, persistent over work units):
 //   unit   = (tap chunk, 128-tile row block, BN-cout column block);
-//   warp 0 = TMA producer: Vq and Uq K-chunks (BK bytes, 32/64/128-byte
-//            swizzle) into a ring of shared-memory stages;
+//   stage  = TPS taps x SK bytes of K (SK a multiple of G, so K-groups never
+//            straddle stages; TPS > 1 only when one stage holds a tap's whole
+//            K); TMA brings the Vq and Uq tiles (3-D boxes over the tap
+//            dimension, 32/64/128-byte swizzle) and the sV / sU scales of the
+//            stage's groups;
+//   warp 0 = TMA producer;
 //   warp 1 = TMEM allocator and MMA issuer: tcgen05.mma kind::i8, M=128,
 //            N=BN, K=32 per instruction; each K-group accumulates into its own
-//            TMEM buffer (a ring of NACC buffers of BN columns) and is
-//            committed to an mbarrier when complete;
-//   warps 2.. = epilogue: tcgen05.ld of a finished buffer, immediate refill of
-//            the buffer with the bias 0x4B400000 (so the next group's int32 sum
-//            lands on 1.5*2^23 and reinterprets as an exact fp32 value), then
-//            the fp32 dequantisation fma per element.
+//            TMEM buffer (a ring of NACC buffers of BN columns, at most NACC/2
+//            groups per stage so the MMAs of the next stage overlap the
+//            epilogue of this one), one commit per group;
+//   warps 2.. = epilogue, 4 TMEM lane quadrants x BN/32 column chunks: one
+//            wait per stage, then per group a 32-column tcgen05.ld and the
+//            dequantisation in packed fp32 pairs; the buffers are refilled with
+//            the bias 0x4B400000 (so the next int32 sum lands on 1.5*2^23 and
+//            reinterprets as an exact fp32 value) and released together.  A
+//            stage returns to the producer when both the MMAs and the epilogue
+//            are done with it.
+// The loops keep wrap-around ring counters (no division in the issue paths).
 // At the end of each tap the epilogue either keeps the running |Y| maximum of
 // each (tile, G-cout group) (absmax pass and fp32-Y pass, published with
 // atomicMax on the float bits at the end of the unit), writes fp32 Y, or
@@ -38,25 +47,38 @@ namespace {
 using namespace sm100;
 
 constexpr int kBM = 128;
+constexpr int kMaxStages = 8;
+constexpr int kMaxNacc = 8;
 
 template <int BN>
 struct TcCfg {
-    static constexpr int kEpiWarps = BN / 8;        // 4 lane quadrants x BN/32 column chunks
+    static constexpr int kEpiWarps = BN / 8;  // 4 lane quadrants x BN/32 column chunks
     static constexpr int kThreads = 64 + 32 * kEpiWarps;
-    static constexpr int kCW = BN * 4 / kEpiWarps;  // columns per epilogue thread
-    static constexpr int kNacc = (512 / BN) < 8 ? (512 / BN) : 8;
+    static constexpr int kNacc = (512 / BN) < kMaxNacc ? (512 / BN) : kMaxNacc;
     static constexpr int kTmemCols = (kNacc * BN) <= 32 ? 32 : (kNacc * BN) <= 64 ? 64 : (kNacc * BN) <= 128 ? 128
                                      : (kNacc * BN) <= 256 ? 256 : 512;
 };
 
 struct SmemTail {
-    uint64_t full[8];
-    uint64_t empty[8];
-    uint64_t acc_full[8];
-    uint64_t acc_empty[8];
+    uint64_t full[kMaxStages];
+    uint64_t empty[kMaxStages];
+    uint64_t acc_full[kMaxNacc];
+    uint64_t acc_empty[kMaxNacc];
     uint64_t done;
     uint32_t tmem_base;
     int abort_flag;
+};
+
+// Ring position with phase bit.
+struct Ring {
+    int idx;
+    uint32_t phase;
+    __device__ __forceinline__ void next(int n) {
+        if (++idx == n) {
+            idx = 0;
+            phase ^= 1u;
+        }
+    }
 };
 
 // Warp-uniform bounded wait: every lane polls, the loop exits for all lanes together.
@@ -77,35 +99,49 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volati
     }
 }
 
-__device__ __forceinline__ void decode_unit(const GemmArgs& p, int unit, int& tc, int& mb, int& nb) {
-    nb = unit % p.num_nb;
-    const int r = unit / p.num_nb;
-    mb = r % p.num_mb;
-    tc = r / p.num_mb;
-}
+// Units are numbered with the column block fastest, then the row block, then the tap chunk.
+struct UnitIter {
+    int unit, nb, mb, tc;
+    __device__ __forceinline__ void init(int first, const GemmArgs& p) {
+        unit = first;
+        nb = first % p.num_nb;
+        const int r = first / p.num_nb;
+        mb = r % p.num_mb;
+        tc = r / p.num_mb;
+    }
+    __device__ __forceinline__ void advance(int step, const GemmArgs& p) { init(unit + step, p); }
+};
 
 template <int BN, int MODE, bool DUMP>
 __global__ void __launch_bounds__(TcCfg<BN>::kThreads, 1)
-    hadamard_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, GemmArgs p) {
+    hadamard_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                       const __grid_constant__ CUtensorMap tmSV, const __grid_constant__ CUtensorMap tmSU, GemmArgs p) {
     using Cfg = TcCfg<BN>;
-    constexpr int CW = Cfg::kCW;
     constexpr int NACC = Cfg::kNacc;
     extern __shared__ __align__(1024) unsigned char smem_raw[];
-    // 1024-byte alignment for the swizzled stage buffers
+    // 1024-byte alignment for the swizzled tiles
     unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    const int BK = p.BK;
-    const int S = p.stages;
-    const uint32_t a_bytes = kBM * BK, b_bytes = BN * BK;
+    const int BK = p.BK;                   // swizzle width = bytes of K per tile row
+    const int KC = p.SK / BK;              // K chunks per stage
+    const int TPS = p.tps;                 // taps per stage
+    const int GPS = p.SK / p.G;            // K-groups per tap per stage
+    const int KSTAGES = p.Cin / p.SK;      // stages per tap
+    const uint32_t a_tile = kBM * BK, b_tile = BN * BK;
+    const uint32_t a_bytes = a_tile * KC * TPS, b_bytes = b_tile * KC * TPS;
     const uint32_t stage_bytes = a_bytes + b_bytes;
-    SmemTail* tail = reinterpret_cast<SmemTail*>(smem + (size_t)S * stage_bytes);
+    const int S = p.stages;
+    float* sv_ring = reinterpret_cast<float*>(smem + (size_t)S * stage_bytes);   // [S][TPS][GPS][128]
+    float* su_ring = sv_ring + (size_t)S * TPS * GPS * kBM;                      // [S][TPS][GPS][BN]
+    SmemTail* tail = reinterpret_cast<SmemTail*>(su_ring + (size_t)S * TPS * GPS * BN);
     volatile int* abort_flag = &tail->abort_flag;
+    const uint32_t scale_bytes = (uint32_t)TPS * GPS * (kBM + BN) * 4;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
     if (warp == 0 && lane == 0) {
         for (int s = 0; s < S; ++s) {
             mbar_init(&tail->full[s], 1);
-            mbar_init(&tail->empty[s], 1);
+            mbar_init(&tail->empty[s], 1 + Cfg::kEpiWarps);   // the MMA commit and every epilogue warp
         }
         for (int b = 0; b < NACC; ++b) {
             mbar_init(&tail->acc_full[b], 1);
@@ -117,6 +153,8 @@ __global__ void __launch_bounds__(TcCfg<BN>::kThreads, 1)
         fence_proxy_async_smem();
         prefetch_tensormap(&tmA);
         prefetch_tensormap(&tmB);
+        prefetch_tensormap(&tmSV);
+        prefetch_tensormap(&tmSU);
     }
     if (warp == 1) {
         tmem_alloc(&tail->tmem_base, Cfg::kTmemCols);
@@ -126,80 +164,92 @@ __global__ void __launch_bounds__(TcCfg<BN>::kThreads, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = tail->tmem_base;
-    const int ksteps = p.Cin / 32;        // K-steps of 32 bytes per tap
-    const int ks_per_stage = BK / 32;
-    const int ks_per_group = p.G / 32;
 
     if (warp == 0) {
         // ------------------------------------------------------- TMA producer
         if (lane == 0) {
-            uint32_t kc = 0;
+            Ring st{0, 0};
+            uint32_t issued = 0;
             bool ok = true;
-            for (int unit = blockIdx.x; ok && unit < p.num_units; unit += gridDim.x) {
-                int tc, mb, nb;
-                decode_unit(p, unit, tc, mb, nb);
-                const int tap_end = min(p.n2, (tc + 1) * p.tpu);
-                for (int tap = tc * p.tpu; ok && tap < tap_end; ++tap)
-                    for (int kb = 0; kb < p.Cin / BK; ++kb) {
-                        const int s = kc % S;
-                        if (!mbar_wait(&tail->empty[s], ((kc / S) & 1) ^ 1, abort_flag, p.err)) {
+            UnitIter u;
+            for (u.init(blockIdx.x, p); ok && u.unit < p.num_units; u.advance(gridDim.x, p)) {
+                const int tap_end = min(p.n2, (u.tc + 1) * p.tpu);
+                for (int tap0 = u.tc * p.tpu; ok && tap0 < tap_end; tap0 += TPS)
+                    for (int ks = 0; ks < KSTAGES; ++ks) {
+                        if (!mbar_wait(&tail->empty[st.idx], st.phase ^ 1u, abort_flag, p.err)) {
                             ok = false;
                             break;
                         }
-                        unsigned char* sa = smem + (size_t)s * stage_bytes;
-                        mbar_arrive_expect_tx(&tail->full[s], stage_bytes);
-                        tma_load_3d(sa, &tmA, &tail->full[s], kb * BK, tap, mb * kBM);
-                        tma_load_3d(sa + a_bytes, &tmB, &tail->full[s], kb * BK, nb * BN, tap);
-                        ++kc;
+                        uint64_t* bar = &tail->full[st.idx];
+                        unsigned char* sa = smem + (size_t)st.idx * stage_bytes;
+                        mbar_arrive_expect_tx(bar, stage_bytes + scale_bytes);
+                        for (int c = 0; c < KC; ++c) {
+                            const int k0 = ks * p.SK + c * BK;
+                            tma_load_3d(sa + (size_t)c * TPS * a_tile, &tmA, bar, k0, u.mb * kBM, tap0);
+                            tma_load_3d(sa + a_bytes + (size_t)c * TPS * b_tile, &tmB, bar, k0, u.nb * BN, tap0);
+                        }
+                        tma_load_3d(sv_ring + (size_t)st.idx * TPS * GPS * kBM, &tmSV, bar, u.mb * kBM, ks * GPS, tap0);
+                        tma_load_3d(su_ring + (size_t)st.idx * TPS * GPS * BN, &tmSU, bar, u.nb * BN, ks * GPS, tap0);
+                        ++issued;
+                        st.next(S);
                     }
             }
             // drain: every issued load must land before the CTA can exit
-            const uint32_t first = kc > (uint32_t)S ? kc - S : 0;
-            for (uint32_t i = first; i < kc; ++i) mbar_wait_teardown(&tail->full[i % S], (i / S) & 1);
+            Ring dr{st.idx, st.phase};
+            for (uint32_t i = 0; i < issued && i < (uint32_t)S; ++i) {
+                if (dr.idx == 0) {
+                    dr.idx = S - 1;
+                    dr.phase ^= 1u;
+                } else {
+                    --dr.idx;
+                }
+                mbar_wait_teardown(&tail->full[dr.idx], dr.phase);
+            }
         }
     } else if (warp == 1) {
         // --------------------------------------------------------- MMA issuer
         if (lane == 0) {
             const uint32_t idesc = idesc_i8(kBM, BN);
-            uint32_t kc = 0, gc = 0;
-            int s = 0, b = 0;
+            const uint64_t a_desc0 = smem_desc_kmajor(smem_u32(smem), BK);
+            const uint64_t b_desc0 = smem_desc_kmajor(smem_u32(smem) + a_bytes, BK);
+            const int ks_per_group = p.G / 32;
+            const int ks_per_chunk = BK / 32;
+            Ring st{0, 0}, bf{0, 0};
             bool ok = true;
-            for (int unit = blockIdx.x; ok && unit < p.num_units; unit += gridDim.x) {
-                int tc, mb, nb;
-                decode_unit(p, unit, tc, mb, nb);
-                const int tap_end = min(p.n2, (tc + 1) * p.tpu);
-                for (int tap = tc * p.tpu; ok && tap < tap_end; ++tap)
-                    for (int ks = 0; ks < ksteps; ++ks) {
-                        const int kin = ks % ks_per_stage;
-                        const int gin = ks % ks_per_group;
-                        if (kin == 0) {
-                            s = kc % S;
-                            if (!mbar_wait(&tail->full[s], (kc / S) & 1, abort_flag, p.err)) {
-                                ok = false;
-                                break;
-                            }
-                            tc_fence_after();
+            UnitIter u;
+            for (u.init(blockIdx.x, p); ok && u.unit < p.num_units; u.advance(gridDim.x, p)) {
+                const int tap_end = min(p.n2, (u.tc + 1) * p.tpu);
+                for (int tap0 = u.tc * p.tpu; ok && tap0 < tap_end; tap0 += TPS)
+                    for (int ks = 0; ok && ks < KSTAGES; ++ks) {
+                        if (!mbar_wait(&tail->full[st.idx], st.phase, abort_flag, p.err)) {
+                            ok = false;
+                            break;
                         }
-                        if (gin == 0) {
-                            b = gc % NACC;
-                            if (!mbar_wait(&tail->acc_empty[b], (gc / NACC) & 1, abort_flag, p.err)) {
-                                ok = false;
-                                break;
-                            }
-                            tc_fence_after();
+                        tc_fence_after();
+                        const uint64_t stage_off = (uint64_t)((st.idx * stage_bytes) >> 4);
+                        for (int t = 0; ok && t < TPS; ++t) {
+                            int gk = 0;  // K-steps into the current group
+                            for (int c = 0; ok && c < KC; ++c)
+                                for (int kin = 0; kin < ks_per_chunk; ++kin) {
+                                    if (gk == 0) {
+                                        if (!mbar_wait(&tail->acc_empty[bf.idx], bf.phase, abort_flag, p.err)) {
+                                            ok = false;
+                                            break;
+                                        }
+                                        tc_fence_after();
+                                    }
+                                    const uint64_t koff = stage_off + (uint64_t)(((c * TPS + t) * a_tile + kin * 32) >> 4);
+                                    const uint64_t kofb = stage_off + (uint64_t)(((c * TPS + t) * b_tile + kin * 32) >> 4);
+                                    mma_i8(tmem_base + (uint32_t)(bf.idx * BN), a_desc0 + koff, b_desc0 + kofb, idesc, 1u);
+                                    if (++gk == ks_per_group) {
+                                        gk = 0;
+                                        mma_commit(&tail->acc_full[bf.idx]);
+                                        bf.next(NACC);
+                                    }
+                                }
                         }
-                        const uint32_t sa = smem_u32(smem + (size_t)s * stage_bytes) + kin * 32;
-                        const uint64_t adesc = smem_desc_kmajor(sa, BK);
-                        const uint64_t bdesc = smem_desc_kmajor(sa + a_bytes, BK);
-                        mma_i8(tmem_base + (uint32_t)(b * BN), adesc, bdesc, idesc, 1u);
-                        if (gin == ks_per_group - 1) {
-                            mma_commit(&tail->acc_full[b]);
-                            ++gc;
-                        }
-                        if (kin == ks_per_stage - 1) {
-                            mma_commit(&tail->empty[s]);
-                            ++kc;
-                        }
+                        mma_commit(&tail->empty[st.idx]);
+                        st.next(S);
                     }
             }
             // all issued MMAs complete before TMEM is released
@@ -210,120 +260,135 @@ __global__ void __launch_bounds__(TcCfg<BN>::kThreads, 1)
         // ----------------------------------------------------------- epilogue
         const int ew = warp - 2;
         const int quad = warp & 3;                    // TMEM lanes 32*quad .. 32*quad+31
-        const int col0 = (ew / 4) * CW;               // this thread's column chunk in the BN block
-        static_assert(CW == 32, "one 32-column TMEM chunk per epilogue thread");
-        const uint32_t t_lane = tmem_base + ((uint32_t)(32 * quad) << 16);
-        constexpr int kChunks = CW / 32;              // 32-column chunks; G >= 32, so each lies in one group
+        const int col0 = (ew / 4) * 32;               // this thread's 32 columns in the BN block
+        const int rloc = 32 * quad + lane;            // row within the 128-tile block
+        const uint32_t t_lane = tmem_base + ((uint32_t)(32 * quad) << 16) + (uint32_t)col0;
+        const uint64_t neg_magic2 = f2_pack(-kRoundMagic, -kRoundMagic);
+        const int gst = TPS * GPS;                    // groups per stage
 
         // every accumulator buffer starts filled with the bias
-        for (int b = 0; b < NACC; ++b)
-#pragma unroll
-            for (int cc = 0; cc < CW / 32; ++cc) tmem_st32_fill(t_lane + b * BN + col0 + 32 * cc, (uint32_t)kRoundMagicBits);
+        for (int b = 0; b < NACC; ++b) tmem_st32_fill(t_lane + b * BN, (uint32_t)kRoundMagicBits);
         tmem_st_wait();
         tc_fence_before();
         __syncwarp();
         if (lane == 0)
             for (int b = 0; b < NACC; ++b) mbar_arrive(&tail->acc_empty[b]);
 
-        uint32_t gc = 0;
+        Ring st{0, 0}, bf{0, 0};
         bool ok = true;
-        for (int unit = blockIdx.x; ok && unit < p.num_units; unit += gridDim.x) {
-            int tc, mb, nb;
-            decode_unit(p, unit, tc, mb, nb);
-            const int row = mb * kBM + 32 * quad + lane;
+        UnitIter u;
+        for (u.init(blockIdx.x, p); ok && u.unit < p.num_units; u.advance(gridDim.x, p)) {
+            const int row = u.mb * kBM + rloc;
             const bool valid = row < p.T;
-            const int colg = nb * BN + col0;
-            float gmax[kChunks], sy[kChunks];
-#pragma unroll
-            for (int k = 0; k < kChunks; ++k) {
-                gmax[k] = 0.0f;
-                sy[k] = 0.0f;
-                if (MODE == kModeQuant && valid)
-                    sy[k] = group_scale(__uint_as_float(p.amax[(size_t)row * p.ngo + (colg + 32 * k) / p.G]));
-            }
-            const int tap_end = min(p.n2, (tc + 1) * p.tpu);
-            for (int tap = tc * p.tpu; ok && tap < tap_end; ++tap) {
-                float y[CW];
-#pragma unroll
-                for (int c = 0; c < CW; ++c) y[c] = 0.0f;
-                for (int j = 0; j < p.ng; ++j) {
-                    const int b = gc % NACC;
-                    const float sv = p.sV[((size_t)tap * p.ng + j) * p.T_pad + row];
-                    const float* su = p.sU + ((size_t)tap * p.ng + j) * p.Cout + colg;
-                    if (!warp_wait(&tail->acc_full[b], (gc / NACC) & 1, abort_flag, p.err)) {
+            const int colg = u.nb * BN + col0;
+            const int cgrp = colg / p.G;              // this thread's 32 columns lie in one Y group
+            float gmax = 0.0f;
+            QScale qy;
+            qy.s = 0.0f;
+            qy.rd = 0.0;
+            if (MODE == kModeQuant && valid) qy = make_qscale(__uint_as_float(p.amax[(size_t)row * p.ngo + cgrp]));
+            const int tap_end = min(p.n2, (u.tc + 1) * p.tpu);
+            uint64_t y2[16];
+            for (int tap0 = u.tc * p.tpu; ok && tap0 < tap_end; tap0 += TPS)
+                for (int ks = 0; ok && ks < KSTAGES; ++ks) {
+                    // the stage's scales and the last of its groups' accumulators
+                    Ring last = bf;
+                    for (int i = 1; i < gst; ++i) last.next(NACC);
+                    if (!warp_wait(&tail->full[st.idx], st.phase, abort_flag, p.err) ||
+                        !warp_wait(&tail->acc_full[last.idx], last.phase, abort_flag, p.err)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
+                    const float* svs = sv_ring + (size_t)st.idx * TPS * GPS * kBM;
+                    const float* sus = su_ring + (size_t)st.idx * TPS * GPS * BN;
+                    Ring b = bf;
+                    for (int t = 0; t < TPS; ++t) {
+                        const int tap = tap0 + t;
+                        if (ks == 0) {
 #pragma unroll
-                    for (int cc = 0; cc < kChunks; ++cc) {
-                        uint32_t r[32];
-                        tmem_ld32(t_lane + b * BN + col0 + 32 * cc, r);
-                        tmem_ld_wait();
-#pragma unroll
-                        for (int c4 = 0; c4 < 32; c4 += 4) {
-                            const int c = 32 * cc + c4;
-                            const float4 u = __ldg(reinterpret_cast<const float4*>(su + c));
-                            y[c + 0] = __fmaf_rn(__fsub_rn(__uint_as_float(r[c4 + 0]), kRoundMagic), __fmul_rn(sv, u.x), y[c + 0]);
-                            y[c + 1] = __fmaf_rn(__fsub_rn(__uint_as_float(r[c4 + 1]), kRoundMagic), __fmul_rn(sv, u.y), y[c + 1]);
-                            y[c + 2] = __fmaf_rn(__fsub_rn(__uint_as_float(r[c4 + 2]), kRoundMagic), __fmul_rn(sv, u.z), y[c + 2]);
-                            y[c + 3] = __fmaf_rn(__fsub_rn(__uint_as_float(r[c4 + 3]), kRoundMagic), __fmul_rn(sv, u.w), y[c + 3]);
+                            for (int c = 0; c < 16; ++c) y2[c] = 0ull;
                         }
-                        if (DUMP && valid) {
+                        for (int j = 0; j < GPS; ++j) {
+                            uint32_t r[32];
+                            tmem_ld32(t_lane + b.idx * BN, r);
+                            tmem_ld_wait();
+                            const float sv = svs[(t * GPS + j) * kBM + rloc];
+                            const uint64_t sv2 = f2_pack(sv, sv);
+                            const float4* su4 = reinterpret_cast<const float4*>(sus + (t * GPS + j) * BN + col0);
 #pragma unroll
-                            for (int c = 0; c < 32; ++c)
-                                p.acc[(((size_t)tap * p.T + row) * p.Cout + colg + 32 * cc + c) * p.ng + j] =
-                                    (int)r[c] - kRoundMagicBits;
+                            for (int c4 = 0; c4 < 8; ++c4) {
+                                const float4 uu = su4[c4];
+                                const uint64_t a0 =
+                                    f2_add(f2_pack(__uint_as_float(r[4 * c4 + 0]), __uint_as_float(r[4 * c4 + 1])), neg_magic2);
+                                const uint64_t a1 =
+                                    f2_add(f2_pack(__uint_as_float(r[4 * c4 + 2]), __uint_as_float(r[4 * c4 + 3])), neg_magic2);
+                                y2[2 * c4 + 0] = f2_fma(a0, f2_mul(sv2, f2_pack(uu.x, uu.y)), y2[2 * c4 + 0]);
+                                y2[2 * c4 + 1] = f2_fma(a1, f2_mul(sv2, f2_pack(uu.z, uu.w)), y2[2 * c4 + 1]);
+                            }
+                            if (DUMP && valid) {
+                                const int jg = ks * GPS + j;
+#pragma unroll
+                                for (int c = 0; c < 32; ++c)
+                                    p.acc[(((size_t)tap * p.T + row) * p.Cout + colg + c) * p.ng + jg] =
+                                        (int)r[c] - kRoundMagicBits;
+                            }
+                            b.next(NACC);
+                        }
+                        if (ks + 1 < KSTAGES) continue;
+                        // ---- end of tap
+                        float y[32];
+#pragma unroll
+                        for (int c = 0; c < 16; ++c) f2_unpack(y2[c], y[2 * c], y[2 * c + 1]);
+                        if (MODE == kModeQuant) {
+                            if (valid) {
+                                int8_t* dst = p.Yq + ((size_t)tap * p.T + row) * p.Cout + colg;
+#pragma unroll
+                                for (int c = 0; c < 32; c += 16) {
+                                    uint32_t w[4];
+#pragma unroll
+                                    for (int e = 0; e < 4; ++e) {
+                                        uint32_t pk = 0;
+#pragma unroll
+                                        for (int bb = 0; bb < 4; ++bb)
+                                            pk |= ((uint32_t)(quant_code_fast(y[c + 4 * e + bb], qy) & 0xff)) << (8 * bb);
+                                        w[e] = pk;
+                                    }
+                                    *reinterpret_cast<uint4*>(dst + c) = make_uint4(w[0], w[1], w[2], w[3]);
+                                }
+                            }
+                        } else {
+#pragma unroll
+                            for (int c = 0; c < 32; ++c) gmax = fmaxf(gmax, fabsf(y[c]));
+                            if (MODE == kModeY32 && valid) {
+                                float* dst = p.Y32 + ((size_t)tap * p.T + row) * p.Cout + colg;
+#pragma unroll
+                                for (int c = 0; c < 32; c += 4)
+                                    *reinterpret_cast<float4*>(dst + c) = make_float4(y[c], y[c + 1], y[c + 2], y[c + 3]);
+                            }
                         }
                     }
-                    // hand the buffer back, refilled with the bias
-#pragma unroll
-                    for (int cc = 0; cc < kChunks; ++cc)
-                        tmem_st32_fill(t_lane + b * BN + col0 + 32 * cc, (uint32_t)kRoundMagicBits);
+                    // refill this stage's buffers with the bias and release them and the stage
+                    b = bf;
+                    for (int i = 0; i < gst; ++i) {
+                        tmem_st32_fill(t_lane + b.idx * BN, (uint32_t)kRoundMagicBits);
+                        b.next(NACC);
+                    }
                     tmem_st_wait();
                     tc_fence_before();
                     __syncwarp();
-                    if (lane == 0) mbar_arrive(&tail->acc_empty[b]);
-                    ++gc;
-                }
-                if (!ok) break;
-                // end of tap
-                if (MODE == kModeQuant) {
-                    if (valid) {
-                        int8_t* dst = p.Yq + ((size_t)row * p.n2 + tap) * p.Cout + colg;
-#pragma unroll
-                        for (int c = 0; c < CW; c += 16) {
-                            uint32_t w[4];
-#pragma unroll
-                            for (int e = 0; e < 4; ++e) {
-                                uint32_t pk = 0;
-#pragma unroll
-                                for (int bb = 0; bb < 4; ++bb) {
-                                    const int cc = c + 4 * e + bb;
-                                    const int q = quant_code(y[cc], sy[cc / 32]);
-                                    pk |= ((uint32_t)(q & 0xff)) << (8 * bb);
-                                }
-                                w[e] = pk;
-                            }
-                            *reinterpret_cast<uint4*>(dst + c) = make_uint4(w[0], w[1], w[2], w[3]);
+                    if (lane == 0) {
+                        b = bf;
+                        for (int i = 0; i < gst; ++i) {
+                            mbar_arrive(&tail->acc_empty[b.idx]);
+                            b.next(NACC);
                         }
+                        mbar_arrive(&tail->empty[st.idx]);
                     }
-                } else {
-#pragma unroll
-                    for (int c = 0; c < CW; ++c) gmax[c / 32] = fmaxf(gmax[c / 32], fabsf(y[c]));
-                    if (MODE == kModeY32 && valid) {
-                        float* dst = p.Y32 + ((size_t)row * p.n2 + tap) * p.Cout + colg;
-#pragma unroll
-                        for (int c = 0; c < CW; c += 4)
-                            *reinterpret_cast<float4*>(dst + c) = make_float4(y[c], y[c + 1], y[c + 2], y[c + 3]);
-                    }
+                    bf = b;
+                    st.next(S);
                 }
-            }
-            if (ok && MODE != kModeQuant && valid) {
-#pragma unroll
-                for (int k = 0; k < kChunks; ++k)
-                    atomicMax(&p.amax[(size_t)row * p.ngo + (colg + 32 * k) / p.G], __float_as_uint(gmax[k]));
-            }
+            if (ok && MODE != kModeQuant && valid) atomicMax(&p.amax[(size_t)row * p.ngo + cgrp], __float_as_uint(gmax));
         }
     }
 
@@ -357,39 +422,80 @@ CUtensorMapSwizzle swizzle_for(int bk) {
     return bk == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : (bk == 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B);
 }
 
+struct Maps {
+    CUtensorMap a, b, sv, su;
+};
+
+size_t smem_bytes(const GemmArgs& a, int BN) {
+    const size_t per_stage = (size_t)a.tps * a.SK * (kBM + BN) + (size_t)a.tps * (a.SK / a.G) * (kBM + BN) * 4;
+    return 1024 + (size_t)a.stages * per_stage + sizeof(SmemTail);
+}
+
 template <int BN, int MODE, bool DUMP>
-cudaError_t launch_cfg(const GemmArgs& a, const CUtensorMap& ta, const CUtensorMap& tb, int num_sms, cudaStream_t st) {
+cudaError_t launch_cfg(const GemmArgs& a, const Maps& m, int num_sms, cudaStream_t st) {
     using Cfg = TcCfg<BN>;
     // at least half the SM's shared memory, so one CTA owns the SM and its TMEM
-    const size_t smem = std::max<size_t>(1024 + (size_t)a.stages * (kBM + BN) * a.BK + sizeof(SmemTail), 116 * 1024);
+    const size_t smem = std::max<size_t>(smem_bytes(a, BN), 116 * 1024);
     auto kern = hadamard_tc_kernel<BN, MODE, DUMP>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     const int grid = a.num_units < num_sms ? a.num_units : num_sms;
-    kern<<<grid, Cfg::kThreads, smem, st>>>(ta, tb, a);
+    kern<<<grid, Cfg::kThreads, smem, st>>>(m.a, m.b, m.sv, m.su, a);
     return cudaGetLastError();
 }
 
 template <int BN>
-cudaError_t launch_bn(const GemmArgs& a, const CUtensorMap& ta, const CUtensorMap& tb, int mode, int num_sms,
-                      cudaStream_t st) {
+cudaError_t launch_bn(const GemmArgs& a, const Maps& m, int mode, int num_sms, cudaStream_t st) {
     const bool dump = a.acc != nullptr && mode != kModeQuant;
     if (mode == kModeAbsmax)
-        return dump ? launch_cfg<BN, kModeAbsmax, true>(a, ta, tb, num_sms, st)
-                    : launch_cfg<BN, kModeAbsmax, false>(a, ta, tb, num_sms, st);
-    if (mode == kModeQuant) return launch_cfg<BN, kModeQuant, false>(a, ta, tb, num_sms, st);
-    return dump ? launch_cfg<BN, kModeY32, true>(a, ta, tb, num_sms, st)
-                : launch_cfg<BN, kModeY32, false>(a, ta, tb, num_sms, st);
+        return dump ? launch_cfg<BN, kModeAbsmax, true>(a, m, num_sms, st)
+                    : launch_cfg<BN, kModeAbsmax, false>(a, m, num_sms, st);
+    if (mode == kModeQuant) return launch_cfg<BN, kModeQuant, false>(a, m, num_sms, st);
+    return dump ? launch_cfg<BN, kModeY32, true>(a, m, num_sms, st) : launch_cfg<BN, kModeY32, false>(a, m, num_sms, st);
+}
+
+bool encode(EncodeTiledFn enc, CUtensorMap* map, CUtensorMapDataType dt, const void* base, const cuuint64_t* dims,
+            const cuuint64_t* strides, const cuuint32_t* box, CUtensorMapSwizzle sw) {
+    const cuuint32_t es[3] = {1u, 1u, 1u};
+    return enc(map, dt, 3u, const_cast<void*>(base), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 }  // namespace
 
 int tc_block_n(int Cout, int G) {
-    if (Cout % 128 == 0 && 128 % G == 0) return 128;
-    if (Cout % 128 == 0 && G == 256) return 128;
+    if (Cout % 128 == 0 && (128 % G == 0 || G == 256)) return 128;
     if (Cout % 64 == 0) return 64;
     if (Cout % 32 == 0 && G == 32) return 32;
     return 0;
+}
+
+// Stage shape: SK bytes of K (a multiple of G dividing Cin, at most NACC/2
+// groups), swizzle width BK dividing SK, and TPS taps when SK == Cin.
+static void choose_stage(GemmArgs& a, int BN) {
+    const int nacc = std::min(512 / BN, kMaxNacc);
+    const int max_groups = nacc / 2;
+    int sk = a.G;
+    for (int m = max_groups; m >= 1; --m)
+        if (a.Cin % (a.G * m) == 0 && a.G * m <= std::max(a.G, 256)) {
+            sk = a.G * m;
+            break;
+        }
+    a.SK = sk;
+    a.BK = sk % 128 == 0 ? 128 : (sk % 64 == 0 ? 64 : 32);
+    const int gps = sk / a.G;
+    a.tps = 1;
+    if (sk == a.Cin)
+        for (int t : {4, 2})
+            if (t * gps <= max_groups && a.n2 % t == 0) {
+                a.tps = t;
+                break;
+            }
+    const size_t per_stage = (size_t)a.tps * sk * (kBM + BN) + (size_t)a.tps * gps * (kBM + BN) * 4;
+    while (a.tps > 1 && (200 * 1024) / per_stage < 3) a.tps /= 2;
+    const size_t ps = (size_t)a.tps * sk * (kBM + BN) + (size_t)a.tps * gps * (kBM + BN) * 4;
+    const int stages = (int)((200 * 1024) / ps);
+    a.stages = stages > kMaxStages ? kMaxStages : (stages < 2 ? 2 : stages);
 }
 
 cudaError_t launch_hadamard_tc(GemmArgs a, const int8_t* Vq, const int8_t* Uq, int mode, int num_sms,
@@ -398,45 +504,52 @@ cudaError_t launch_hadamard_tc(GemmArgs a, const int8_t* Vq, const int8_t* Uq, i
     if (BN == 0) return cudaErrorInvalidValue;
     EncodeTiledFn enc = get_encode_fn();
     if (!enc) return cudaErrorNotSupported;
-    a.BK = a.Cin % 128 == 0 ? 128 : (a.Cin % 64 == 0 ? 64 : 32);
-    const size_t stage_bytes = (size_t)(kBM + BN) * a.BK;
-    int stages = (int)((200 * 1024) / stage_bytes);
-    a.stages = stages > 8 ? 8 : (stages < 2 ? 2 : stages);
+    choose_stage(a, BN);
     a.num_mb = (a.T + kBM - 1) / kBM;
     a.num_nb = a.Cout / BN;
-    // tap chunking: enough units to fill the SMs a few times over
+    // tap chunking: enough units to fill the SMs a few times over; chunks are whole stages of taps
     const int base = a.num_mb * a.num_nb;
     int tpu = a.n2;
-    while (tpu > 1 && (long)base * ((a.n2 + tpu - 1) / tpu) < 4L * num_sms) tpu = (tpu + 1) / 2;
+    while (tpu > a.tps && (tpu / 2) % a.tps == 0 && (long)base * ((a.n2 + tpu - 1) / tpu) < 4L * num_sms)
+        tpu /= 2;
+    if (tpu % a.tps) tpu = a.tps;
     a.tpu = tpu;
     a.num_tc = (a.n2 + tpu - 1) / tpu;
     a.num_units = base * a.num_tc;
 
-    CUtensorMap ta, tb;
-    {
-        cuuint64_t dims[3] = {(cuuint64_t)a.Cin, (cuuint64_t)a.n2, (cuuint64_t)a.T_pad};
-        cuuint64_t strides[2] = {(cuuint64_t)a.Cin, (cuuint64_t)a.n2 * a.Cin};
-        cuuint32_t box[3] = {(cuuint32_t)a.BK, 1u, (cuuint32_t)kBM};
-        cuuint32_t es[3] = {1u, 1u, 1u};
-        if (enc(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<int8_t*>(Vq), dims, strides, box, es,
-                CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle_for(a.BK), CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    Maps m;
+    const CUtensorMapSwizzle sw = swizzle_for(a.BK);
+    const int gps = a.SK / a.G;
+    {   // Vq [n2][T_pad][Cin] int8, box BK x 128 x TPS
+        const cuuint64_t dims[3] = {(cuuint64_t)a.Cin, (cuuint64_t)a.T_pad, (cuuint64_t)a.n2};
+        const cuuint64_t strides[2] = {(cuuint64_t)a.Cin, (cuuint64_t)a.T_pad * a.Cin};
+        const cuuint32_t box[3] = {(cuuint32_t)a.BK, (cuuint32_t)kBM, (cuuint32_t)a.tps};
+        if (!encode(enc, &m.a, CU_TENSOR_MAP_DATA_TYPE_UINT8, Vq, dims, strides, box, sw)) return cudaErrorInvalidValue;
+    }
+    {   // Uq [n2][Cout][Cin] int8, box BK x BN x TPS
+        const cuuint64_t dims[3] = {(cuuint64_t)a.Cin, (cuuint64_t)a.Cout, (cuuint64_t)a.n2};
+        const cuuint64_t strides[2] = {(cuuint64_t)a.Cin, (cuuint64_t)a.Cout * a.Cin};
+        const cuuint32_t box[3] = {(cuuint32_t)a.BK, (cuuint32_t)BN, (cuuint32_t)a.tps};
+        if (!encode(enc, &m.b, CU_TENSOR_MAP_DATA_TYPE_UINT8, Uq, dims, strides, box, sw)) return cudaErrorInvalidValue;
+    }
+    {   // sV [n2][ng][T_pad] fp32, box 128 x gps x TPS
+        const cuuint64_t dims[3] = {(cuuint64_t)a.T_pad, (cuuint64_t)a.ng, (cuuint64_t)a.n2};
+        const cuuint64_t strides[2] = {(cuuint64_t)a.T_pad * 4, (cuuint64_t)a.ng * a.T_pad * 4};
+        const cuuint32_t box[3] = {(cuuint32_t)kBM, (cuuint32_t)gps, (cuuint32_t)a.tps};
+        if (!encode(enc, &m.sv, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, a.sV, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_NONE))
             return cudaErrorInvalidValue;
     }
-    {
-        cuuint64_t dims[3] = {(cuuint64_t)a.Cin, (cuuint64_t)a.Cout, (cuuint64_t)a.n2};
-        cuuint64_t strides[2] = {(cuuint64_t)a.Cin, (cuuint64_t)a.Cout * a.Cin};
-        cuuint32_t box[3] = {(cuuint32_t)a.BK, (cuuint32_t)BN, 1u};
-        cuuint32_t es[3] = {1u, 1u, 1u};
-        if (enc(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<int8_t*>(Uq), dims, strides, box, es,
-                CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle_for(a.BK), CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    {   // sU [n2][ng][Cout] fp32, box BN x gps x TPS
+        const cuuint64_t dims[3] = {(cuuint64_t)a.Cout, (cuuint64_t)a.ng, (cuuint64_t)a.n2};
+        const cuuint64_t strides[2] = {(cuuint64_t)a.Cout * 4, (cuuint64_t)a.ng * a.Cout * 4};
+        const cuuint32_t box[3] = {(cuuint32_t)BN, (cuuint32_t)gps, (cuuint32_t)a.tps};
+        if (!encode(enc, &m.su, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, a.sU, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_NONE))
             return cudaErrorInvalidValue;
     }
     if (launches) ++*launches;
-    if (BN == 128) return launch_bn<128>(a, ta, tb, mode, num_sms, st);
-    if (BN == 64) return launch_bn<64>(a, ta, tb, mode, num_sms, st);
-    return launch_bn<32>(a, ta, tb, mode, num_sms, st);
+    if (BN == 128) return launch_bn<128>(a, m, mode, num_sms, st);
+    if (BN == 64) return launch_bn<64>(a, m, mode, num_sms, st);
+    return launch_bn<32>(a, m, mode, num_sms, st);
 }
 
 }  // namespace wino

@@ -10,12 +10,16 @@
 //   exact-zero coefficients are skipped, which can change only the sign of a zero).
 // Q then runs over G consecutive channels at fixed (tile, tap).
 //
-// CTA: TX consecutive tiles of one tile row x CC channels; one thread per
-// (tile, channel), lanes along channels.  The halo patch is staged in shared
-// memory with 16-byte loads; the per-(tile, tap) absmax of a 32-channel warp
-// is a recursive-halving shuffle reduction (each lane ends with two taps),
-// combined across the G/32 warps of a group in shared memory; the int8 codes
-// are staged in shared memory and written with 16-byte stores.
+// CTA: TX consecutive tiles of one tile row x one quantisation group of G
+// channels (128 threads, 256 for G = 256); one thread per (tile, channel),
+// lanes along channels, so each warp-wide load of a pixel is contiguous.  The
+// n x n patch is read straight from global memory (neighbouring tiles share
+// two columns, which the L1 absorbs) and transformed in registers.  V then
+// goes to shared memory (rows padded to 33 words), where lane l of the warp
+// owns taps l and l + 32: it takes their absmax over the warp's 32 channels
+// (the G/32 warps of a group combine theirs in shared memory), the group
+// scale, and the 32 codes of each of its taps, packed into two 16-byte stores
+// of the tap-major Vq.
 #include "kernels.h"
 
 namespace wino {
@@ -25,156 +29,159 @@ template <typename T>
 __device__ __forceinline__ float load_as_float(const T* p);
 template <>
 __device__ __forceinline__ float load_as_float<float>(const float* p) {
-    return *p;
+    return __ldg(p);
 }
 template <>
 __device__ __forceinline__ float load_as_float<uint16_t>(const uint16_t* p) {
-    return bf16_bits_to_float(*p);
+    return bf16_bits_to_float(__ldg(reinterpret_cast<const unsigned short*>(p)));
 }
 
-template <int M, uint64_t MASK, typename Tin, int CC, int TX>
-__global__ void __launch_bounds__(CC* TX) input_transform_kernel(InputArgs p, TransformArgs tf) {
-    constexpr int N = M + 2, N2 = N * N, PW = TX * M + 2;
-    constexpr int VEC = 16 / sizeof(Tin);
-    constexpr int WPT = CC / 32;  // warps per tile
-    extern __shared__ __align__(16) unsigned char smem[];
-    Tin* patch = reinterpret_cast<Tin*>(smem);                                 // [N][PW][CC]
-    float* red = reinterpret_cast<float*>(smem + sizeof(Tin) * N * PW * CC);   // [TX*WPT][64]
-    float* scl = red + TX * WPT * 64;                                          // [TX*WPT][64] (per group leader)
-    int8_t* outb = reinterpret_cast<int8_t*>(scl + TX * WPT * 64);             // [TX][N2][CC]
+template <int M>
+struct InCfg {
+    static constexpr int N = M + 2, N2 = N * N;
+    static constexpr int kPitch = 33;  // words per V row in shared memory
+};
+
+template <int M, uint64_t MASK, typename Tin, int G, int TX>
+__global__ void __launch_bounds__(G* TX) input_transform_kernel(InputArgs p, TransformArgs tf) {
+    constexpr int N = M + 2, N2 = N * N;
+    constexpr int WPT = G / 32;      // warps per tile (= per group)
+    constexpr int NW = TX * WPT;     // warps per CTA
+    constexpr int P = InCfg<M>::kPitch;
+    extern __shared__ float vbuf[];  // [NW][N2][P]
+    __shared__ float red[NW][64];
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int row_id = blockIdx.y;  // img * TH + ty
     const int img = row_id / p.TH, ty = row_id - img * p.TH;
-    const int tx0 = blockIdx.x * TX;
-    const int c0 = blockIdx.z * CC;
+    const int tl = warp / WPT;
+    const int tx = blockIdx.x * TX + tl;
+    const bool valid = tx < p.TW;
+    const int g = blockIdx.z;
+    const int cw = g * G + (warp % WPT) * 32;  // first channel of this warp
+    const long t = (long)row_id * p.TW + tx;
     const Tin* x = reinterpret_cast<const Tin*>(p.x);
 
-    if (blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0 && tid == 0) *p.err = 0;
-    if (blockIdx.z == 0) {
+    if (blockIdx.x == 0 && blockIdx.y == 0 && g == 0 && tid == 0) *p.err = 0;
+    if (g == 0)
         for (int i = tid; i < TX * p.ngo; i += blockDim.x) {
-            const int tl = i / p.ngo, k = i - tl * p.ngo;
-            if (tx0 + tl < p.TW) p.amax[((size_t)row_id * p.TW + tx0 + tl) * p.ngo + k] = 0u;
+            const int tt = i / p.ngo, k = i - tt * p.ngo;
+            if (blockIdx.x * TX + tt < p.TW) p.amax[((size_t)row_id * p.TW + blockIdx.x * TX + tt) * p.ngo + k] = 0u;
         }
-    }
 
-    // 1. halo patch -> shared memory (zeros outside the image)
-    for (int v = tid; v < N * PW * (CC / VEC); v += blockDim.x) {
-        const int cv = v % (CC / VEC);
-        const int rest = v / (CC / VEC);
-        const int col = rest % PW, r = rest / PW;
-        const int yy = ty * M - 1 + r, xx = tx0 * M - 1 + col;
-        uint4 val = make_uint4(0u, 0u, 0u, 0u);
-        if (yy >= 0 && yy < p.H && xx >= 0 && xx < p.W)
-            val = *reinterpret_cast<const uint4*>(x + (((size_t)img * p.H + yy) * p.W + xx) * p.Cin + c0 + cv * VEC);
-        *reinterpret_cast<uint4*>(patch + ((size_t)(r * PW + col) * CC + cv * VEC)) = val;
-    }
-    __syncthreads();
-
-    // 2. transform for (tile tl, channel cl)
-    const int tl = warp / WPT;
-    const int cl = (warp % WPT) * 32 + lane;
-    float v[N][N];
+    {
+        // 1. the n x n patch of channel cw + lane (zeros outside the image)
+        float v[N][N];
 #pragma unroll
-    for (int r = 0; r < N; ++r)
+        for (int r = 0; r < N; ++r) {
+            const int yy = ty * M - 1 + r;
+            const bool row_in = valid && yy >= 0 && yy < p.H;
+            const Tin* xr = x + ((size_t)img * p.H + (row_in ? yy : 0)) * p.W * p.Cin + cw + lane;
 #pragma unroll
-        for (int l = 0; l < N; ++l) v[r][l] = load_as_float<Tin>(patch + (size_t)(r * PW + tl * M + l) * CC + cl);
+            for (int l = 0; l < N; ++l) {
+                const int xx = tx * M - 1 + l;
+                v[r][l] = (row_in && xx >= 0 && xx < p.W) ? load_as_float<Tin>(xr + (size_t)xx * p.Cin) : 0.0f;
+            }
+        }
+        // 2. V = B^T d B
 #pragma unroll
-    for (int l = 0; l < N; ++l) {
-        float t[N];
+        for (int l = 0; l < N; ++l) {
+            float tcol[N];
+#pragma unroll
+            for (int i = 0; i < N; ++i) {
+                float acc = 0.0f;
+#pragma unroll
+                for (int k = 0; k < N; ++k)
+                    if ((MASK >> (i * N + k)) & 1ull) acc = __fmaf_rn(tf.BT[i * N + k], v[k][l], acc);
+                tcol[i] = acc;
+            }
+#pragma unroll
+            for (int i = 0; i < N; ++i) v[i][l] = tcol[i];
+        }
+        float* vw = vbuf + (size_t)warp * N2 * P;
 #pragma unroll
         for (int i = 0; i < N; ++i) {
-            float acc = 0.0f;
 #pragma unroll
-            for (int k = 0; k < N; ++k)
-                if ((MASK >> (i * N + k)) & 1ull) acc = __fmaf_rn(tf.BT[i * N + k], v[k][l], acc);
-            t[i] = acc;
+            for (int j = 0; j < N; ++j) {
+                float acc = 0.0f;
+#pragma unroll
+                for (int l = 0; l < N; ++l)
+                    if ((MASK >> (j * N + l)) & 1ull) acc = __fmaf_rn(v[i][l], tf.BT[j * N + l], acc);
+                vw[(i * N + j) * P + lane] = acc;   // 3. V row of tap (i, j), this lane's channel
+            }
         }
-#pragma unroll
-        for (int i = 0; i < N; ++i) v[i][l] = t[i];
     }
+    __syncwarp();
+
+    // 4. absmax of this lane's taps over the warp's 32 channels
+    const float* vw = vbuf + (size_t)warp * N2 * P;
+    float am[2] = {0.0f, 0.0f};
 #pragma unroll
-    for (int i = 0; i < N; ++i) {
-        float t[N];
-#pragma unroll
-        for (int j = 0; j < N; ++j) {
-            float acc = 0.0f;
-#pragma unroll
-            for (int l = 0; l < N; ++l)
-                if ((MASK >> (j * N + l)) & 1ull) acc = __fmaf_rn(v[i][l], tf.BT[j * N + l], acc);
-            t[j] = acc;
+    for (int e = 0; e < 2; ++e) {
+        const int tap = lane + 32 * e;
+        if (tap < N2) {
+            float a = 0.0f;
+#pragma unroll 8
+            for (int j = 0; j < 32; ++j) a = fmaxf(a, fabsf(vw[tap * P + j]));
+            am[e] = a;
         }
-#pragma unroll
-        for (int j = 0; j < N; ++j) v[i][j] = t[j];
     }
-
-    // 3. per-(tile, tap) absmax over this warp's 32 channels
-    {
-        float a[64];
-#pragma unroll
-        for (int k = 0; k < 64; ++k) a[k] = k < N2 ? fabsf(v[k / N][k % N]) : 0.0f;
-        warp_max_scatter64(a, lane);
-        red[warp * 64 + 2 * lane] = a[0];
-        red[warp * 64 + 2 * lane + 1] = a[1];
-    }
-    __syncthreads();
-
-    // 4. group scales: the first warp of each group combines its G/32 warps
-    const int wpg = p.G / 32;
-    const int leader = warp - (warp % wpg);
-    const int ng = p.Cin / p.G;
-    const int tx = tx0 + tl;
-    const long t = (long)row_id * p.TW + tx;
-    if (warp == leader) {
-        const int g = (c0 + (warp % WPT) * 32) / p.G;
+    if (WPT > 1) {
+        red[warp][lane] = am[0];
+        red[warp][lane + 32] = am[1];
+        __syncthreads();
+        const int leader = warp - warp % WPT;
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
-            const int tap = 2 * lane + e;
-            float amax = 0.0f;
-            for (int i = 0; i < wpg; ++i) amax = fmaxf(amax, red[(warp + i) * 64 + tap]);
-            const float s = group_scale(amax);
-            scl[warp * 64 + tap] = s;
-            if (tap < N2 && tx < p.TW) p.sV[((size_t)tap * ng + g) * p.T_pad + t] = s;
+            float a = 0.0f;
+#pragma unroll
+            for (int i = 0; i < WPT; ++i) a = fmaxf(a, red[leader + i][lane + 32 * e]);
+            am[e] = a;
         }
     }
-    __syncthreads();
 
-    // 5. int8 codes -> shared staging
+    // 5. scales and codes of this lane's taps
+    if (valid) {
 #pragma unroll
-    for (int k = 0; k < N2; ++k)
-        outb[(tl * N2 + k) * CC + cl] = (int8_t)quant_code(v[k / N][k % N], scl[leader * 64 + k]);
-    __syncthreads();
-
-    // 6. 16-byte stores of Vq[t][tap][c0 .. c0+CC)
-    for (int i = tid; i < TX * N2 * (CC / 16); i += blockDim.x) {
-        const int cv = i % (CC / 16);
-        const int rest = i / (CC / 16);
-        const int tap = rest % N2, tl2 = rest / N2;
-        if (tx0 + tl2 >= p.TW) continue;
-        const size_t t2 = (size_t)row_id * p.TW + tx0 + tl2;
-        *reinterpret_cast<uint4*>(p.Vq + (t2 * N2 + tap) * p.Cin + c0 + cv * 16) =
-            *reinterpret_cast<const uint4*>(outb + (tl2 * N2 + tap) * CC + cv * 16);
+        for (int e = 0; e < 2; ++e) {
+            const int tap = lane + 32 * e;
+            if (tap >= N2) continue;
+            const QScale q = make_qscale(am[e]);
+            if (warp % WPT == 0) p.sV[((size_t)tap * (p.Cin / G) + g) * p.T_pad + t] = q.s;
+            uint32_t w[8];
+#pragma unroll
+            for (int j4 = 0; j4 < 8; ++j4) {
+                uint32_t pk = 0;
+#pragma unroll
+                for (int b = 0; b < 4; ++b)
+                    pk |= ((uint32_t)(quant_code_fast(vw[tap * P + 4 * j4 + b], q) & 0xff)) << (8 * b);
+                w[j4] = pk;
+            }
+            uint4* dst = reinterpret_cast<uint4*>(p.Vq + ((size_t)tap * p.T_pad + t) * p.Cin + cw);
+            dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
+            dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
+        }
     }
 }
 
-template <int M, uint64_t MASK, typename Tin, int CC, int TX>
-cudaError_t launch_one(const InputArgs& a, const TransformArgs& tf, cudaStream_t st) {
-    constexpr int N = M + 2, N2 = N * N, PW = TX * M + 2, WPT = CC / 32;
-    const size_t smem = sizeof(Tin) * N * PW * CC + 2 * sizeof(float) * TX * WPT * 64 + (size_t)TX * N2 * CC;
-    auto kern = input_transform_kernel<M, MASK, Tin, CC, TX>;
+template <int M, uint64_t MASK, typename Tin, int G>
+cudaError_t launch_g(const InputArgs& a, const TransformArgs& tf, cudaStream_t st) {
+    constexpr int TX = G >= 128 ? 1 : 128 / G;
+    constexpr int NW = TX * G / 32;
+    const size_t smem = sizeof(float) * NW * InCfg<M>::N2 * InCfg<M>::kPitch;
+    auto kern = input_transform_kernel<M, MASK, Tin, G, TX>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    dim3 grid((a.TW + TX - 1) / TX, a.N * a.TH, a.Cin / CC);
-    kern<<<grid, CC * TX, smem, st>>>(a, tf);
+    dim3 grid((a.TW + TX - 1) / TX, a.N * a.TH, a.Cin / G);
+    kern<<<grid, G * TX, smem, st>>>(a, tf);
     return cudaGetLastError();
 }
 
 template <int M, uint64_t MASK, typename Tin>
 cudaError_t launch_cc(const InputArgs& a, const TransformArgs& tf, cudaStream_t st) {
-    // channel chunk: a multiple of G dividing Cin; 256 threads per CTA
-    if (a.G == 256) return launch_one<M, MASK, Tin, 256, 1>(a, tf, st);
-    if (a.Cin % 64 == 0) return launch_one<M, MASK, Tin, 64, 4>(a, tf, st);
-    if (a.G == 32) return launch_one<M, MASK, Tin, 32, 8>(a, tf, st);
+    if (a.G == 32) return launch_g<M, MASK, Tin, 32>(a, tf, st);
+    if (a.G == 64) return launch_g<M, MASK, Tin, 64>(a, tf, st);
+    if (a.G == 256) return launch_g<M, MASK, Tin, 256>(a, tf, st);
     return cudaErrorInvalidValue;
 }
 

@@ -21,7 +21,7 @@ struct InputArgs {
     long T_pad;      // T rounded up to 128
     int G;
     int ngo;         // Cout / G (rows of the Y absmax table to clear)
-    int8_t* Vq;      // [T][n*n][Cin]
+    int8_t* Vq;      // [n*n][T_pad][Cin] (tap-major)
     float* sV;       // [n*n][Cin/G][T_pad]
     unsigned* amax;  // [T_pad][Cout/G], cleared here
     int* err;        // device error word, cleared here
@@ -34,17 +34,17 @@ enum GemmMode { kModeAbsmax = 0, kModeQuant = 1, kModeY32 = 2 };
 
 struct GemmArgs {
     int T, T_pad, Cin, Cout, n2, G, ng, ngo;
-    int BK, stages, tpu, num_tc, num_mb, num_nb, num_units;
+    int SK, BK, tps, stages, tpu, num_tc, num_mb, num_nb, num_units;  // stage shape and work split (set by the launcher)
     const float* sV;   // [n2][ng][T_pad]
     const float* sU;   // [n2][ng][Cout]
     unsigned* amax;    // [T_pad][ngo] fp32 bits of |Y| maxima
-    int8_t* Yq;        // [T][n2][Cout]   (quant mode)
-    float* Y32;        // [T][n2][Cout]   (Y32 mode)
+    int8_t* Yq;        // [n2][T][Cout]   (quant mode)
+    float* Y32;        // [n2][T][Cout]   (Y32 mode)
     int* acc;          // [n2][T][Cout][ng] (debug dump) or null
     int* err;
 };
 
-// Tensor maps and launch of the tcgen05 kernel; `Vq` is [T_pad][n2][Cin], `Uq` [n2][Cout][Cin].
+// Tensor maps and launch of the tcgen05 kernel; `Vq` is [n2][T_pad][Cin], `Uq` [n2][Cout][Cin].
 cudaError_t launch_hadamard_tc(GemmArgs a, const int8_t* Vq, const int8_t* Uq, int mode, int num_sms,
                                cudaStream_t st, int* launches);
 int tc_block_n(int Cout, int G);  // 0 if unsupported
@@ -56,8 +56,8 @@ struct OutputArgs {
     int N, H, W, Cout, TH, TW;
     long T;
     int n2, G, ngo;
-    const int8_t* Yq;      // [T][n2][Cout] (Yq source) or written (debug)
-    const float* Y32;      // [T][n2][Cout] (Y32 source)
+    const int8_t* Yq;      // [n2][T][Cout] (Yq source)
+    const float* Y32;      // [n2][T][Cout] (Y32 source)
     const unsigned* amax;  // [T_pad][ngo]
     int8_t* Yq_dbg;        // debug copy of Yq (Y32 source), or null
     float* sY_dbg;         // debug copy of sY [T][ngo], or null

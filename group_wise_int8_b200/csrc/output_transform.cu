@@ -24,19 +24,20 @@ __global__ void __launch_bounds__(256) output_transform_kernel(OutputArgs p, Tra
     const int co = (int)(i - t * p.Cout);
     if (t >= p.T) return;
     const int cg = co / p.G;
-    const float s = group_scale(__uint_as_float(p.amax[(size_t)t * p.ngo + cg]));
+    const QScale qs = make_qscale(__uint_as_float(p.amax[(size_t)t * p.ngo + cg]));
+    const float s = qs.s;
     if (DEBUG && co % p.G == 0) p.sY_dbg[(size_t)t * p.ngo + cg] = s;
 
     float Y[N][N];
-    const size_t base = (size_t)t * N2 * p.Cout + co;
+    const size_t base = (size_t)t * p.Cout + co;   // Yq / Y32 are tap-major [n2][T][Cout]
 #pragma unroll
     for (int k = 0; k < N2; ++k) {
         int q;
         if (SRC_Y32) {
-            q = quant_code(p.Y32[base + (size_t)k * p.Cout], s);
-            if (DEBUG) p.Yq_dbg[base + (size_t)k * p.Cout] = (int8_t)q;
+            q = quant_code_fast(p.Y32[base + (size_t)k * p.T * p.Cout], qs);
+            if (DEBUG) p.Yq_dbg[base + (size_t)k * p.T * p.Cout] = (int8_t)q;
         } else {
-            q = p.Yq[base + (size_t)k * p.Cout];
+            q = p.Yq[base + (size_t)k * p.T * p.Cout];
         }
         Y[k / N][k % N] = __fmul_rn(s, (float)q);
     }

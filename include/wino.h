@@ -83,7 +83,8 @@ typedef struct wino_opts {
 #define WINO_DEBUG_YQ 1
 #define WINO_DEBUG_ACC32 2
 
-/* Debug dump selectors for wino_debug_dump (logical layouts of the copy). */
+/* Debug dump selectors for wino_debug_dump (logical, tile-major layouts of the copy;
+ * the kernels keep Vq, sV, Yq and Y tap-major in the workspace). */
 #define WINO_DUMP_VQ 0    /* int8  [T][n*n][Cin]        quantised input transform */
 #define WINO_DUMP_SV 1    /* fp32  [T][n*n][Cin/G]      its scales */
 #define WINO_DUMP_YQ 2    /* int8  [T][n*n][Cout]       requantised Y (needs WINO_DEBUG_YQ on the Y32 path) */
