@@ -160,6 +160,23 @@ class ClockSampler:
                 "samples": len(sm)}
 
 
+# ---------------------------------------------------------------- multi-rank
+def max_over_ranks(value: float, world: int, device=None) -> float:
+    """The largest of every rank's value (all ranks call it, in the same order)."""
+    if world <= 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(units_per_rank: float, world: int, max_ms: float) -> float:
+    """Whole-job rate (weak scaling: every rank processes its own batch)."""
+    return world * units_per_rank / (max_ms * 1e-3)
+
+
 # --------------------------------------------------------------- our CUDA path
 def run_ours(args, layer, rank, world):
     import torch
@@ -221,11 +238,7 @@ def run_ours(args, layer, rank, world):
     stage_ms, calls = plan.profile_end()
     assert calls == args.steps
     assert plan.check_device_error(ws, N, H, W, Cin, Cout) == wino.OK
-    total_ms = sum(s.elapsed_time(e) for s, e in zip(starts, ends))
-    if world > 1:
-        t = torch.tensor([total_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(sum(s.elapsed_time(e) for s, e in zip(starts, ends)), world, dev)
 
     # end to end through the host-buffer entry point (H2D of x, conv, D2H of y per step)
     e2e = None
@@ -249,12 +262,8 @@ def run_ours(args, layer, rank, world):
             plan.conv2d_host(x_host, wt, Cout, y_host, ws_h)
         e1.record(stream)
         torch.cuda.synchronize()
-        e_ms = e0.elapsed_time(e1)
-        if world > 1:
-            t = torch.tensor([e_ms], device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e_ms = float(t.item())
-        e2e = {"value": world * k * layer.direct_flops / (e_ms * 1e-3) / 1e12, "unit": UNIT,
+        e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
+        e2e = {"value": job_throughput(k * layer.direct_flops, world, e_ms) / 1e12, "unit": UNIT,
                "h2d_bytes_per_step": int(N * H * W * Cin * xs), "d2h_bytes_per_step": int(N * H * W * Cout * 2),
                "steps": k, "ms_per_step": e_ms / k}
 
@@ -275,7 +284,7 @@ def run_ours(args, layer, rank, world):
                    "int8_tops": round(m[2] / (a * 1e-3) / 1e12, 2) if m[2] else None}
                   for m, a in zip(model, avg_ms)]
     ms_step = total_ms / args.steps
-    value = world * args.steps * layer.direct_flops / (total_ms * 1e-3) / 1e12
+    value = job_throughput(args.steps * layer.direct_flops, world, total_ms) / 1e12
     return {
         "value": value, "ms_per_step": ms_step, "e2e": e2e, "roofline": roofline, "clocks": clocks,
         "gpu_launches": args.steps * launches, "per_kernel": per_kernel, "wall_s": t_wall,

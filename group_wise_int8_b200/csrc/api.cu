@@ -195,6 +195,7 @@ int run_conv(wino_plan_s* p, const void* x, int x_dtype, int N, int H, int W, in
     ga.Y32 = Y32;
     ga.acc = acc;
     ga.err = err;
+    ga.force_timeout = (p->opts.debug & WINO_DEBUG_FORCE_TIMEOUT) != 0 && L.gemm == WINO_GEMM_TCGEN05;
     auto gemm = [&](int mode) -> cudaError_t {
         prof_mark(p, slot++, st);
         if (L.gemm == WINO_GEMM_SIMT) return launch_hadamard_simt(ga, Vq, Uq, mode, st);

@@ -65,6 +65,7 @@ struct SmemTail {
     uint64_t acc_full[kMaxNacc];
     uint64_t acc_empty[kMaxNacc];
     uint64_t done;
+    uint64_t never;      // completed by nobody: the forced-timeout test hook waits on it
     uint32_t tmem_base;
     int abort_flag;
 };
@@ -148,6 +149,7 @@ __global__ void __launch_bounds__(TcCfg<BN>::kThreads, 1)
             mbar_init(&tail->acc_empty[b], Cfg::kEpiWarps);
         }
         mbar_init(&tail->done, 1);
+        mbar_init(&tail->never, 1);
         tail->abort_flag = 0;
         fence_mbar_init();
         fence_proxy_async_smem();
@@ -216,6 +218,7 @@ __global__ void __launch_bounds__(TcCfg<BN>::kThreads, 1)
             const int ks_per_chunk = BK / 32;
             Ring st{0, 0}, bf{0, 0};
             bool ok = true;
+            if (p.force_timeout) ok = mbar_wait(&tail->never, 0, abort_flag, p.err, 1000000ull);
             UnitIter u;
             for (u.init(blockIdx.x, p); ok && u.unit < p.num_units; u.advance(gridDim.x, p)) {
                 const int tap_end = min(p.n2, (u.tc + 1) * p.tpu);

@@ -42,6 +42,7 @@ struct GemmArgs {
     float* Y32;        // [n2][T][Cout]   (Y32 mode)
     int* acc;          // [n2][T][Cout][ng] (debug dump) or null
     int* err;
+    int force_timeout; // test hook: the MMA thread first waits 1 ms on a barrier nothing completes
 };
 
 // Tensor maps and launch of the tcgen05 kernel; `Vq` is [n2][T_pad][Cin], `Uq` [n2][Cout][Cin].

@@ -30,7 +30,7 @@ BF16 = 1
 
 YPATH_AUTO, YPATH_RECOMPUTE, YPATH_Y32 = 0, 1, 2
 GEMM_AUTO, GEMM_TCGEN05, GEMM_SIMT = 0, 1, 2
-DEBUG_YQ, DEBUG_ACC32 = 1, 2
+DEBUG_YQ, DEBUG_ACC32, DEBUG_FORCE_TIMEOUT = 1, 2, 4
 DUMP_VQ, DUMP_SV, DUMP_YQ, DUMP_SY, DUMP_Y32, DUMP_ACC32 = range(6)
 
 EXPORTED = [

@@ -76,12 +76,18 @@ typedef struct wino_opts {
     int gemm;      /* WINO_GEMM_* */
     int debug;     /* bit 0: materialise Yq and sY in the workspace on every path;
                       bit 1: dump the int32 per-K-group accumulators (needs the
-                             larger workspace wino_workspace_bytes reports) */
+                             larger workspace wino_workspace_bytes reports);
+                      bit 2: failure-detection test hook: the tcgen05 GEMM first
+                             waits 1 ms on a barrier nothing completes, so its
+                             bounded wait expires, every CTA returns early and
+                             wino_check_device_error reports
+                             WINO_ERR_DEVICE_TIMEOUT (output undefined) */
     int reserved[5];
 } wino_opts;
 
 #define WINO_DEBUG_YQ 1
 #define WINO_DEBUG_ACC32 2
+#define WINO_DEBUG_FORCE_TIMEOUT 4
 
 /* Debug dump selectors for wino_debug_dump (logical, tile-major layouts of the copy;
  * the kernels keep Vq, sV, Yq and Y tap-major in the workspace). */
