@@ -47,8 +47,8 @@ UNIT = "TFLOP/s"
 # line is the named file under profiles/.  None until a capture of the
 # current kernel exists.
 NCU_TRAFFIC = {
-    # profiles/resnet18_f63_g32_launches_and_full.md (input transform, CC=64 TX=4 kernel)
-    ("resnet18", 0, "input_transform"): 12904448,
+    # (workload, layer, kernel) -> dram read+write bytes per launch from one ncu capture of the
+    # CURRENT kernel; entries are removed whenever that kernel changes.
 }
 
 

@@ -48,15 +48,48 @@ __device__ __forceinline__ int quant_code(float v, float s) {
 // Group scale from an absmax.
 __device__ __forceinline__ float group_scale(float amax) { return __fdiv_rn(amax, 127.0f); }
 
-// A group scale with the fp64 reciprocal of its value, for quant_code_fast.
+// Packed fp32 pairs (sm_100): each lane of the pair is rounded exactly as the
+// scalar instruction would round it.
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+__device__ __forceinline__ void f2_unpack(uint64_t v, float& lo, float& hi) {
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ uint64_t f2_sub(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+
+// A group scale with its reciprocals for the quantisers below.
 struct QScale {
     float s;
+    float r;    // RN24(1 / s); 0 when s == 0 or s lies outside [2^-100, 2^100]
     double rd;  // RN53(1 / s); 0 when s == 0
 };
 
 __device__ __forceinline__ QScale make_qscale(float amax) {
     QScale q;
     q.s = group_scale(amax);
+    q.r = (q.s >= 0x1p-100f && q.s <= 0x1p100f) ? __frcp_rn(q.s) : 0.0f;
     q.rd = q.s != 0.0f ? __drcp_rn((double)q.s) : 0.0;
     return q;
 }
@@ -75,6 +108,50 @@ __device__ __forceinline__ int quant_code_fast(float v, QScale q) {
     int c = __float_as_int(__fadd_rn(r, kRoundMagic)) - kRoundMagicBits;
     c = c > 127 ? 127 : c;
     return c < -127 ? -127 : c;
+}
+
+// Codes of four values of one group (|v| <= the group's absmax), in fp32
+// pairs: t = RN(v * RN(1/s)) lies within 2.3e-5 of RN(v/s) (|v/s| < 127.0001;
+// one rounding each in 1/s, in t and in RN(v/s), at most 2^-24 relative), so
+// when every t is more than 2^-12 from a half-integer, rne(t) = rne(RN(v/s))
+// and the clamp cannot act (|rne| <= 127).  a = t + 1.5*2^23 holds rne(t) in
+// its low mantissa bits, so byte 0 of a's bits is the int8 code and k = a -
+// 1.5*2^23 is rne(t) as a float.  Otherwise (about one value in 4000, or a
+// scale outside [2^-100, 2^100]) the fp64 quotient decides.
+struct Quad {
+    uint64_t k01, k23;  // rne codes as floats
+    uint32_t packed;    // the four int8 codes, value 0 in byte 0
+};
+
+__device__ __forceinline__ Quad quant4(float v0, float v1, float v2, float v3, const QScale& q) {
+    Quad o;
+    const uint64_t magic2 = f2_pack(kRoundMagic, kRoundMagic);
+    if (q.r != 0.0f || q.s == 0.0f) {
+        const uint64_t r2 = f2_pack(q.r, q.r);
+        const uint64_t t01 = f2_mul(f2_pack(v0, v1), r2), t23 = f2_mul(f2_pack(v2, v3), r2);
+        const uint64_t a01 = f2_add(t01, magic2), a23 = f2_add(t23, magic2);
+        o.k01 = f2_sub(a01, magic2);
+        o.k23 = f2_sub(a23, magic2);
+        float d0, d1, d2, d3;
+        f2_unpack(f2_sub(t01, o.k01), d0, d1);
+        f2_unpack(f2_sub(t23, o.k23), d2, d3);
+        const float dmax = fmaxf(fmaxf(fabsf(d0), fabsf(d1)), fmaxf(fabsf(d2), fabsf(d3)));
+        if (dmax < 0.5f - 0x1p-12f) {
+            float a0, a1, a2, a3;
+            f2_unpack(a01, a0, a1);
+            f2_unpack(a23, a2, a3);
+            o.packed = __byte_perm(__byte_perm(__float_as_uint(a0), __float_as_uint(a1), 0x0040),
+                                   __byte_perm(__float_as_uint(a2), __float_as_uint(a3), 0x0040), 0x5410);
+            return o;
+        }
+    }
+    const int c0 = quant_code_fast(v0, q), c1 = quant_code_fast(v1, q);
+    const int c2 = quant_code_fast(v2, q), c3 = quant_code_fast(v3, q);
+    o.k01 = f2_pack((float)c0, (float)c1);
+    o.k23 = f2_pack((float)c2, (float)c3);
+    o.packed = (uint32_t)(c0 & 0xff) | ((uint32_t)(c1 & 0xff) << 8) | ((uint32_t)(c2 & 0xff) << 16) |
+               ((uint32_t)(c3 & 0xff) << 24);
+    return o;
 }
 
 // Recursive-halving max over the 32 lanes of a warp for 64 values per lane.

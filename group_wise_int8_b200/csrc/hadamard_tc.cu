@@ -287,7 +287,7 @@ __global__ void __launch_bounds__(TcCfg<BN>::kThreads, 1)
             const int cgrp = colg / p.G;              // this thread's 32 columns lie in one Y group
             float gmax = 0.0f;
             QScale qy;
-            qy.s = 0.0f;
+            qy.s = qy.r = 0.0f;
             qy.rd = 0.0;
             if (MODE == kModeQuant && valid) qy = make_qscale(__uint_as_float(p.amax[(size_t)row * p.ngo + cgrp]));
             const int tap_end = min(p.n2, (u.tc + 1) * p.tpu);
@@ -350,13 +350,9 @@ __global__ void __launch_bounds__(TcCfg<BN>::kThreads, 1)
                                 for (int c = 0; c < 32; c += 16) {
                                     uint32_t w[4];
 #pragma unroll
-                                    for (int e = 0; e < 4; ++e) {
-                                        uint32_t pk = 0;
-#pragma unroll
-                                        for (int bb = 0; bb < 4; ++bb)
-                                            pk |= ((uint32_t)(quant_code_fast(y[c + 4 * e + bb], qy) & 0xff)) << (8 * bb);
-                                        w[e] = pk;
-                                    }
+                                    for (int e = 0; e < 4; ++e)
+                                        w[e] = quant4(y[c + 4 * e], y[c + 4 * e + 1], y[c + 4 * e + 2], y[c + 4 * e + 3], qy)
+                                                   .packed;
                                     *reinterpret_cast<uint4*>(dst + c) = make_uint4(w[0], w[1], w[2], w[3]);
                                 }
                             }
@@ -465,6 +461,16 @@ bool encode(EncodeTiledFn enc, CUtensorMap* map, CUtensorMapDataType dt, const v
 }
 
 }  // namespace
+
+bool make_tensor_map(CUtensorMap* map, CUtensorMapDataType dt, int rank, const void* base, const cuuint64_t* dims,
+                     const cuuint64_t* strides, const cuuint32_t* box, CUtensorMapSwizzle sw) {
+    EncodeTiledFn enc = get_encode_fn();
+    if (!enc || rank < 1 || rank > 5) return false;
+    const cuuint32_t es[5] = {1u, 1u, 1u, 1u, 1u};
+    return enc(map, dt, (cuuint32_t)rank, const_cast<void*>(base), dims, strides, box, es,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
 
 int tc_block_n(int Cout, int G) {
     if (Cout % 128 == 0 && (128 % G == 0 || G == 256)) return 128;

@@ -8,6 +8,11 @@
 
 namespace wino {
 
+// Encodes a tiled TMA tensor map (rank 2..5; strides in bytes for dims 1..rank-1,
+// no interleave, no L2 promotion change beyond 256 B, zero fill out of bounds).
+bool make_tensor_map(CUtensorMap* map, CUtensorMapDataType dt, int rank, const void* base, const cuuint64_t* dims,
+                     const cuuint64_t* strides, const cuuint32_t* box, CUtensorMapSwizzle sw);
+
 // ----------------------------------------------------------- weight transform
 cudaError_t launch_weight_transform(const WeightArgs& wa, int m, const float* w, int Cin, int Cout, int G,
                                     int8_t* Uq, float* sU, cudaStream_t st);

@@ -30,16 +30,21 @@ __global__ void __launch_bounds__(256) output_transform_kernel(OutputArgs p, Tra
 
     float Y[N][N];
     const size_t base = (size_t)t * p.Cout + co;   // Yq / Y32 are tap-major [n2][T][Cout]
+    const size_t tstride = (size_t)p.T * p.Cout;
+    if (SRC_Y32) {
+        const uint64_t s2 = f2_pack(s, s);
 #pragma unroll
-    for (int k = 0; k < N2; ++k) {
-        int q;
-        if (SRC_Y32) {
-            q = quant_code_fast(p.Y32[base + (size_t)k * p.T * p.Cout], qs);
-            if (DEBUG) p.Yq_dbg[base + (size_t)k * p.T * p.Cout] = (int8_t)q;
-        } else {
-            q = p.Yq[base + (size_t)k * p.T * p.Cout];
+        for (int k = 0; k < N2; k += 4) {
+            const float* src = p.Y32 + base + (size_t)k * tstride;
+            const Quad qd = quant4(src[0], src[tstride], src[2 * tstride], src[3 * tstride], qs);
+            f2_unpack(f2_mul(s2, qd.k01), Y[k / N][k % N], Y[(k + 1) / N][(k + 1) % N]);
+            f2_unpack(f2_mul(s2, qd.k23), Y[(k + 2) / N][(k + 2) % N], Y[(k + 3) / N][(k + 3) % N]);
+            if (DEBUG)
+                for (int e = 0; e < 4; ++e) p.Yq_dbg[base + (size_t)(k + e) * tstride] = (int8_t)(qd.packed >> (8 * e));
         }
-        Y[k / N][k % N] = __fmul_rn(s, (float)q);
+    } else {
+#pragma unroll
+        for (int k = 0; k < N2; ++k) Y[k / N][k % N] = __fmul_rn(s, (float)p.Yq[base + (size_t)k * tstride]);
     }
     float Z[M][N];
 #pragma unroll
