@@ -13,6 +13,8 @@ namespace {
 template <int MODE, bool DUMP>
 __global__ void __launch_bounds__(256) hadamard_simt_kernel(GemmArgs p, const int8_t* __restrict__ Vq,
                                                             const int8_t* __restrict__ Uq) {
+    grid_dependents_launch();
+    grid_dependency_wait();
     const int tap = blockIdx.y;
     const long i = (long)blockIdx.x * blockDim.x + threadIdx.x;
     const long t = i / p.Cout;
@@ -51,20 +53,13 @@ cudaError_t launch_hadamard_simt(const GemmArgs& a, const int8_t* Vq, const int8
     const long threads = (long)a.T * a.Cout;
     const dim3 grid((unsigned)((threads + 255) / 256), a.n2);
     const bool dump = a.acc != nullptr && mode != kModeQuant;
-    switch (mode) {
-        case kModeAbsmax:
-            if (dump) hadamard_simt_kernel<kModeAbsmax, true><<<grid, 256, 0, st>>>(a, Vq, Uq);
-            else hadamard_simt_kernel<kModeAbsmax, false><<<grid, 256, 0, st>>>(a, Vq, Uq);
-            break;
-        case kModeQuant:
-            hadamard_simt_kernel<kModeQuant, false><<<grid, 256, 0, st>>>(a, Vq, Uq);
-            break;
-        default:
-            if (dump) hadamard_simt_kernel<kModeY32, true><<<grid, 256, 0, st>>>(a, Vq, Uq);
-            else hadamard_simt_kernel<kModeY32, false><<<grid, 256, 0, st>>>(a, Vq, Uq);
-            break;
-    }
-    return cudaGetLastError();
+    if (mode == kModeAbsmax)
+        return dump ? launch_dependent(hadamard_simt_kernel<kModeAbsmax, true>, grid, dim3(256), 0, st, a, Vq, Uq)
+                    : launch_dependent(hadamard_simt_kernel<kModeAbsmax, false>, grid, dim3(256), 0, st, a, Vq, Uq);
+    if (mode == kModeQuant)
+        return launch_dependent(hadamard_simt_kernel<kModeQuant, false>, grid, dim3(256), 0, st, a, Vq, Uq);
+    return dump ? launch_dependent(hadamard_simt_kernel<kModeY32, true>, grid, dim3(256), 0, st, a, Vq, Uq)
+                : launch_dependent(hadamard_simt_kernel<kModeY32, false>, grid, dim3(256), 0, st, a, Vq, Uq);
 }
 
 }  // namespace wino

@@ -17,17 +17,18 @@
 //            stage's groups;
 //   warp 0 = TMA producer;
 //   warp 1 = TMEM allocator and MMA issuer: tcgen05.mma kind::i8, M=128,
-//            N=BN, K=32 per instruction; each K-group accumulates into its own
-//            TMEM buffer (a ring of NACC buffers of BN columns, at most NACC/2
-//            groups per stage so the MMAs of the next stage overlap the
-//            epilogue of this one), one commit per group;
-//   warps 2.. = epilogue, 4 TMEM lane quadrants x BN/32 column chunks: one
-//            wait per stage, then per group a 32-column tcgen05.ld and the
+//            N=BN, K=32 per instruction; each K-group of a stage accumulates
+//            into its own BN-column TMEM buffer; the buffers of one stage form
+//            a slot, a ring of at least two slots lets the MMAs of the next
+//            stage overlap the epilogue of this one; one wait for a free slot
+//            and one commit per stage;
+//   warps 2..9 = epilogue, 4 TMEM lane quadrants x 2 pairs of column chunks
+//            of BN/4: per tap one wait, then per chunk and group a tcgen05.ld and the
 //            dequantisation in packed fp32 pairs; the buffers are refilled with
 //            the bias 0x4B400000 (so the next int32 sum lands on 1.5*2^23 and
-//            reinterprets as an exact fp32 value) and released together.  A
-//            stage returns to the producer when both the MMAs and the epilogue
-//            are done with it.
+//            reinterprets as an exact fp32 value) and the slot is released.  A
+//            stage's shared memory returns to the producer when every epilogue
+//            warp is done with it (which is after its MMAs completed).
 // The loops keep wrap-around ring counters (no division in the issue paths).
 // At the end of each tap the epilogue either keeps the running |Y| maximum of
 // each (tile, G-cout group) (absmax pass and fp32-Y pass, published with
@@ -52,12 +53,21 @@ constexpr int kMaxNacc = 8;
 
 template <int BN>
 struct TcCfg {
-    static constexpr int kEpiWarps = BN / 8;  // 4 lane quadrants x BN/32 column chunks
+    static constexpr int kCPT = BN / 4;       // columns per column chunk
+    static constexpr int kPasses = 2;         // column chunks per epilogue thread
+    static constexpr int kEpiWarps = 8;       // 4 TMEM lane quadrants x 2 chunk pairs
     static constexpr int kThreads = 64 + 32 * kEpiWarps;
     static constexpr int kNacc = (512 / BN) < kMaxNacc ? (512 / BN) : kMaxNacc;
     static constexpr int kTmemCols = (kNacc * BN) <= 32 ? 32 : (kNacc * BN) <= 64 ? 64 : (kNacc * BN) <= 128 ? 128
                                      : (kNacc * BN) <= 256 ? 256 : 512;
 };
+
+// max(a, |b|, |c|) in one three-input max (exact, like any max).
+__device__ __forceinline__ float max_abs3(float a, float b, float c) {
+    float r;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(fabsf(b)), "f"(fabsf(c)));
+    return r;
+}
 
 struct SmemTail {
     uint64_t full[kMaxStages];
@@ -100,17 +110,33 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volati
     }
 }
 
-// Units are numbered with the column block fastest, then the row block, then the tap chunk.
-struct UnitIter {
-    int unit, nb, mb, tc;
-    __device__ __forceinline__ void init(int first, const GemmArgs& p) {
-        unit = first;
-        nb = first % p.num_nb;
-        const int r = first / p.num_nb;
-        mb = r % p.num_mb;
-        tc = r / p.num_mb;
+// The tap-units L = (mb * num_nb + nb) * n2 + tap (one tap of one 128-row block
+// and one BN-column block) are split into equal contiguous ranges, one per
+// CTA.  Every role of a CTA walks its range the same way: a stage covers up to
+// TPS consecutive taps of one (mb, nb) block; the walk never divides.
+struct Walk {
+    int L, L1, tap, nb, mb;
+    __device__ __forceinline__ void init(const GemmArgs& p) {
+        const long tot = p.num_units;
+        L = (int)(tot * blockIdx.x / gridDim.x);
+        L1 = (int)(tot * (blockIdx.x + 1) / gridDim.x);
+        tap = L % p.n2;
+        const int r = L / p.n2;
+        nb = r % p.num_nb;
+        mb = r / p.num_nb;
     }
-    __device__ __forceinline__ void advance(int step, const GemmArgs& p) { init(unit + step, p); }
+    __device__ __forceinline__ int stage_taps(int tps, int n2) const { return min(min(tps, n2 - tap), L1 - L); }
+    __device__ __forceinline__ void advance(int k, const GemmArgs& p) {
+        L += k;
+        tap += k;
+        if (tap == p.n2) {
+            tap = 0;
+            if (++nb == p.num_nb) {
+                nb = 0;
+                ++mb;
+            }
+        }
+    }
 };
 
 template <int BN, int MODE, bool DUMP>
@@ -125,8 +151,9 @@ __global__ void __launch_bounds__(TcCfg<BN>::kThreads, 1)
     const int BK = p.BK;                   // swizzle width = bytes of K per tile row
     const int KC = p.SK / BK;              // K chunks per stage
     const int TPS = p.tps;                 // taps per stage
-    const int GPS = p.SK / p.G;            // K-groups per tap per stage
-    const int KSTAGES = p.Cin / p.SK;      // stages per tap
+    const int GPS = p.SK / p.G;            // K-groups per tap per stage = accumulator buffers per slot
+    const int KSTAGES = p.Cin / p.SK;      // stages per tap (TPS == 1 when > 1)
+    const int NSLOT = NACC / GPS;          // accumulator slots (>= 2)
     const uint32_t a_tile = kBM * BK, b_tile = BN * BK;
     const uint32_t a_bytes = a_tile * KC * TPS, b_bytes = b_tile * KC * TPS;
     const uint32_t stage_bytes = a_bytes + b_bytes;
@@ -138,14 +165,15 @@ __global__ void __launch_bounds__(TcCfg<BN>::kThreads, 1)
     const uint32_t scale_bytes = (uint32_t)TPS * GPS * (kBM + BN) * 4;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    grid_dependents_launch();
 
     if (warp == 0 && lane == 0) {
         for (int s = 0; s < S; ++s) {
             mbar_init(&tail->full[s], 1);
-            mbar_init(&tail->empty[s], 1 + Cfg::kEpiWarps);   // the MMA commit and every epilogue warp
+            mbar_init(&tail->empty[s], Cfg::kEpiWarps);   // every epilogue warp, after the stage's MMAs completed
         }
         for (int b = 0; b < NACC; ++b) {
-            mbar_init(&tail->acc_full[b], 1);
+            mbar_init(&tail->acc_full[b], 1);                 // one commit per tap
             mbar_init(&tail->acc_empty[b], Cfg::kEpiWarps);
         }
         mbar_init(&tail->done, 1);
@@ -162,6 +190,8 @@ __global__ void __launch_bounds__(TcCfg<BN>::kThreads, 1)
         tmem_alloc(&tail->tmem_base, Cfg::kTmemCols);
         tmem_relinquish();
     }
+    // barrier setup, TMEM allocation and descriptor prefetch overlap the previous kernel's tail
+    grid_dependency_wait();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -173,28 +203,29 @@ __global__ void __launch_bounds__(TcCfg<BN>::kThreads, 1)
             Ring st{0, 0};
             uint32_t issued = 0;
             bool ok = true;
-            UnitIter u;
-            for (u.init(blockIdx.x, p); ok && u.unit < p.num_units; u.advance(gridDim.x, p)) {
-                const int tap_end = min(p.n2, (u.tc + 1) * p.tpu);
-                for (int tap0 = u.tc * p.tpu; ok && tap0 < tap_end; tap0 += TPS)
-                    for (int ks = 0; ks < KSTAGES; ++ks) {
-                        if (!mbar_wait(&tail->empty[st.idx], st.phase ^ 1u, abort_flag, p.err)) {
-                            ok = false;
-                            break;
-                        }
-                        uint64_t* bar = &tail->full[st.idx];
-                        unsigned char* sa = smem + (size_t)st.idx * stage_bytes;
-                        mbar_arrive_expect_tx(bar, stage_bytes + scale_bytes);
-                        for (int c = 0; c < KC; ++c) {
-                            const int k0 = ks * p.SK + c * BK;
-                            tma_load_3d(sa + (size_t)c * TPS * a_tile, &tmA, bar, k0, u.mb * kBM, tap0);
-                            tma_load_3d(sa + a_bytes + (size_t)c * TPS * b_tile, &tmB, bar, k0, u.nb * BN, tap0);
-                        }
-                        tma_load_3d(sv_ring + (size_t)st.idx * TPS * GPS * kBM, &tmSV, bar, u.mb * kBM, ks * GPS, tap0);
-                        tma_load_3d(su_ring + (size_t)st.idx * TPS * GPS * BN, &tmSU, bar, u.nb * BN, ks * GPS, tap0);
-                        ++issued;
-                        st.next(S);
+            Walk w;
+            for (w.init(p); ok && w.L < w.L1;) {
+                const int nt = w.stage_taps(TPS, p.n2);
+                for (int ks = 0; ks < KSTAGES; ++ks) {
+                    if (!mbar_wait(&tail->empty[st.idx], st.phase ^ 1u, abort_flag, p.err)) {
+                        ok = false;
+                        break;
                     }
+                    // whole boxes of TPS taps; taps past n2 read zeros and taps past the range go unused
+                    uint64_t* bar = &tail->full[st.idx];
+                    unsigned char* sa = smem + (size_t)st.idx * stage_bytes;
+                    mbar_arrive_expect_tx(bar, stage_bytes + scale_bytes);
+                    for (int c = 0; c < KC; ++c) {
+                        const int k0 = ks * p.SK + c * BK;
+                        tma_load_3d(sa + (size_t)c * TPS * a_tile, &tmA, bar, k0, w.mb * kBM, w.tap);
+                        tma_load_3d(sa + a_bytes + (size_t)c * TPS * b_tile, &tmB, bar, k0, w.nb * BN, w.tap);
+                    }
+                    tma_load_3d(sv_ring + (size_t)st.idx * TPS * GPS * kBM, &tmSV, bar, w.mb * kBM, ks * GPS, w.tap);
+                    tma_load_3d(su_ring + (size_t)st.idx * TPS * GPS * BN, &tmSU, bar, w.nb * BN, ks * GPS, w.tap);
+                    ++issued;
+                    st.next(S);
+                }
+                w.advance(nt, p);
             }
             // drain: every issued load must land before the CTA can exit
             Ring dr{st.idx, st.phase};
@@ -214,46 +245,48 @@ __global__ void __launch_bounds__(TcCfg<BN>::kThreads, 1)
             const uint32_t idesc = idesc_i8(kBM, BN);
             const uint64_t a_desc0 = smem_desc_kmajor(smem_u32(smem), BK);
             const uint64_t b_desc0 = smem_desc_kmajor(smem_u32(smem) + a_bytes, BK);
+            const int ksteps = p.SK / 32;          // K-steps per tap and stage
             const int ks_per_group = p.G / 32;
             const int ks_per_chunk = BK / 32;
-            Ring st{0, 0}, bf{0, 0};
+            Ring st{0, 0}, sl{0, 0};
             bool ok = true;
             if (p.force_timeout) ok = mbar_wait(&tail->never, 0, abort_flag, p.err, 1000000ull);
-            UnitIter u;
-            for (u.init(blockIdx.x, p); ok && u.unit < p.num_units; u.advance(gridDim.x, p)) {
-                const int tap_end = min(p.n2, (u.tc + 1) * p.tpu);
-                for (int tap0 = u.tc * p.tpu; ok && tap0 < tap_end; tap0 += TPS)
-                    for (int ks = 0; ok && ks < KSTAGES; ++ks) {
-                        if (!mbar_wait(&tail->full[st.idx], st.phase, abort_flag, p.err)) {
+            Walk w;
+            for (w.init(p); ok && w.L < w.L1;) {
+                const int nt = w.stage_taps(TPS, p.n2);
+                for (int ks = 0; ok && ks < KSTAGES; ++ks) {
+                    if (!mbar_wait(&tail->full[st.idx], st.phase, abort_flag, p.err)) {
+                        ok = false;
+                        break;
+                    }
+                    const uint64_t stage_off = (uint64_t)((st.idx * stage_bytes) >> 4);
+                    for (int t = 0; t < nt; ++t) {
+                        if (!mbar_wait(&tail->acc_empty[sl.idx], sl.phase, abort_flag, p.err)) {
                             ok = false;
                             break;
                         }
                         tc_fence_after();
-                        const uint64_t stage_off = (uint64_t)((st.idx * stage_bytes) >> 4);
-                        for (int t = 0; ok && t < TPS; ++t) {
-                            int gk = 0;  // K-steps into the current group
-                            for (int c = 0; ok && c < KC; ++c)
-                                for (int kin = 0; kin < ks_per_chunk; ++kin) {
-                                    if (gk == 0) {
-                                        if (!mbar_wait(&tail->acc_empty[bf.idx], bf.phase, abort_flag, p.err)) {
-                                            ok = false;
-                                            break;
-                                        }
-                                        tc_fence_after();
-                                    }
-                                    const uint64_t koff = stage_off + (uint64_t)(((c * TPS + t) * a_tile + kin * 32) >> 4);
-                                    const uint64_t kofb = stage_off + (uint64_t)(((c * TPS + t) * b_tile + kin * 32) >> 4);
-                                    mma_i8(tmem_base + (uint32_t)(bf.idx * BN), a_desc0 + koff, b_desc0 + kofb, idesc, 1u);
-                                    if (++gk == ks_per_group) {
-                                        gk = 0;
-                                        mma_commit(&tail->acc_full[bf.idx]);
-                                        bf.next(NACC);
-                                    }
-                                }
+                        const uint32_t d = tmem_base + (uint32_t)(sl.idx * GPS * BN);
+                        int c = 0, kin = 0, g = 0, gk = 0;
+                        for (int kk = 0; kk < ksteps; ++kk) {
+                            const uint64_t koff = stage_off + (uint64_t)(((c * TPS + t) * a_tile + kin * 32) >> 4);
+                            const uint64_t kofb = stage_off + (uint64_t)(((c * TPS + t) * b_tile + kin * 32) >> 4);
+                            mma_i8(d + (uint32_t)(g * BN), a_desc0 + koff, b_desc0 + kofb, idesc, 1u);
+                            if (++kin == ks_per_chunk) {
+                                kin = 0;
+                                ++c;
+                            }
+                            if (++gk == ks_per_group) {
+                                gk = 0;
+                                ++g;
+                            }
                         }
-                        mma_commit(&tail->empty[st.idx]);
-                        st.next(S);
+                        mma_commit(&tail->acc_full[sl.idx]);
+                        sl.next(NSLOT);
                     }
+                    st.next(S);
+                }
+                w.advance(nt, p);
             }
             // all issued MMAs complete before TMEM is released
             mma_commit(&tail->done);
@@ -261,134 +294,172 @@ __global__ void __launch_bounds__(TcCfg<BN>::kThreads, 1)
         }
     } else {
         // ----------------------------------------------------------- epilogue
+        // Thread (quad, lane) of epilogue warp ew owns row 32*quad + lane and the
+        // column chunks (ew >> 2) + 2h, h = 0, 1, of CPT columns each, handled in turn.
+        constexpr int CPT = Cfg::kCPT, NP = Cfg::kPasses;
         const int ew = warp - 2;
         const int quad = warp & 3;                    // TMEM lanes 32*quad .. 32*quad+31
-        const int col0 = (ew / 4) * 32;               // this thread's 32 columns in the BN block
         const int rloc = 32 * quad + lane;            // row within the 128-tile block
-        const uint32_t t_lane = tmem_base + ((uint32_t)(32 * quad) << 16) + (uint32_t)col0;
+        int col0[NP];
+#pragma unroll
+        for (int h = 0; h < NP; ++h) col0[h] = ((ew >> 2) + 2 * h) * CPT;
+        const uint32_t t_lane = tmem_base + ((uint32_t)(32 * quad) << 16);
         const uint64_t neg_magic2 = f2_pack(-kRoundMagic, -kRoundMagic);
-        const int gst = TPS * GPS;                    // groups per stage
 
         // every accumulator buffer starts filled with the bias
-        for (int b = 0; b < NACC; ++b) tmem_st32_fill(t_lane + b * BN, (uint32_t)kRoundMagicBits);
+        for (int b = 0; b < NSLOT * GPS; ++b)
+#pragma unroll
+            for (int h = 0; h < NP; ++h) tmem_fill<CPT>(t_lane + (uint32_t)(b * BN + col0[h]), (uint32_t)kRoundMagicBits);
         tmem_st_wait();
         tc_fence_before();
         __syncwarp();
         if (lane == 0)
-            for (int b = 0; b < NACC; ++b) mbar_arrive(&tail->acc_empty[b]);
+            for (int b = 0; b < NSLOT; ++b) mbar_arrive(&tail->acc_empty[b]);
 
-        Ring st{0, 0}, bf{0, 0};
+        Ring st{0, 0}, sl{0, 0};
         bool ok = true;
-        UnitIter u;
-        for (u.init(blockIdx.x, p); ok && u.unit < p.num_units; u.advance(gridDim.x, p)) {
-            const int row = u.mb * kBM + rloc;
-            const bool valid = row < p.T;
-            const int colg = u.nb * BN + col0;
-            const int cgrp = colg / p.G;              // this thread's 32 columns lie in one Y group
-            float gmax = 0.0f;
-            QScale qy;
-            qy.s = qy.r = 0.0f;
-            qy.rd = 0.0;
-            if (MODE == kModeQuant && valid) qy = make_qscale(__uint_as_float(p.amax[(size_t)row * p.ngo + cgrp]));
-            const int tap_end = min(p.n2, (u.tc + 1) * p.tpu);
-            uint64_t y2[16];
-            for (int tap0 = u.tc * p.tpu; ok && tap0 < tap_end; tap0 += TPS)
-                for (int ks = 0; ok && ks < KSTAGES; ++ks) {
-                    // the stage's scales and the last of its groups' accumulators
-                    Ring last = bf;
-                    for (int i = 1; i < gst; ++i) last.next(NACC);
-                    if (!warp_wait(&tail->full[st.idx], st.phase, abort_flag, p.err) ||
-                        !warp_wait(&tail->acc_full[last.idx], last.phase, abort_flag, p.err)) {
+        int row = 0, blk = -1;
+        bool valid = false;
+        int colg[NP], cgrp[NP];
+        float gmax[NP];
+        QScale qy[NP];
+#pragma unroll
+        for (int h = 0; h < NP; ++h) {
+            colg[h] = cgrp[h] = 0;
+            gmax[h] = 0.0f;
+            qy[h].s = qy[h].r = 0.0f;
+            qy[h].rd = 0.0;
+        }
+        uint64_t y2[NP][CPT / 2];
+        Walk w;
+        for (w.init(p); ok && w.L < w.L1;) {
+            const int nt = w.stage_taps(TPS, p.n2);
+            const int b_id = w.mb * p.num_nb + w.nb;
+            if (b_id != blk) {
+                // a new (row block, column block): publish the running |Y| maxima of the previous one
+#pragma unroll
+                for (int h = 0; h < NP; ++h) {
+                    if (MODE != kModeQuant && valid && blk >= 0)
+                        atomicMax(&p.amax[(size_t)row * p.ngo + cgrp[h]], __float_as_uint(gmax[h]));
+                }
+                blk = b_id;
+                row = w.mb * kBM + rloc;
+                valid = row < p.T;
+#pragma unroll
+                for (int h = 0; h < NP; ++h) {
+                    colg[h] = w.nb * BN + col0[h];
+                    cgrp[h] = colg[h] / p.G;          // CPT <= G: a chunk's columns lie in one Y group
+                    gmax[h] = 0.0f;
+                    if (MODE == kModeQuant && valid)
+                        qy[h] = make_qscale(__uint_as_float(p.amax[(size_t)row * p.ngo + cgrp[h]]));
+                }
+            }
+            for (int ks = 0; ok && ks < KSTAGES; ++ks) {
+                if (!warp_wait(&tail->full[st.idx], st.phase, abort_flag, p.err)) {   // the stage's scales
+                    ok = false;
+                    break;
+                }
+                const float* svs = sv_ring + (size_t)st.idx * TPS * GPS * kBM + rloc;
+                const float* sus = su_ring + (size_t)st.idx * TPS * GPS * BN;
+                for (int t = 0; t < nt; ++t) {
+                    const int tap = w.tap + t;
+                    if (!warp_wait(&tail->acc_full[sl.idx], sl.phase, abort_flag, p.err)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
-                    const float* svs = sv_ring + (size_t)st.idx * TPS * GPS * kBM;
-                    const float* sus = su_ring + (size_t)st.idx * TPS * GPS * BN;
-                    Ring b = bf;
-                    for (int t = 0; t < TPS; ++t) {
-                        const int tap = tap0 + t;
-                        if (ks == 0) {
+                    if (ks == 0) {
 #pragma unroll
-                            for (int c = 0; c < 16; ++c) y2[c] = 0ull;
-                        }
+                        for (int h = 0; h < NP; ++h)
+#pragma unroll
+                            for (int c = 0; c < CPT / 2; ++c) y2[h][c] = 0ull;
+                    }
+                    const uint32_t t_slot = t_lane + (uint32_t)(sl.idx * GPS * BN);
+#pragma unroll
+                    for (int h = 0; h < NP; ++h)
                         for (int j = 0; j < GPS; ++j) {
-                            uint32_t r[32];
-                            tmem_ld32(t_lane + b.idx * BN, r);
+                            // one chunk of one group at a time; after the slot's last load, refill and release it
+                            uint32_t r[CPT];
+                            tmem_ld<CPT>(t_slot + (uint32_t)(j * BN + col0[h]), r);
                             tmem_ld_wait();
-                            const float sv = svs[(t * GPS + j) * kBM + rloc];
-                            const uint64_t sv2 = f2_pack(sv, sv);
-                            const float4* su4 = reinterpret_cast<const float4*>(sus + (t * GPS + j) * BN + col0);
+                            if (h + 1 == NP && j + 1 == GPS) {
+                                for (int b = 0; b < GPS; ++b)
 #pragma unroll
-                            for (int c4 = 0; c4 < 8; ++c4) {
+                                    for (int hh = 0; hh < NP; ++hh)
+                                        tmem_fill<CPT>(t_slot + (uint32_t)(b * BN + col0[hh]), (uint32_t)kRoundMagicBits);
+                                tmem_st_wait();
+                                tc_fence_before();
+                                __syncwarp();
+                                if (lane == 0) mbar_arrive(&tail->acc_empty[sl.idx]);
+                            }
+                            const float sv = svs[(t * GPS + j) * kBM];
+                            const uint64_t sv2 = f2_pack(sv, sv);
+                            const float4* su4 = reinterpret_cast<const float4*>(sus + (t * GPS + j) * BN + col0[h]);
+#pragma unroll
+                            for (int c4 = 0; c4 < CPT / 4; ++c4) {
                                 const float4 uu = su4[c4];
-                                const uint64_t a0 =
-                                    f2_add(f2_pack(__uint_as_float(r[4 * c4 + 0]), __uint_as_float(r[4 * c4 + 1])), neg_magic2);
-                                const uint64_t a1 =
-                                    f2_add(f2_pack(__uint_as_float(r[4 * c4 + 2]), __uint_as_float(r[4 * c4 + 3])), neg_magic2);
-                                y2[2 * c4 + 0] = f2_fma(a0, f2_mul(sv2, f2_pack(uu.x, uu.y)), y2[2 * c4 + 0]);
-                                y2[2 * c4 + 1] = f2_fma(a1, f2_mul(sv2, f2_pack(uu.z, uu.w)), y2[2 * c4 + 1]);
+                                const uint64_t a0 = f2_add(
+                                    f2_pack(__uint_as_float(r[4 * c4 + 0]), __uint_as_float(r[4 * c4 + 1])), neg_magic2);
+                                const uint64_t a1 = f2_add(
+                                    f2_pack(__uint_as_float(r[4 * c4 + 2]), __uint_as_float(r[4 * c4 + 3])), neg_magic2);
+                                y2[h][2 * c4 + 0] = f2_fma(a0, f2_mul(sv2, f2_pack(uu.x, uu.y)), y2[h][2 * c4 + 0]);
+                                y2[h][2 * c4 + 1] = f2_fma(a1, f2_mul(sv2, f2_pack(uu.z, uu.w)), y2[h][2 * c4 + 1]);
                             }
                             if (DUMP && valid) {
                                 const int jg = ks * GPS + j;
 #pragma unroll
-                                for (int c = 0; c < 32; ++c)
-                                    p.acc[(((size_t)tap * p.T + row) * p.Cout + colg + c) * p.ng + jg] =
+                                for (int c = 0; c < CPT; ++c)
+                                    p.acc[(((size_t)tap * p.T + row) * p.Cout + colg[h] + c) * p.ng + jg] =
                                         (int)r[c] - kRoundMagicBits;
                             }
-                            b.next(NACC);
                         }
-                        if (ks + 1 < KSTAGES) continue;
-                        // ---- end of tap
-                        float y[32];
+                    sl.next(NSLOT);
+                    if (ks + 1 < KSTAGES) continue;
+                    // ---- end of tap
 #pragma unroll
-                        for (int c = 0; c < 16; ++c) f2_unpack(y2[c], y[2 * c], y[2 * c + 1]);
+                    for (int h = 0; h < NP; ++h) {
+                        float y[CPT];
+#pragma unroll
+                        for (int c = 0; c < CPT / 2; ++c) f2_unpack(y2[h][c], y[2 * c], y[2 * c + 1]);
                         if (MODE == kModeQuant) {
                             if (valid) {
-                                int8_t* dst = p.Yq + ((size_t)tap * p.T + row) * p.Cout + colg;
+                                uint32_t q[CPT / 4];
 #pragma unroll
-                                for (int c = 0; c < 32; c += 16) {
-                                    uint32_t w[4];
+                                for (int e = 0; e < CPT / 4; ++e)
+                                    q[e] = quant4(y[4 * e], y[4 * e + 1], y[4 * e + 2], y[4 * e + 3], qy[h]).packed;
+                                int8_t* dst = p.Yq + ((size_t)tap * p.T + row) * p.Cout + colg[h];
+                                if (CPT == 8) {
+                                    *reinterpret_cast<uint2*>(dst) = make_uint2(q[0], q[1 % (CPT / 4)]);
+                                } else {
 #pragma unroll
-                                    for (int e = 0; e < 4; ++e)
-                                        w[e] = quant4(y[c + 4 * e], y[c + 4 * e + 1], y[c + 4 * e + 2], y[c + 4 * e + 3], qy)
-                                                   .packed;
-                                    *reinterpret_cast<uint4*>(dst + c) = make_uint4(w[0], w[1], w[2], w[3]);
+                                    for (int c = 0; c < CPT / 16; ++c)
+                                        *reinterpret_cast<uint4*>(dst + 16 * c) =
+                                            make_uint4(q[4 * c], q[4 * c + 1], q[4 * c + 2], q[4 * c + 3]);
                                 }
                             }
                         } else {
 #pragma unroll
-                            for (int c = 0; c < 32; ++c) gmax = fmaxf(gmax, fabsf(y[c]));
+                            for (int c = 0; c < CPT; c += 2) gmax[h] = max_abs3(gmax[h], y[c], y[c + 1]);
                             if (MODE == kModeY32 && valid) {
-                                float* dst = p.Y32 + ((size_t)tap * p.T + row) * p.Cout + colg;
+                                float* dst = p.Y32 + ((size_t)tap * p.T + row) * p.Cout + colg[h];
 #pragma unroll
-                                for (int c = 0; c < 32; c += 4)
+                                for (int c = 0; c < CPT; c += 4)
                                     *reinterpret_cast<float4*>(dst + c) = make_float4(y[c], y[c + 1], y[c + 2], y[c + 3]);
                             }
                         }
                     }
-                    // refill this stage's buffers with the bias and release them and the stage
-                    b = bf;
-                    for (int i = 0; i < gst; ++i) {
-                        tmem_st32_fill(t_lane + b.idx * BN, (uint32_t)kRoundMagicBits);
-                        b.next(NACC);
-                    }
-                    tmem_st_wait();
-                    tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0) {
-                        b = bf;
-                        for (int i = 0; i < gst; ++i) {
-                            mbar_arrive(&tail->acc_empty[b.idx]);
-                            b.next(NACC);
-                        }
-                        mbar_arrive(&tail->empty[st.idx]);
-                    }
-                    bf = b;
-                    st.next(S);
                 }
-            if (ok && MODE != kModeQuant && valid) atomicMax(&p.amax[(size_t)row * p.ngo + cgrp], __float_as_uint(gmax));
+                // the stage's shared memory (operands read by the completed MMAs, scales read above) is free
+                __syncwarp();
+                if (ok && lane == 0) mbar_arrive(&tail->empty[st.idx]);
+                st.next(S);
+            }
+            w.advance(nt, p);
         }
+#pragma unroll
+        for (int h = 0; h < NP; ++h)
+            if (ok && MODE != kModeQuant && valid && blk >= 0)
+                atomicMax(&p.amax[(size_t)row * p.ngo + cgrp[h]], __float_as_uint(gmax[h]));
     }
 
     tc_fence_before();
@@ -438,9 +509,8 @@ cudaError_t launch_cfg(const GemmArgs& a, const Maps& m, int num_sms, cudaStream
     auto kern = hadamard_tc_kernel<BN, MODE, DUMP>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    const int grid = a.num_units < num_sms ? a.num_units : num_sms;
-    kern<<<grid, Cfg::kThreads, smem, st>>>(m.a, m.b, m.sv, m.su, a);
-    return cudaGetLastError();
+    const int grid = a.num_units < num_sms ? a.num_units : num_sms;   // every CTA gets at least one tap-unit
+    return launch_dependent(kern, dim3(grid), dim3(Cfg::kThreads), smem, st, m.a, m.b, m.sv, m.su, a);
 }
 
 template <int BN>
@@ -473,14 +543,15 @@ bool make_tensor_map(CUtensorMap* map, CUtensorMapDataType dt, int rank, const v
 }
 
 int tc_block_n(int Cout, int G) {
-    if (Cout % 128 == 0 && (128 % G == 0 || G == 256)) return 128;
     if (Cout % 64 == 0) return 64;
     if (Cout % 32 == 0 && G == 32) return 32;
     return 0;
 }
 
 // Stage shape: SK bytes of K (a multiple of G dividing Cin, at most NACC/2
-// groups), swizzle width BK dividing SK, and TPS taps when SK == Cin.
+// groups so that at least two accumulator slots exist), swizzle width BK
+// dividing SK, and TPS taps per stage when SK == Cin (as many as keep three
+// stages in the shared-memory budget).
 static void choose_stage(GemmArgs& a, int BN) {
     const int nacc = std::min(512 / BN, kMaxNacc);
     const int max_groups = nacc / 2;
@@ -493,17 +564,16 @@ static void choose_stage(GemmArgs& a, int BN) {
     a.SK = sk;
     a.BK = sk % 128 == 0 ? 128 : (sk % 64 == 0 ? 64 : 32);
     const int gps = sk / a.G;
+    const size_t budget = 200 * 1024;
+    const size_t per_tap = (size_t)sk * (kBM + BN) + (size_t)gps * (kBM + BN) * 4;
     a.tps = 1;
     if (sk == a.Cin)
-        for (int t : {4, 2})
-            if (t * gps <= max_groups && a.n2 % t == 0) {
+        for (int t : {8, 4, 2})
+            if (t <= a.n2 && budget / (per_tap * t) >= 3) {
                 a.tps = t;
                 break;
             }
-    const size_t per_stage = (size_t)a.tps * sk * (kBM + BN) + (size_t)a.tps * gps * (kBM + BN) * 4;
-    while (a.tps > 1 && (200 * 1024) / per_stage < 3) a.tps /= 2;
-    const size_t ps = (size_t)a.tps * sk * (kBM + BN) + (size_t)a.tps * gps * (kBM + BN) * 4;
-    const int stages = (int)((200 * 1024) / ps);
+    const int stages = (int)(budget / (per_tap * a.tps));
     a.stages = stages > kMaxStages ? kMaxStages : (stages < 2 ? 2 : stages);
 }
 
@@ -516,15 +586,7 @@ cudaError_t launch_hadamard_tc(GemmArgs a, const int8_t* Vq, const int8_t* Uq, i
     choose_stage(a, BN);
     a.num_mb = (a.T + kBM - 1) / kBM;
     a.num_nb = a.Cout / BN;
-    // tap chunking: enough units to fill the SMs a few times over; chunks are whole stages of taps
-    const int base = a.num_mb * a.num_nb;
-    int tpu = a.n2;
-    while (tpu > a.tps && (tpu / 2) % a.tps == 0 && (long)base * ((a.n2 + tpu - 1) / tpu) < 4L * num_sms)
-        tpu /= 2;
-    if (tpu % a.tps) tpu = a.tps;
-    a.tpu = tpu;
-    a.num_tc = (a.n2 + tpu - 1) / tpu;
-    a.num_units = base * a.num_tc;
+    a.num_units = a.num_mb * a.num_nb * a.n2;   // tap-units, split evenly over the CTAs
 
     Maps m;
     const CUtensorMapSwizzle sw = swizzle_for(a.BK);
@@ -556,7 +618,6 @@ cudaError_t launch_hadamard_tc(GemmArgs a, const int8_t* Vq, const int8_t* Uq, i
             return cudaErrorInvalidValue;
     }
     if (launches) ++*launches;
-    if (BN == 128) return launch_bn<128>(a, m, mode, num_sms, st);
     if (BN == 64) return launch_bn<64>(a, m, mode, num_sms, st);
     return launch_bn<32>(a, m, mode, num_sms, st);
 }

@@ -64,6 +64,8 @@ __global__ void __launch_bounds__(G* TX) input_transform_kernel(const __grid_con
     __shared__ int load_ok;
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    grid_dependents_launch();
+    grid_dependency_wait();
     const int row_id = blockIdx.y;  // img * TH + ty
     const int img = row_id / p.TH, ty = row_id - img * p.TH;
     const int tl = warp / WPT;
@@ -206,8 +208,7 @@ cudaError_t launch_g(const InputArgs& a, const TransformArgs& tf, cudaStream_t s
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Cfg::kSmem);
     if (e != cudaSuccess) return e;
     dim3 grid((a.TW + TX - 1) / TX, a.N * a.TH, a.Cin / G);
-    kern<<<grid, G * TX, Cfg::kSmem, st>>>(tm, a, tf);
-    return cudaGetLastError();
+    return launch_dependent(kern, grid, dim3(G * TX), Cfg::kSmem, st, tm, a, tf);
 }
 
 template <int M, uint64_t MASK, typename Tin>

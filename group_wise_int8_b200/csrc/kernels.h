@@ -8,6 +8,33 @@
 
 namespace wino {
 
+// Programmatic dependent launch: every per-call kernel is launched with the
+// programmatic stream-serialisation attribute, so its CTAs may be scheduled
+// while the previous kernel of the stream drains.  Each such kernel calls
+// grid_dependency_wait() before its first global-memory access (it returns once
+// the previous grid has completed and its writes are visible) and
+// grid_dependents_launch() to let the next kernel be scheduled.  Launched
+// without the attribute (or after a kernel that never triggers), both are
+// ordinary stream order.
+__device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void grid_dependents_launch() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+template <typename... KArgs, typename... Args>
+cudaError_t launch_dependent(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                             Args&&... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, static_cast<Args&&>(args)...);
+}
+
 // Encodes a tiled TMA tensor map (rank 2..5; strides in bytes for dims 1..rank-1,
 // no interleave, no L2 promotion change beyond 256 B, zero fill out of bounds).
 bool make_tensor_map(CUtensorMap* map, CUtensorMapDataType dt, int rank, const void* base, const cuuint64_t* dims,
@@ -39,7 +66,7 @@ enum GemmMode { kModeAbsmax = 0, kModeQuant = 1, kModeY32 = 2 };
 
 struct GemmArgs {
     int T, T_pad, Cin, Cout, n2, G, ng, ngo;
-    int SK, BK, tps, stages, tpu, num_tc, num_mb, num_nb, num_units;  // stage shape and work split (set by the launcher)
+    int SK, BK, tps, stages, num_mb, num_nb, num_units;  // stage shape and work split (set by the launcher)
     const float* sV;   // [n2][ng][T_pad]
     const float* sU;   // [n2][ng][Cout]
     unsigned* amax;    // [T_pad][ngo] fp32 bits of |Y| maxima

@@ -19,6 +19,8 @@ namespace {
 template <int M, uint64_t MASK, bool SRC_Y32, bool BF16_OUT, bool DEBUG>
 __global__ void __launch_bounds__(256) output_transform_kernel(OutputArgs p, TransformArgs tf) {
     constexpr int N = M + 2, N2 = N * N;
+    grid_dependents_launch();
+    grid_dependency_wait();
     const long i = (long)blockIdx.x * blockDim.x + threadIdx.x;
     const long t = i / p.Cout;
     const int co = (int)(i - t * p.Cout);
@@ -87,7 +89,8 @@ cudaError_t launch_m(const OutputArgs& a, const TransformArgs& tf, bool src_y32,
                      cudaStream_t st) {
     const long threads = a.T * (long)a.Cout;
     const dim3 grid((unsigned)((threads + 255) / 256));
-#define WINO_OUT_LAUNCH(Y32, BF, DBG) output_transform_kernel<M, MASK, Y32, BF, DBG><<<grid, 256, 0, st>>>(a, tf)
+#define WINO_OUT_LAUNCH(Y32, BF, DBG) \
+    return launch_dependent(output_transform_kernel<M, MASK, Y32, BF, DBG>, grid, dim3(256), 0, st, a, tf)
     if (src_y32) {
         if (bf16_out) {
             if (debug) WINO_OUT_LAUNCH(true, true, true); else WINO_OUT_LAUNCH(true, true, false);
@@ -102,7 +105,7 @@ cudaError_t launch_m(const OutputArgs& a, const TransformArgs& tf, bool src_y32,
         }
     }
 #undef WINO_OUT_LAUNCH
-    return cudaGetLastError();
+    return cudaErrorInvalidValue;  // not reached
 }
 
 }  // namespace
