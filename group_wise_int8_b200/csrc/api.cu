@@ -277,6 +277,16 @@ int wino_plan(wino_plan_t* out, int m, const double* points, const float* S_B, c
     std::memset(&p->tf, 0, sizeof(p->tf));
     std::memcpy(p->tf.BT, p->mat.BT, sizeof(float) * n * n);
     std::memcpy(p->tf.AT, p->mat.AT, sizeof(float) * m * n);
+    for (int i = 0; i < n * n; ++i) {
+        uint32_t b;
+        std::memcpy(&b, &p->mat.BT[i], 4);
+        p->tf.BTd[i] = ((uint64_t)b << 32) | b;
+    }
+    for (int i = 0; i < m * n; ++i) {
+        uint32_t b;
+        std::memcpy(&b, &p->mat.AT[i], 4);
+        p->tf.ATd[i] = ((uint64_t)b << 32) | b;
+    }
     std::memcpy(p->wa.G, p->mat.G, sizeof(double) * n * 3);
     const uint64_t bt_mask = m == 4 ? kMaskBT_F4 : kMaskBT_F6;
     const uint64_t at_mask = m == 4 ? kMaskAT_F4 : kMaskAT_F6;

@@ -19,10 +19,13 @@ constexpr uint64_t kMaskBT_F6 = 0xaa7e7e7e7e7e7e55ull;
 constexpr uint64_t kMaskAT_F6 = 0x0000fe7e7e7e7e7full;
 constexpr uint64_t kMaskAll = ~0ull;
 
-// The fp32 transforms as kernel arguments (they live in the constant bank).
+// The fp32 transforms as kernel arguments (they live in the constant bank),
+// also as packed pairs (c, c) for the two-lane fp32 instructions.
 struct TransformArgs {
     float BT[kMaxN * kMaxN];
     float AT[6 * kMaxN];
+    uint64_t BTd[kMaxN * kMaxN];
+    uint64_t ATd[6 * kMaxN];
 };
 
 struct WeightArgs {
