@@ -97,6 +97,13 @@ __device__ __forceinline__ QScale make_qscale(float amax) {
     return q;
 }
 
+// max(a, |b|, |c|) in one three-input max (exact, like any max).
+__device__ __forceinline__ float max_abs3(float a, float b, float c) {
+    float r;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(fabsf(b)), "f"(fabsf(c)));
+    return r;
+}
+
 // The same code as quant_code(v, s) without a division or a branch.
 // RN24(v/s) = (float)((double)v * RN53(1/s)) for fp32 v and s > 0: the exact
 // quotient of two 24-bit numbers is never an fp32 rounding midpoint and lies at

@@ -62,13 +62,6 @@ struct TcCfg {
                                      : (kNacc * BN) <= 256 ? 256 : 512;
 };
 
-// max(a, |b|, |c|) in one three-input max (exact, like any max).
-__device__ __forceinline__ float max_abs3(float a, float b, float c) {
-    float r;
-    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(fabsf(b)), "f"(fabsf(c)));
-    return r;
-}
-
 struct SmemTail {
     uint64_t full[kMaxStages];
     uint64_t empty[kMaxStages];

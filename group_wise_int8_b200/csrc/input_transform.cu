@@ -1,6 +1,6 @@
 // Input transform with group-wise int8 quantisation ("Data-Free Group-Wise
-// Fully Quantized Winograd Convolution via Learnable Scales", Fig. 2: the
-// input transform B^T d B is group-wise quantised).
+// Fully Quantized Winograd Convolution via Learnable Scales", Fig. 2: the input
+// transform B^T d B is group-wise quantised).
 //
 // Tile t = (img*TH + ty)*TW + tx reads rows ty*m-1 .. ty*m+m and columns
 // tx*m-1 .. tx*m+m of the NHWC input (zeros outside: stride 1, pad 1) and
@@ -10,17 +10,20 @@
 //   exact-zero coefficients are skipped, which can change only the sign of a zero).
 // Q then runs over G consecutive channels at fixed (tile, tap).
 //
-// CTA: TX consecutive tiles of one tile row x one quantisation group of G
-// channels (128 threads, 256 for G = 256); one thread per (tile, channel),
-// lanes along channels.  One 4-D TMA box brings the CTA's halo patch
-// (n rows x TX*m+2 columns x G channels; outside the image the box reads
-// zeros, which is the pad-1 border) into shared memory; each thread reads its
-// n x n patch from there and transforms it in registers.  V then goes to
-// shared memory (rows padded to 36 words: 16-byte reads without bank
-// conflicts), where lane l of the warp owns taps l and l + 32: it takes their
-// absmax over the warp's 32 channels (the G/32 warps of a group combine theirs
-// in shared memory), the group scale, and the 32 codes of each of its taps
-// (quant4), packed into two 16-byte stores of the tap-major Vq.
+// CTA: TX consecutive tiles of one tile row (TX = TW, or a balanced share of
+// a long row) and one quantisation group of G channels; each thread owns one
+// tile and a pair of adjacent channels, so both chains run as one two-lane
+// fp32 instruction per step (the per-channel chains are unchanged).  One 4-D
+// TMA box brings the CTA's halo patch (n rows x TX*m+2 columns x G channels;
+// outside the image the box reads zeros, which is the pad-1 border) into
+// shared memory.  V goes to shared memory half the taps at a time, a
+// [tap][64 channels] block per warp (rows padded to 68 words: conflict-free
+// 16-byte reads), where lane l owns one tap of each 32-channel chunk: its
+// absmax (the chunks of one group combine in registers, or in shared memory
+// across warps for G > 64), the group scale, and the 32 codes (quant4),
+// written as two 16-byte stores of the tap-major Vq.
+#include <algorithm>
+
 #include "kernels.h"
 #include "sm100.cuh"
 
@@ -28,60 +31,63 @@ namespace wino {
 namespace {
 
 template <typename T>
-__device__ __forceinline__ float to_float(T v);
+struct Pair;
 template <>
-__device__ __forceinline__ float to_float<float>(float v) {
-    return v;
-}
+struct Pair<uint16_t> {   // bf16 x 2 -> fp32 x 2 (exact)
+    static __device__ __forceinline__ uint64_t load(const uint16_t* p) {
+        const uint32_t x = *reinterpret_cast<const uint32_t*>(p);
+        return f2_pack(__uint_as_float(x << 16), __uint_as_float(x & 0xffff0000u));
+    }
+};
 template <>
-__device__ __forceinline__ float to_float<uint16_t>(uint16_t v) {
-    return bf16_bits_to_float(v);
-}
-
-template <int M, typename Tin, int G, int TX>
-struct InCfg {
-    static constexpr int N = M + 2, N2 = N * N;
-    static constexpr int kPitch = 36;                   // words per V row in shared memory
-    static constexpr int kNW = TX * G / 32;             // warps per CTA
-    static constexpr int kPW = TX * M + 2;              // patch columns
-    static constexpr size_t kPatchBytes = sizeof(Tin) * N * kPW * G;
-    static constexpr size_t kPatchOff = 0;
-    static constexpr size_t kVbufOff = (kPatchBytes + 127) / 128 * 128;
-    static constexpr size_t kSmem = kVbufOff + sizeof(float) * kNW * N2 * kPitch;
+struct Pair<float> {
+    static __device__ __forceinline__ uint64_t load(const float* p) { return *reinterpret_cast<const uint64_t*>(p); }
 };
 
-template <int M, uint64_t MASK, typename Tin, int G, int TX>
-__global__ void __launch_bounds__(G* TX) input_transform_kernel(const __grid_constant__ CUtensorMap tmX, InputArgs p,
-                                                                TransformArgs tf) {
-    using Cfg = InCfg<M, Tin, G, TX>;
-    constexpr int N = M + 2, N2 = N * N, P = Cfg::kPitch, PW = Cfg::kPW;
-    constexpr int WPT = G / 32;      // warps per tile (= per group)
+template <int M, typename Tin, int G>
+struct InCfg {
+    static constexpr int N = M + 2, N2 = N * N, H2 = N2 / 2;   // taps per half
+    static constexpr int kMaxThreads = 256;
+    static constexpr int kPitch = 68;                   // words per V row in shared memory (64 channels + pad)
+    static constexpr int kMaxWarps = kMaxThreads / 32;
+    static constexpr size_t kVbufBytes = sizeof(float) * kMaxWarps * H2 * kPitch;
+    __host__ __device__ static size_t patch_bytes(int tx) { return sizeof(Tin) * N * (size_t)(tx * M + 2) * G; }
+    __host__ __device__ static int threads(int tx) { return (tx * (G / 2) + 31) / 32 * 32; }
+    // the V blocks reuse the patch's shared memory once every thread holds its patch values
+    __host__ __device__ static size_t smem(int tx) {
+        const size_t v = sizeof(float) * (threads(tx) / 32) * H2 * kPitch;
+        return patch_bytes(tx) > v ? patch_bytes(tx) : v;
+    }
+};
+
+template <int M, uint64_t MASK, typename Tin, int G>
+// at most 168 registers: two CTAs of a 10-tile row (160 threads) share an SM
+__global__ void __maxnreg__(MASK == kMaskAll ? 255 : 168)
+    input_transform_kernel(const __grid_constant__ CUtensorMap tmX, InputArgs p, TransformArgs tf, int TX) {
+    using Cfg = InCfg<M, Tin, G>;
+    constexpr int N = M + 2, N2 = N * N, H2 = Cfg::H2, P = Cfg::kPitch;
+    constexpr int CPW = G <= 64 ? 1 : G / 64;    // warps per group (G > 64)
     extern __shared__ __align__(128) unsigned char smem[];
-    const Tin* patch = reinterpret_cast<const Tin*>(smem + Cfg::kPatchOff);   // [N][PW][G]
-    float* vbuf = reinterpret_cast<float*>(smem + Cfg::kVbufOff);            // [NW][N2][P]
-    __shared__ float red[Cfg::kNW][64];
+    const Tin* patch = reinterpret_cast<const Tin*>(smem);   // [N][PW][G]
+    float* vbuf = reinterpret_cast<float*>(smem);             // [warps][H2][P], after the patch is consumed
+    __shared__ float red[Cfg::kMaxWarps][32];
     __shared__ uint64_t bar;
     __shared__ int load_ok;
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     grid_dependents_launch();
     grid_dependency_wait();
+    const int PW = TX * M + 2;
     const int row_id = blockIdx.y;  // img * TH + ty
     const int img = row_id / p.TH, ty = row_id - img * p.TH;
-    const int tl = warp / WPT;
     const int tx0 = blockIdx.x * TX;
-    const int tx = tx0 + tl;
-    const bool valid = tx < p.TW;
     const int g = blockIdx.z;
-    const int cl = (warp % WPT) * 32;  // first channel of this warp within the group
-    const int cw = g * G + cl;
-    const long t = (long)row_id * p.TW + tx;
 
     if (tid == 0) {
         sm100::mbar_init(&bar, 1);
         sm100::fence_mbar_init();
-        sm100::mbar_arrive_expect_tx(&bar, (uint32_t)Cfg::kPatchBytes);
-        sm100::tma_load_4d(smem + Cfg::kPatchOff, &tmX, &bar, g * G, tx0 * M - 1, ty * M - 1, img);
+        sm100::mbar_arrive_expect_tx(&bar, (uint32_t)Cfg::patch_bytes(TX));
+        sm100::tma_load_4d(smem, &tmX, &bar, g * G, tx0 * M - 1, ty * M - 1, img);
     }
     if (blockIdx.x == 0 && blockIdx.y == 0 && g == 0 && tid == 0) *p.err = 0;
     if (g == 0)
@@ -102,89 +108,96 @@ __global__ void __launch_bounds__(G* TX) input_transform_kernel(const __grid_con
     __syncthreads();
     if (!load_ok) return;   // uniform across the CTA; the host reads the error word
 
-    {
-        // 1.-2. the n x n patch of channel cw + lane, V = B^T d B
-        float v[N][N];
+    // 1. this thread's tile and channel pair (threads past the CTA's tiles read tile 0 and store nothing)
+    const int tl = tid / (G / 2) < TX ? tid / (G / 2) : 0;   // tile within the CTA
+    const int cp = 2 * (tid % (G / 2));                       // first channel of the pair within the group
+    uint64_t v[N][N];
 #pragma unroll
-        for (int r = 0; r < N; ++r)
+    for (int r = 0; r < N; ++r)
 #pragma unroll
-            for (int l = 0; l < N; ++l) v[r][l] = to_float<Tin>(patch[(r * PW + tl * M + l) * G + cl + lane]);
+        for (int l = 0; l < N; ++l) v[r][l] = Pair<Tin>::load(patch + (r * PW + tl * M + l) * G + cp);
+    __syncthreads();   // the patch is consumed; its shared memory now holds the V blocks
+    // 2. T1 = B^T d, in place, column by column
 #pragma unroll
-        for (int l = 0; l < N; ++l) {
-            float tcol[N];
-#pragma unroll
-            for (int i = 0; i < N; ++i) {
-                float acc = 0.0f;
-#pragma unroll
-                for (int k = 0; k < N; ++k)
-                    if ((MASK >> (i * N + k)) & 1ull) acc = __fmaf_rn(tf.BT[i * N + k], v[k][l], acc);
-                tcol[i] = acc;
-            }
-#pragma unroll
-            for (int i = 0; i < N; ++i) v[i][l] = tcol[i];
-        }
-        float* vw = vbuf + (size_t)warp * N2 * P;
+    for (int l = 0; l < N; ++l) {
+        uint64_t tcol[N];
 #pragma unroll
         for (int i = 0; i < N; ++i) {
+            uint64_t acc = 0ull;
+#pragma unroll
+            for (int k = 0; k < N; ++k)
+                if ((MASK >> (i * N + k)) & 1ull) acc = f2_fma(tf.BTd[i * N + k], v[k][l], acc);
+            tcol[i] = acc;
+        }
+#pragma unroll
+        for (int i = 0; i < N; ++i) v[i][l] = tcol[i];
+    }
+    float* vw = vbuf + (size_t)warp * H2 * P;
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        // 3. V = T1 B for the rows of this half: taps h*H2 .. h*H2 + H2 - 1
+        if (h) __syncwarp();   // the previous half's codes are written
+#pragma unroll
+        for (int i = h * N / 2; i < (h + 1) * N / 2; ++i) {
 #pragma unroll
             for (int j = 0; j < N; ++j) {
-                float acc = 0.0f;
+                uint64_t acc = 0ull;
 #pragma unroll
                 for (int l = 0; l < N; ++l)
-                    if ((MASK >> (j * N + l)) & 1ull) acc = __fmaf_rn(v[i][l], tf.BT[j * N + l], acc);
-                vw[(i * N + j) * P + lane] = acc;   // 3. V row of tap (i, j), this lane's channel
+                    if ((MASK >> (j * N + l)) & 1ull) acc = f2_fma(v[i][l], tf.BTd[j * N + l], acc);
+                *reinterpret_cast<uint64_t*>(vw + (i * N + j - h * H2) * P + 2 * lane) = acc;
             }
         }
-    }
-    __syncwarp();
+        __syncwarp();
 
-    // 4. absmax of this lane's taps over the warp's 32 channels
-    const float* vw = vbuf + (size_t)warp * N2 * P;
-    float am[2] = {0.0f, 0.0f};
+        // 4. absmax of this lane's tap over each 32-channel chunk of the warp
+        const bool own = lane < H2;
+        const int tap = h * H2 + lane;
+        const float* vrow = vw + (own ? lane : 0) * P;
+        float am[2] = {0.0f, 0.0f};
 #pragma unroll
-    for (int e = 0; e < 2; ++e) {
-        const int tap = lane + 32 * e;
-        if (tap < N2) {
-            const float4* row = reinterpret_cast<const float4*>(vw + tap * P);
-            float a = 0.0f;
+        for (int c = 0; c < 2; ++c) {
+            const float4* row = reinterpret_cast<const float4*>(vrow + 32 * c);
 #pragma unroll
             for (int j = 0; j < 8; ++j) {
-                const float4 q = row[j];
-                a = fmaxf(a, fmaxf(fmaxf(fabsf(q.x), fabsf(q.y)), fmaxf(fabsf(q.z), fabsf(q.w))));
+                const float4 x4 = row[j];
+                am[c] = max_abs3(am[c], x4.x, x4.y);
+                am[c] = max_abs3(am[c], x4.z, x4.w);
             }
-            am[e] = a;
         }
-    }
-    if (WPT > 1) {
-        red[warp][lane] = am[0];
-        red[warp][lane + 32] = am[1];
-        __syncthreads();
-        const int leader = warp - warp % WPT;
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
+        // group maxima: G = 32: one chunk; G = 64: the warp's two chunks; G > 64: CPW warps
+        if (G == 64) {
+            am[0] = am[1] = fmaxf(am[0], am[1]);
+        } else if (G > 64) {
+            red[warp][lane] = fmaxf(am[0], am[1]);
+            __syncthreads();
+            const int leader = warp - warp % CPW;
             float a = 0.0f;
 #pragma unroll
-            for (int i = 0; i < WPT; ++i) a = fmaxf(a, red[leader + i][lane + 32 * e]);
-            am[e] = a;
+            for (int i = 0; i < CPW; ++i) a = fmaxf(a, red[leader + i][lane]);
+            am[0] = am[1] = a;
+            __syncthreads();   // red is reused by the next half
         }
-    }
 
-    // 5. scales and codes of this lane's taps
-    if (valid) {
+        // 5. scales and codes, chunk by chunk
 #pragma unroll
-        for (int e = 0; e < 2; ++e) {
-            const int tap = lane + 32 * e;
-            if (tap >= N2) continue;
-            const QScale q = make_qscale(am[e]);
-            if (warp % WPT == 0) p.sV[((size_t)tap * (p.Cin / G) + g) * p.T_pad + t] = q.s;
-            const float4* row = reinterpret_cast<const float4*>(vw + tap * P);
+        for (int c = 0; c < 2; ++c) {
+            const int th = warp * 32 + 16 * c;     // first thread of the chunk
+            const int ctl = th / (G / 2);          // its tile
+            const int ch = 2 * (th % (G / 2));     // its first channel within the group
+            const int tx = tx0 + ctl;
+            if (!own || ctl >= TX || tx >= p.TW) continue;
+            const long t = (long)row_id * p.TW + tx;
+            const QScale q = make_qscale(am[c]);
+            if (ch == 0) p.sV[((size_t)tap * (p.Cin / G) + g) * p.T_pad + t] = q.s;
+            const float4* row = reinterpret_cast<const float4*>(vrow + 32 * c);
             uint32_t w[8];
 #pragma unroll
             for (int j = 0; j < 8; ++j) {
                 const float4 x4 = row[j];
                 w[j] = quant4(x4.x, x4.y, x4.z, x4.w, q).packed;
             }
-            uint4* dst = reinterpret_cast<uint4*>(p.Vq + ((size_t)tap * p.T_pad + t) * p.Cin + cw);
+            uint4* dst = reinterpret_cast<uint4*>(p.Vq + ((size_t)tap * p.T_pad + t) * p.Cin + g * G + ch);
             dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
             dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
         }
@@ -193,22 +206,26 @@ __global__ void __launch_bounds__(G* TX) input_transform_kernel(const __grid_con
 
 template <int M, uint64_t MASK, typename Tin, int G>
 cudaError_t launch_g(const InputArgs& a, const TransformArgs& tf, cudaStream_t st) {
-    constexpr int TX = G >= 128 ? 1 : 128 / G;
-    using Cfg = InCfg<M, Tin, G, TX>;
+    using Cfg = InCfg<M, Tin, G>;
+    // tiles per CTA: the whole tile row when it fits, else the row split into equal shares
+    const int max_tx = std::min(Cfg::kMaxThreads / (G / 2), (256 - 2) / M);
+    const int nblk = (a.TW + max_tx - 1) / max_tx;
+    const int TX = (a.TW + nblk - 1) / nblk;
     // x [N][H][W][Cin] as a 4-D tensor (Cin, W, H, N); box G x (TX*m+2) x n x 1
     CUtensorMap tm;
     const cuuint64_t es = sizeof(Tin);
     const cuuint64_t dims[4] = {(cuuint64_t)a.Cin, (cuuint64_t)a.W, (cuuint64_t)a.H, (cuuint64_t)a.N};
     const cuuint64_t strides[3] = {es * a.Cin, es * a.Cin * a.W, es * a.Cin * a.W * a.H};
-    const cuuint32_t box[4] = {(cuuint32_t)G, (cuuint32_t)Cfg::kPW, (cuuint32_t)Cfg::N, 1u};
+    const cuuint32_t box[4] = {(cuuint32_t)G, (cuuint32_t)(TX * M + 2), (cuuint32_t)Cfg::N, 1u};
     if (!make_tensor_map(&tm, sizeof(Tin) == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4,
                          a.x, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_NONE))
         return cudaErrorInvalidValue;
-    auto kern = input_transform_kernel<M, MASK, Tin, G, TX>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Cfg::kSmem);
+    auto kern = input_transform_kernel<M, MASK, Tin, G>;
+    const size_t smem = Cfg::smem(TX);
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    dim3 grid((a.TW + TX - 1) / TX, a.N * a.TH, a.Cin / G);
-    return launch_dependent(kern, grid, dim3(G * TX), Cfg::kSmem, st, tm, a, tf);
+    const dim3 grid(nblk, a.N * a.TH, a.Cin / G);
+    return launch_dependent(kern, grid, dim3(Cfg::threads(TX)), smem, st, tm, a, tf, TX);
 }
 
 template <int M, uint64_t MASK, typename Tin>
