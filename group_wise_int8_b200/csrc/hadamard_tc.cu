@@ -55,7 +55,7 @@ template <int BN>
 struct TcCfg {
     static constexpr int kCPT = BN / 4;       // columns per column chunk
     static constexpr int kPasses = 2;         // column chunks per epilogue thread
-    static constexpr int kEpiWarps = 8;       // 4 TMEM lane quadrants x 2 chunk pairs
+    static constexpr int kEpiWarps = 16 / kPasses;   // 4 TMEM lane quadrants x (4 / kPasses) chunk sets
     static constexpr int kThreads = 64 + 32 * kEpiWarps;
     static constexpr int kNacc = (512 / BN) < kMaxNacc ? (512 / BN) : kMaxNacc;
     static constexpr int kTmemCols = (kNacc * BN) <= 32 ? 32 : (kNacc * BN) <= 64 ? 64 : (kNacc * BN) <= 128 ? 128
@@ -288,14 +288,14 @@ __global__ void __launch_bounds__(TcCfg<BN>::kThreads, 1)
     } else {
         // ----------------------------------------------------------- epilogue
         // Thread (quad, lane) of epilogue warp ew owns row 32*quad + lane and the
-        // column chunks (ew >> 2) + 2h, h = 0, 1, of CPT columns each, handled in turn.
+        // column chunks (ew >> 2) + (4 / NP) h, h < NP, of CPT columns each.
         constexpr int CPT = Cfg::kCPT, NP = Cfg::kPasses;
         const int ew = warp - 2;
         const int quad = warp & 3;                    // TMEM lanes 32*quad .. 32*quad+31
         const int rloc = 32 * quad + lane;            // row within the 128-tile block
         int col0[NP];
 #pragma unroll
-        for (int h = 0; h < NP; ++h) col0[h] = ((ew >> 2) + 2 * h) * CPT;
+        for (int h = 0; h < NP; ++h) col0[h] = ((ew >> 2) + (4 / NP) * h) * CPT;
         const uint32_t t_lane = tmem_base + ((uint32_t)(32 * quad) << 16);
         const uint64_t neg_magic2 = f2_pack(-kRoundMagic, -kRoundMagic);
 
@@ -368,33 +368,29 @@ __global__ void __launch_bounds__(TcCfg<BN>::kThreads, 1)
                             for (int c = 0; c < CPT / 2; ++c) y2[h][c] = 0ull;
                     }
                     const uint32_t t_slot = t_lane + (uint32_t)(sl.idx * GPS * BN);
+                    for (int j = 0; j < GPS; ++j) {
+                        // one group per round, both chunks' loads in flight at once
+                        uint32_t r[NP][CPT];
 #pragma unroll
-                    for (int h = 0; h < NP; ++h)
-                        for (int j = 0; j < GPS; ++j) {
-                            // one chunk of one group at a time; after the slot's last load, refill and release it
-                            uint32_t r[CPT];
-                            tmem_ld<CPT>(t_slot + (uint32_t)(j * BN + col0[h]), r);
-                            tmem_ld_wait();
-                            if (h + 1 == NP && j + 1 == GPS) {
-                                for (int b = 0; b < GPS; ++b)
+                        for (int h = 0; h < NP; ++h) tmem_ld<CPT>(t_slot + (uint32_t)(j * BN + col0[h]), r[h]);
+                        tmem_ld_wait();
+                        if (j + 1 == GPS)   // the slot is read: refill it with the bias (completion awaited below)
+                            for (int b = 0; b < GPS; ++b)
 #pragma unroll
-                                    for (int hh = 0; hh < NP; ++hh)
-                                        tmem_fill<CPT>(t_slot + (uint32_t)(b * BN + col0[hh]), (uint32_t)kRoundMagicBits);
-                                tmem_st_wait();
-                                tc_fence_before();
-                                __syncwarp();
-                                if (lane == 0) mbar_arrive(&tail->acc_empty[sl.idx]);
-                            }
-                            const float sv = svs[(t * GPS + j) * kBM];
-                            const uint64_t sv2 = f2_pack(sv, sv);
+                                for (int h = 0; h < NP; ++h)
+                                    tmem_fill<CPT>(t_slot + (uint32_t)(b * BN + col0[h]), (uint32_t)kRoundMagicBits);
+                        const float sv = svs[(t * GPS + j) * kBM];
+                        const uint64_t sv2 = f2_pack(sv, sv);
+#pragma unroll
+                        for (int h = 0; h < NP; ++h) {
                             const float4* su4 = reinterpret_cast<const float4*>(sus + (t * GPS + j) * BN + col0[h]);
 #pragma unroll
                             for (int c4 = 0; c4 < CPT / 4; ++c4) {
                                 const float4 uu = su4[c4];
                                 const uint64_t a0 = f2_add(
-                                    f2_pack(__uint_as_float(r[4 * c4 + 0]), __uint_as_float(r[4 * c4 + 1])), neg_magic2);
+                                    f2_pack(__uint_as_float(r[h][4 * c4 + 0]), __uint_as_float(r[h][4 * c4 + 1])), neg_magic2);
                                 const uint64_t a1 = f2_add(
-                                    f2_pack(__uint_as_float(r[4 * c4 + 2]), __uint_as_float(r[4 * c4 + 3])), neg_magic2);
+                                    f2_pack(__uint_as_float(r[h][4 * c4 + 2]), __uint_as_float(r[h][4 * c4 + 3])), neg_magic2);
                                 y2[h][2 * c4 + 0] = f2_fma(a0, f2_mul(sv2, f2_pack(uu.x, uu.y)), y2[h][2 * c4 + 0]);
                                 y2[h][2 * c4 + 1] = f2_fma(a1, f2_mul(sv2, f2_pack(uu.z, uu.w)), y2[h][2 * c4 + 1]);
                             }
@@ -403,9 +399,15 @@ __global__ void __launch_bounds__(TcCfg<BN>::kThreads, 1)
 #pragma unroll
                                 for (int c = 0; c < CPT; ++c)
                                     p.acc[(((size_t)tap * p.T + row) * p.Cout + colg[h] + c) * p.ng + jg] =
-                                        (int)r[c] - kRoundMagicBits;
+                                        (int)r[h][c] - kRoundMagicBits;
                             }
                         }
+                    }
+                    // the refill is complete: release the slot
+                    tmem_st_wait();
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&tail->acc_empty[sl.idx]);
                     sl.next(NSLOT);
                     if (ks + 1 < KSTAGES) continue;
                     // ---- end of tap
