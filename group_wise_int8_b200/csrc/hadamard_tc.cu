@@ -17,22 +17,23 @@
 //            stage's groups;
 //   warp 0 = TMA producer;
 //   warp 1 = TMEM allocator and MMA issuer: tcgen05.mma kind::i8, M=128,
-//            N=BN, K=32 per instruction; each K-group of a stage accumulates
-//            into its own BN-column TMEM buffer; the buffers of one stage form
-//            a slot, a ring of at least two slots lets the MMAs of the next
-//            stage overlap the epilogue of this one; one wait for a free slot
-//            and one commit per stage;
-//   warps 2..9 = epilogue, 4 TMEM lane quadrants x 2 pairs of column chunks
-//            of BN/4: per tap one wait, then per chunk and group a tcgen05.ld and the
-//            dequantisation in packed fp32 pairs; the buffers are refilled with
-//            the bias 0x4B400000 (so the next int32 sum lands on 1.5*2^23 and
-//            reinterprets as an exact fp32 value) and the slot is released.  A
-//            stage's shared memory returns to the producer when every epilogue
-//            warp is done with it (which is after its MMAs completed).
+//            N=BN, K=32 per instruction; each K-group of a tap accumulates into
+//            its own BN-column TMEM buffer (its first K-step overwrites); the
+//            buffers of one tap form a slot, a ring of at least two slots lets
+//            the MMAs run ahead of the epilogue; one wait for a free slot and
+//            one commit per tap;
+//   warps 2..9 = epilogue, 4 TMEM lane quadrants x 2 column chunks of BN/4:
+//            per tap one wait, then per group both chunks' tcgen05.ld, one
+//            wait, the slot released as soon as it is read (TMEM to register
+//            traffic is the epilogue's bottleneck, so nothing is written back),
+//            and the dequantisation in packed fp32 pairs, with (float)acc taken
+//            exactly as asfloat(acc + 0x4B400000) - 1.5*2^23.  A stage's shared
+//            memory returns to the producer when every epilogue warp is done
+//            with it (which is after its MMAs completed).
 // The loops keep wrap-around ring counters (no division in the issue paths).
 // At the end of each tap the epilogue either keeps the running |Y| maximum of
 // each (tile, G-cout group) (absmax pass and fp32-Y pass, published with
-// atomicMax on the float bits at the end of the unit), writes fp32 Y, or
+// atomicMax on the float bits when the CTA leaves a block), writes fp32 Y, or
 // requantises Y with sY = absmax/127 and writes int8 Yq.
 // Every mbarrier wait is bounded (%globaltimer); on expiry the CTA raises an
 // abort flag and the device error word, drains its in-flight TMA loads and
@@ -264,7 +265,8 @@ __global__ void __launch_bounds__(TcCfg<BN>::kThreads, 1)
                         for (int kk = 0; kk < ksteps; ++kk) {
                             const uint64_t koff = stage_off + (uint64_t)(((c * TPS + t) * a_tile + kin * 32) >> 4);
                             const uint64_t kofb = stage_off + (uint64_t)(((c * TPS + t) * b_tile + kin * 32) >> 4);
-                            mma_i8(d + (uint32_t)(g * BN), a_desc0 + koff, b_desc0 + kofb, idesc, 1u);
+                            // the first K-step of a group overwrites its buffer, the others accumulate
+                            mma_i8(d + (uint32_t)(g * BN), a_desc0 + koff, b_desc0 + kofb, idesc, gk != 0 ? 1u : 0u);
                             if (++kin == ks_per_chunk) {
                                 kin = 0;
                                 ++c;
@@ -299,13 +301,7 @@ __global__ void __launch_bounds__(TcCfg<BN>::kThreads, 1)
         const uint32_t t_lane = tmem_base + ((uint32_t)(32 * quad) << 16);
         const uint64_t neg_magic2 = f2_pack(-kRoundMagic, -kRoundMagic);
 
-        // every accumulator buffer starts filled with the bias
-        for (int b = 0; b < NSLOT * GPS; ++b)
-#pragma unroll
-            for (int h = 0; h < NP; ++h) tmem_fill<CPT>(t_lane + (uint32_t)(b * BN + col0[h]), (uint32_t)kRoundMagicBits);
-        tmem_st_wait();
-        tc_fence_before();
-        __syncwarp();
+        // every accumulator slot starts free
         if (lane == 0)
             for (int b = 0; b < NSLOT; ++b) mbar_arrive(&tail->acc_empty[b]);
 
@@ -374,11 +370,11 @@ __global__ void __launch_bounds__(TcCfg<BN>::kThreads, 1)
 #pragma unroll
                         for (int h = 0; h < NP; ++h) tmem_ld<CPT>(t_slot + (uint32_t)(j * BN + col0[h]), r[h]);
                         tmem_ld_wait();
-                        if (j + 1 == GPS)   // the slot is read: refill it with the bias (completion awaited below)
-                            for (int b = 0; b < GPS; ++b)
-#pragma unroll
-                                for (int h = 0; h < NP; ++h)
-                                    tmem_fill<CPT>(t_slot + (uint32_t)(b * BN + col0[h]), (uint32_t)kRoundMagicBits);
+                        if (j + 1 == GPS) {   // the slot is read: release it
+                            tc_fence_before();
+                            __syncwarp();
+                            if (lane == 0) mbar_arrive(&tail->acc_empty[sl.idx]);
+                        }
                         const float sv = svs[(t * GPS + j) * kBM];
                         const uint64_t sv2 = f2_pack(sv, sv);
 #pragma unroll
@@ -387,10 +383,13 @@ __global__ void __launch_bounds__(TcCfg<BN>::kThreads, 1)
 #pragma unroll
                             for (int c4 = 0; c4 < CPT / 4; ++c4) {
                                 const float4 uu = su4[c4];
-                                const uint64_t a0 = f2_add(
-                                    f2_pack(__uint_as_float(r[h][4 * c4 + 0]), __uint_as_float(r[h][4 * c4 + 1])), neg_magic2);
-                                const uint64_t a1 = f2_add(
-                                    f2_pack(__uint_as_float(r[h][4 * c4 + 2]), __uint_as_float(r[h][4 * c4 + 3])), neg_magic2);
+                                // (float)acc exactly: acc + 1.5*2^23 in the integer unit, then - 1.5*2^23 (|acc| < 2^22)
+                                const uint64_t a0 = f2_add(f2_pack(__uint_as_float(r[h][4 * c4 + 0] + kRoundMagicBits),
+                                                                   __uint_as_float(r[h][4 * c4 + 1] + kRoundMagicBits)),
+                                                           neg_magic2);
+                                const uint64_t a1 = f2_add(f2_pack(__uint_as_float(r[h][4 * c4 + 2] + kRoundMagicBits),
+                                                                   __uint_as_float(r[h][4 * c4 + 3] + kRoundMagicBits)),
+                                                           neg_magic2);
                                 y2[h][2 * c4 + 0] = f2_fma(a0, f2_mul(sv2, f2_pack(uu.x, uu.y)), y2[h][2 * c4 + 0]);
                                 y2[h][2 * c4 + 1] = f2_fma(a1, f2_mul(sv2, f2_pack(uu.z, uu.w)), y2[h][2 * c4 + 1]);
                             }
@@ -398,16 +397,10 @@ __global__ void __launch_bounds__(TcCfg<BN>::kThreads, 1)
                                 const int jg = ks * GPS + j;
 #pragma unroll
                                 for (int c = 0; c < CPT; ++c)
-                                    p.acc[(((size_t)tap * p.T + row) * p.Cout + colg[h] + c) * p.ng + jg] =
-                                        (int)r[h][c] - kRoundMagicBits;
+                                    p.acc[(((size_t)tap * p.T + row) * p.Cout + colg[h] + c) * p.ng + jg] = (int)r[h][c];
                             }
                         }
                     }
-                    // the refill is complete: release the slot
-                    tmem_st_wait();
-                    tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(&tail->acc_empty[sl.idx]);
                     sl.next(NSLOT);
                     if (ks + 1 < KSTAGES) continue;
                     // ---- end of tap
