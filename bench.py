@@ -63,7 +63,7 @@ def parse():
     ap.add_argument("--steps", type=int, default=3000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--workload", default="resnet18",
-                    help="resnet18 (default) | resnet34:<i> | sd15:<i> | sd15_stack:<i>")
+                    help="resnet18 (default) | resnet34:<i> | sd15:<i> | sd15_stack:<i> | probe:<i>")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=200)

@@ -39,7 +39,7 @@ INF = math.inf
 POINTS_F4 = (0.0, 1.0, -1.0, 2.0, -2.0, INF)
 POINTS_F6 = (0.0, 1.0, -1.0, 2.0, -2.0, 0.5, -0.5, INF)
 
-WORKLOAD_IDS = {"tiny": 0, "resnet18": 1, "resnet34": 2, "sd15": 3, "sd15_stack": 4}
+WORKLOAD_IDS = {"tiny": 0, "resnet18": 1, "resnet34": 2, "sd15": 3, "sd15_stack": 4, "probe": 5}
 
 # tensor ids of the per-tensor streams
 _T_X, _T_W, _T_SB, _T_SG, _T_OUTLIER = 1, 2, 3, 4, 5
@@ -194,4 +194,9 @@ def workload(name: str, seed: int = 0) -> List[Layer]:
                                  "student_t_outliers", 1.0, "loguniform", seed))
         assert len(out) == 44
         return out
+    if name == "probe":
+        # Hadamard-stage capability probe: a compute-bound per-tap GEMM (T = 8192 tiles,
+        # Cin = Cout = 2560, G = 64, F(6,3)) and a quarter-size copy (T = 2048) for profiling.
+        return [Layer("probe", 0, 6, 2, 384, 384, 2560, 2560, 64, "bf16", "relu_normal", 2.0, "loguniform", seed),
+                Layer("probe", 1, 6, 2, 192, 192, 2560, 2560, 64, "bf16", "relu_normal", 2.0, "loguniform", seed)]
     raise KeyError(name)
