@@ -104,30 +104,47 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volati
     }
 }
 
-// The tap-units L = (mb * num_nb + nb) * n2 + tap (one tap of one 128-row block
-// and one BN-column block) are split into equal contiguous ranges, one per
-// CTA.  Every role of a CTA walks its range the same way: a stage covers up to
-// TPS consecutive taps of one (mb, nb) block; the walk never divides.
+// The tap-units (one tap of one 128-row block and one BN-column block) are
+// numbered L = (mb * num_nb + nb) * n2 + tap when there is one column block
+// (a stage then covers up to TPS consecutive taps of one block), and
+// L = (mb * n2 + tap) * num_nb + nb otherwise (one tap per stage; the column
+// blocks of a (row block, tap) follow each other, so its A tile is read from
+// DRAM once and the CTAs working on the same taps share the B tiles in L2).
+// The units are split into equal contiguous ranges, one per CTA; every role
+// of a CTA walks its range the same way, without division.
 struct Walk {
     int L, L1, tap, nb, mb;
     __device__ __forceinline__ void init(const GemmArgs& p) {
         const long tot = p.num_units;
         L = (int)(tot * blockIdx.x / gridDim.x);
         L1 = (int)(tot * (blockIdx.x + 1) / gridDim.x);
-        tap = L % p.n2;
-        const int r = L / p.n2;
-        nb = r % p.num_nb;
-        mb = r / p.num_nb;
+        if (p.num_nb == 1) {
+            tap = L % p.n2;
+            nb = 0;
+            mb = L / p.n2;
+        } else {
+            nb = L % p.num_nb;
+            const int r = L / p.num_nb;
+            tap = r % p.n2;
+            mb = r / p.n2;
+        }
     }
     __device__ __forceinline__ int stage_taps(int tps, int n2) const { return min(min(tps, n2 - tap), L1 - L); }
     __device__ __forceinline__ void advance(int k, const GemmArgs& p) {
         L += k;
-        tap += k;
-        if (tap == p.n2) {
-            tap = 0;
+        if (p.num_nb == 1) {
+            tap += k;
+            if (tap == p.n2) {
+                tap = 0;
+                ++mb;
+            }
+        } else {   // k == 1
             if (++nb == p.num_nb) {
                 nb = 0;
-                ++mb;
+                if (++tap == p.n2) {
+                    tap = 0;
+                    ++mb;
+                }
             }
         }
     }
@@ -538,7 +555,8 @@ int tc_block_n(int Cout, int G) {
 
 // Stage shape: SK bytes of K (a multiple of G dividing Cin, at most NACC/2
 // groups so that at least two accumulator slots exist), swizzle width BK
-// dividing SK, and TPS taps per stage when SK == Cin (as many as keep three
+// dividing SK, and TPS taps per stage when SK == Cin and there is one column
+// block (as many as keep three
 // stages in the shared-memory budget).
 static void choose_stage(GemmArgs& a, int BN) {
     const int nacc = std::min(512 / BN, kMaxNacc);
@@ -555,7 +573,7 @@ static void choose_stage(GemmArgs& a, int BN) {
     const size_t budget = 200 * 1024;
     const size_t per_tap = (size_t)sk * (kBM + BN) + (size_t)gps * (kBM + BN) * 4;
     a.tps = 1;
-    if (sk == a.Cin)
+    if (sk == a.Cin && a.num_nb == 1)   // several column blocks: one tap per stage (see Walk)
         for (int t : {8, 4, 2})
             if (t <= a.n2 && budget / (per_tap * t) >= 3) {
                 a.tps = t;
@@ -571,9 +589,9 @@ cudaError_t launch_hadamard_tc(GemmArgs a, const int8_t* Vq, const int8_t* Uq, i
     if (BN == 0) return cudaErrorInvalidValue;
     EncodeTiledFn enc = get_encode_fn();
     if (!enc) return cudaErrorNotSupported;
-    choose_stage(a, BN);
     a.num_mb = (a.T + kBM - 1) / kBM;
     a.num_nb = a.Cout / BN;
+    choose_stage(a, BN);
     a.num_units = a.num_mb * a.num_nb * a.n2;   // tap-units, split evenly over the CTAs
 
     Maps m;
