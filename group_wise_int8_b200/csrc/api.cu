@@ -288,8 +288,8 @@ int wino_plan(wino_plan_t* out, int m, const double* points, const float* S_B, c
         p->tf.ATd[i] = ((uint64_t)b << 32) | b;
     }
     std::memcpy(p->wa.G, p->mat.G, sizeof(double) * n * 3);
-    const uint64_t bt_mask = m == 4 ? kMaskBT_F4 : kMaskBT_F6;
-    const uint64_t at_mask = m == 4 ? kMaskAT_F4 : kMaskAT_F6;
+    const uint64_t bt_mask = m == 2 ? kMaskBT_F2 : (m == 4 ? kMaskBT_F4 : kMaskBT_F6);
+    const uint64_t at_mask = m == 2 ? kMaskAT_F2 : (m == 4 ? kMaskAT_F4 : kMaskAT_F6);
     p->bt_masked = (p->mat.bt_nonzero & ~bt_mask) == 0;
     p->at_masked = (p->mat.at_nonzero & ~at_mask) == 0;
     *out = p;

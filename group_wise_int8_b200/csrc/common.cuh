@@ -9,10 +9,13 @@
 namespace wino {
 
 // Zero patterns (bit i*n+k) of the unscaled transforms for the standard
-// point orders 0,1,-1,2,-2,inf (F(4,3)) and 0,1,-1,2,-2,1/2,-1/2,inf (F(6,3)).
+// point orders 0,1,-1,inf (F(2,3)), 0,1,-1,2,-2,inf (F(4,3)) and
+// 0,1,-1,2,-2,1/2,-1/2,inf (F(6,3)).
 // Diagonal scales keep the pattern.  The host verifies a plan's exact pattern
 // is contained in the mask before choosing a masked kernel; otherwise the
 // all-ones (generic) kernel runs.
+constexpr uint64_t kMaskBT_F2 = 0x000000000000a665ull;
+constexpr uint64_t kMaskAT_F2 = 0x00000000000000e7ull;
 constexpr uint64_t kMaskBT_F4 = 0x0000000a9e79e795ull;
 constexpr uint64_t kMaskAT_F4 = 0x0000000000f9e79full;
 constexpr uint64_t kMaskBT_F6 = 0xaa7e7e7e7e7e7e55ull;

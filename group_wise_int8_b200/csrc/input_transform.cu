@@ -240,6 +240,11 @@ cudaError_t launch_cc(const InputArgs& a, const TransformArgs& tf, cudaStream_t 
 
 cudaError_t launch_input_transform(const InputArgs& a, const TransformArgs& tf, int m, bool masked, bool bf16_in,
                                    cudaStream_t st) {
+    if (m == 2) {
+        if (bf16_in)
+            return masked ? launch_cc<2, kMaskBT_F2, uint16_t>(a, tf, st) : launch_cc<2, kMaskAll, uint16_t>(a, tf, st);
+        return masked ? launch_cc<2, kMaskBT_F2, float>(a, tf, st) : launch_cc<2, kMaskAll, float>(a, tf, st);
+    }
     if (m == 4) {
         if (bf16_in)
             return masked ? launch_cc<4, kMaskBT_F4, uint16_t>(a, tf, st) : launch_cc<4, kMaskAll, uint16_t>(a, tf, st);

@@ -139,6 +139,9 @@ cudaError_t launch_m(const OutputArgs& a, const TransformArgs& tf, bool src_y32,
 cudaError_t launch_output_transform(const OutputArgs& a, const TransformArgs& tf, int m, bool masked, bool src_y32,
                                     bool bf16_out, cudaStream_t st) {
     const bool debug = a.sY_dbg != nullptr;
+    if (m == 2)
+        return masked ? launch_m<2, kMaskAT_F2>(a, tf, src_y32, bf16_out, debug, st)
+                      : launch_m<2, kMaskAll>(a, tf, src_y32, bf16_out, debug, st);
     if (m == 4)
         return masked ? launch_m<4, kMaskAT_F4>(a, tf, src_y32, bf16_out, debug, st)
                       : launch_m<4, kMaskAll>(a, tf, src_y32, bf16_out, debug, st);

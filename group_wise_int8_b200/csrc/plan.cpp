@@ -111,7 +111,7 @@ Q vand(bool at_inf, Q p, int j, int b) {
 }  // namespace
 
 int build_matrices(int m, const double* points, const float* S_B, const float* S_G, Matrices* out) {
-    if ((m != 4 && m != 6) || !points || !out) return WINO_ERR_INVALID_ARG;
+    if ((m != 2 && m != 4 && m != 6) || !points || !out) return WINO_ERR_INVALID_ARG;
     const int n = m + 2;
     g_bad = false;
     bool inf[kMaxN];

@@ -77,7 +77,9 @@ __global__ void __launch_bounds__(256) weight_transform_kernel(WeightArgs wa, co
 cudaError_t launch_weight_transform(const WeightArgs& wa, int m, const float* w, int Cin, int Cout, int G,
                                     int8_t* Uq, float* sU, cudaStream_t st) {
     dim3 grid(Cin / G, Cout);
-    if (m == 4)
+    if (m == 2)
+        weight_transform_kernel<2><<<grid, G, 0, st>>>(wa, w, Cin, Cout, G, Uq, sU);
+    else if (m == 4)
         weight_transform_kernel<4><<<grid, G, 0, st>>>(wa, w, Cin, Cout, G, Uq, sU);
     else
         weight_transform_kernel<6><<<grid, G, 0, st>>>(wa, w, Cin, Cout, G, Uq, sU);

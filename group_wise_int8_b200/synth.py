@@ -36,6 +36,7 @@ import numpy as np
 
 INF = math.inf
 
+POINTS_F2 = (0.0, 1.0, -1.0, INF)
 POINTS_F4 = (0.0, 1.0, -1.0, 2.0, -2.0, INF)
 POINTS_F6 = (0.0, 1.0, -1.0, 2.0, -2.0, 0.5, -0.5, INF)
 
@@ -65,7 +66,7 @@ class Layer:
 
     @property
     def points(self):
-        return POINTS_F4 if self.m == 4 else POINTS_F6
+        return {2: POINTS_F2, 4: POINTS_F4}.get(self.m, POINTS_F6)
 
     @property
     def n(self):

@@ -102,7 +102,7 @@ typedef struct wino_plan_s* wino_plan_t;
 
 /*
  * wino_plan -- build the transforms of F(m,3) on the host.
- *   m       4 or 6 (n = m + 2 interpolation points).
+ *   m       2, 4 or 6 (n = m + 2 interpolation points).
  *   points  n doubles, the points in tap order; INFINITY is the point at
  *           infinity (homogeneous (1,0)); finite points must be exact
  *           dyadic-friendly doubles and pairwise distinct.

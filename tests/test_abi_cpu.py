@@ -68,6 +68,13 @@ def test_plan_other_point_orders_match_oracle(lib):
     assert np.array_equal(BT, op.BT_f) and np.array_equal(G, op.G_d) and np.array_equal(AT, op.AT_f)
 
 
+@pytest.mark.parametrize("pts", [synth.POINTS_F2, (math.inf, -1.0, 0.0, 1.0)])
+def test_plan_f23_matches_oracle(lib, pts):
+    op = oracle.Plan(2, pts)
+    BT, G, AT = wino.Plan(2, pts, None, None, 32).matrices()
+    assert np.array_equal(BT, op.BT_f) and np.array_equal(G, op.G_d) and np.array_equal(AT, op.AT_f)
+
+
 @pytest.mark.parametrize("bad", [
     dict(m=5), dict(group=48), dict(points=(0.0, 1.0, 1.0, 2.0, -2.0, math.inf)),
     dict(points=(0.0, 1.0, -1.0, math.inf, -2.0, math.inf)), dict(points=(0.0, 1.0, -1.0, 2.0, float("nan"), math.inf)),

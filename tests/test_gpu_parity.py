@@ -21,7 +21,7 @@ from tests.gpu_util import assert_bits_equal, bf16_round, rel_l2, run_gpu, run_o
 
 pytestmark = pytest.mark.gpu
 
-P4, P6 = synth.POINTS_F4, synth.POINTS_F6
+P2, P4, P6 = synth.POINTS_F2, synth.POINTS_F4, synth.POINTS_F6
 
 # name: (m, points, N, H, W, Cin, Cout, G, dtype, act, scales)
 CASES = {
@@ -36,6 +36,9 @@ CASES = {
     "f6_one_pixel": (6, P6, 3, 1, 1, 64, 32, 32, "bf16", "relu_normal", "identity"),
     "f4_permuted_points": (4, (math.inf, 0.5, -2.0, 1.0, 0.0, -1.0), 1, 10, 9, 64, 64, 64, "bf16",
                            "relu_normal", "loguniform"),
+    "f2_ragged": (2, P2, 2, 13, 11, 64, 64, 32, "bf16", "relu_normal", "loguniform"),
+    "f2_g64_cout128_f32": (2, P2, 1, 30, 30, 128, 128, 64, "f32", "student_t_outliers", "loguniform"),
+    "f2_permuted_points": (2, (math.inf, -1.0, 0.0, 1.0), 1, 9, 10, 32, 64, 32, "bf16", "normal", "loguniform"),
 }
 
 

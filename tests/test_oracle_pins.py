@@ -27,7 +27,7 @@ import torch
 import oracle
 from group_wise_int8_b200 import synth
 
-P4, P6 = synth.POINTS_F4, synth.POINTS_F6
+P2, P4, P6 = synth.POINTS_F2, synth.POINTS_F4, synth.POINTS_F6
 
 
 def torch_conv_f64(x, w):
@@ -65,7 +65,7 @@ def _vandermonde_frac(points, b):
     return rows
 
 
-@pytest.mark.parametrize("m,pts", [(4, P4), (6, P6)])
+@pytest.mark.parametrize("m,pts", [(2, P2), (4, P4), (6, P6)])
 def test_plan_inverse_property(m, pts):
     """B^T V^T = S_B (B^T = S_B V^{-T}); with identity scales B^T V^T = I to rounding."""
     n = m + 2
@@ -92,6 +92,19 @@ def test_lavin_gray_f43_special_case():
     assert np.allclose(p.AT_d, AT, rtol=1e-7, atol=0)
 
 
+def test_textbook_f23_special_case():
+    """The textbook F(2x2,3x3) matrices (points 0, 1, -1, inf), reproduced exactly by S_B, S_G below."""
+    BT = np.array([[1, 0, -1, 0], [0, 1, 1, 0], [0, -1, 1, 0], [0, 1, 0, -1]], np.float64)
+    G = np.array([[1, 0, 0], [0.5, 0.5, 0.5], [0.5, -0.5, 0.5], [0, 0, 1]], np.float64)
+    AT = np.array([[1, 1, 1, 0], [0, 1, -1, -1]], np.float64)
+    sb = np.array([1, 2, 2, -1], np.float32)
+    sg = np.array([1, 0.5, 0.5, 1], np.float32)
+    p = oracle.Plan(2, P2, sb, sg)
+    assert np.array_equal(p.BT_f.astype(np.float64), BT)
+    assert np.array_equal(p.G_d, G)          # dyadic entries: exact
+    assert np.array_equal(p.AT_d, AT)
+
+
 def test_plan_rejects_duplicate_points():
     with pytest.raises(ValueError):
         oracle.Plan(4, (0.0, 1.0, 1.0, 2.0, -2.0, math.inf))
@@ -99,7 +112,7 @@ def test_plan_rejects_duplicate_points():
 
 # --------------------------------------------------- Winograd identity (quant off)
 
-@pytest.mark.parametrize("m,pts", [(4, P4), (6, P6)])
+@pytest.mark.parametrize("m,pts", [(2, P2), (4, P4), (6, P6)])
 @pytest.mark.parametrize("scaled", [False, True])
 def test_winograd_identity_f64(m, pts, scaled):
     x, w = rand_case(10 + m)
@@ -124,7 +137,7 @@ def test_winograd_identity_f32(m, pts, tol):
     assert err < 2e-5   # fp32 transforms: far inside the stated bound
 
 
-@pytest.mark.parametrize("m,pts", [(4, P4), (6, P6)])
+@pytest.mark.parametrize("m,pts", [(2, P2), (4, P4), (6, P6)])
 def test_scale_invariance_unquantised(m, pts):
     """Any S_B, S_G with S_A = (S_B S_G)^{-1} leaves the unquantised output unchanged."""
     x, w = rand_case(30 + m, N=1, H=12, W=12, Cin=4, Cout=3)
@@ -157,7 +170,7 @@ def test_identity_pin_catches_planted_matrix_mistakes(mutation):
 
 # ------------------------------------------------------------ stage pins
 
-@pytest.mark.parametrize("m,pts", [(4, P4), (6, P6)])
+@pytest.mark.parametrize("m,pts", [(2, P2), (4, P4), (6, P6)])
 def test_input_transform_matches_matmul(m, pts):
     """V = B^T d B per tile and channel (tile origin (ty m - 1, tx m - 1), zero padding)."""
     n = m + 2
@@ -179,7 +192,7 @@ def test_input_transform_matches_matmul(m, pts):
             assert np.all(np.abs(got - ref) <= bound)
 
 
-@pytest.mark.parametrize("m,pts", [(4, P4), (6, P6)])
+@pytest.mark.parametrize("m,pts", [(2, P2), (4, P4), (6, P6)])
 def test_weight_transform_matches_matmul(m, pts):
     n = m + 2
     _, w = rand_case(60, Cin=8, Cout=3)
