@@ -44,6 +44,8 @@ def lib():
         L.orc_y_requant.argtypes = [ctypes.c_int, _f32p, ctypes.c_long, ctypes.c_int, ctypes.c_int, _i8p, _f32p]
         L.orc_output_transform.argtypes = [ctypes.c_int, _f32p, _i8p, _f32p, ctypes.c_int, ctypes.c_int,
                                            ctypes.c_int, ctypes.c_int, ctypes.c_int, _f32p]
+        L.orc_y_requant_tap.argtypes = L.orc_y_requant.argtypes
+        L.orc_output_transform_tap.argtypes = L.orc_output_transform.argtypes
         L.orc_conv_direct_f64.argtypes = [_f32p, _f32p, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                           ctypes.c_int, ctypes.c_int, _f64p]
         L.orc_conv_wino_f64.argtypes = [ctypes.c_int, _f64p, _f64p, _f64p, _f32p, _f32p, ctypes.c_int,
@@ -51,8 +53,8 @@ def lib():
         L.orc_conv_wino_f32.argtypes = [ctypes.c_int, _f32p, _f64p, _f32p, _f32p, _f32p, ctypes.c_int,
                                         ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, _f32p]
         for name in ("orc_weight_transform", "orc_input_transform", "orc_hadamard", "orc_y_requant",
-                     "orc_output_transform", "orc_conv_direct_f64", "orc_conv_wino_f64",
-                     "orc_conv_wino_f32"):
+                     "orc_output_transform", "orc_y_requant_tap", "orc_output_transform_tap",
+                     "orc_conv_direct_f64", "orc_conv_wino_f64", "orc_conv_wino_f32"):
             getattr(L, name).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -138,20 +140,24 @@ def hadamard(n2: int, Vq, sV, Uq, sU, G: int, want_acc: bool = False):
     return Y, acc
 
 
-def y_requant(n2: int, Y: np.ndarray, G: int):
+def y_requant(n2: int, Y: np.ndarray, G: int, per_tap: bool = False):
+    """Y groups of G couts spanning all n2 taps of a tile (sY [T][Cout/G]), or, with
+    per_tap (the Y_TAP reading), one group per tap (sY [T][n2][Cout/G])."""
     T, _, Cout = Y.shape
     Yq = np.zeros(Y.shape, np.int8)
-    sY = np.zeros((T, Cout // G), np.float32)
-    rc = lib().orc_y_requant(n2, _p(np.ascontiguousarray(Y), _f32p), T, Cout, G, _p(Yq, _i8p), _p(sY, _f32p))
+    sY = np.zeros((T, n2, Cout // G) if per_tap else (T, Cout // G), np.float32)
+    fn = lib().orc_y_requant_tap if per_tap else lib().orc_y_requant
+    rc = fn(n2, _p(np.ascontiguousarray(Y), _f32p), T, Cout, G, _p(Yq, _i8p), _p(sY, _f32p))
     assert rc == 0
     return Yq, sY
 
 
-def output_transform(plan: Plan, Yq, sY, N: int, H: int, W: int, G: int):
+def output_transform(plan: Plan, Yq, sY, N: int, H: int, W: int, G: int, per_tap: bool = False):
     Cout = Yq.shape[2]
     out = np.zeros((N, H, W, Cout), np.float32)
-    rc = lib().orc_output_transform(plan.m, _p(plan.AT_f, _f32p), _p(Yq, _i8p), _p(sY, _f32p), N, H, W, Cout,
-                                    G, _p(out, _f32p))
+    fn = lib().orc_output_transform_tap if per_tap else lib().orc_output_transform
+    rc = fn(plan.m, _p(plan.AT_f, _f32p), _p(Yq, _i8p), _p(np.ascontiguousarray(sY), _f32p), N, H, W, Cout,
+            G, _p(out, _f32p))
     assert rc == 0
     return out
 
@@ -191,15 +197,17 @@ def conv_wino_f32(plan: Plan, x: np.ndarray, w: np.ndarray) -> np.ndarray:
     return out
 
 
-def run_pipeline(plan: Plan, x: np.ndarray, w: np.ndarray, G: int, want_acc: bool = False) -> Dict[str, np.ndarray]:
-    """The full quantised pipeline, every stage kept for comparison."""
+def run_pipeline(plan: Plan, x: np.ndarray, w: np.ndarray, G: int, want_acc: bool = False,
+                 per_tap: bool = False) -> Dict[str, np.ndarray]:
+    """The full quantised pipeline, every stage kept for comparison (per_tap: the Y_TAP
+    reading of the Y groups)."""
     N, H, W, _ = x.shape
     n2 = plan.n * plan.n
     Uq, sU, _ = weight_transform(plan, w, G)
     Vq, sV, _ = input_transform(plan, x, G)
     Y, acc = hadamard(n2, Vq, sV, Uq, sU, G, want_acc=want_acc)
-    Yq, sY = y_requant(n2, Y, G)
-    out = output_transform(plan, Yq, sY, N, H, W, G)
+    Yq, sY = y_requant(n2, Y, G, per_tap)
+    out = output_transform(plan, Yq, sY, N, H, W, G, per_tap)
     return dict(Uq=Uq, sU=sU, Vq=Vq, sV=sV, Y=Y, acc=acc, Yq=Yq, sY=sY, out=out)
 
 

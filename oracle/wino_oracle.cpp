@@ -467,6 +467,64 @@ int orc_y_requant(int n2, const float* Y, long T, int Cout, int G, signed char* 
     return 0;
 }
 
+// Stage 4a, per-tap reading (Y_TAP): one scale per (tile, tap, block of G
+// consecutive couts) instead of one spanning all n*n taps of the tile.
+//   Y [T][n2][Cout] fp32 -> Yq [T][n2][Cout] int8, sY [T][n2][Cout/G]
+int orc_y_requant_tap(int n2, const float* Y, long T, int Cout, int G, signed char* Yq, float* sY) {
+    if (G <= 0 || Cout % G != 0) return -1;
+    const int ng = Cout / G;
+    set_omp();
+#pragma omp parallel for schedule(static)
+    for (long t = 0; t < T; ++t)
+        for (int tap = 0; tap < n2; ++tap)
+            for (int j = 0; j < ng; ++j) {
+                const float* y = Y + ((size_t)t * n2 + tap) * Cout + (size_t)j * G;
+                signed char* q = Yq + ((size_t)t * n2 + tap) * Cout + (size_t)j * G;
+                quantize_group(y, 1, G, q, 1, &sY[((size_t)t * n2 + tap) * ng + j]);
+            }
+    return 0;
+}
+
+// Stage 4b, per-tap reading: as orc_output_transform, with Yd[xi][nu] scaled by
+// the scale of tap (xi, nu).  sY [T][n2][Cout/G]
+int orc_output_transform_tap(int m, const float* AT_f, const signed char* Yq, const float* sY, int N, int H,
+                             int W, int Cout, int G, float* out) {
+    const int n = m + 2, n2 = n * n;
+    if (G <= 0 || Cout % G != 0) return -1;
+    const int TH = (H + m - 1) / m, TW = (W + m - 1) / m;
+    const long T = (long)N * TH * TW;
+    const int ng = Cout / G;
+    set_omp();
+#pragma omp parallel for schedule(static)
+    for (long t = 0; t < T; ++t) {
+        const int img = (int)(t / ((long)TH * TW));
+        const int ty = (int)((t / TW) % TH), tx = (int)(t % TW);
+        for (int co = 0; co < Cout; ++co) {
+            float Yd[8][8], Z[8][8];
+            for (int xi = 0; xi < n; ++xi)
+                for (int nu = 0; nu < n; ++nu) {
+                    const int tap = xi * n + nu;
+                    const float s = sY[((size_t)t * n2 + tap) * ng + co / G];
+                    Yd[xi][nu] = s * (float)Yq[((size_t)t * n2 + tap) * Cout + co];
+                }
+            for (int i = 0; i < m; ++i)
+                for (int nu = 0; nu < n; ++nu) {
+                    float acc = 0.0f;
+                    for (int xi = 0; xi < n; ++xi) acc = std::fmaf(AT_f[i * n + xi], Yd[xi][nu], acc);
+                    Z[i][nu] = acc;
+                }
+            for (int i = 0; i < m; ++i)
+                for (int j = 0; j < m; ++j) {
+                    float acc = 0.0f;
+                    for (int nu = 0; nu < n; ++nu) acc = std::fmaf(Z[i][nu], AT_f[j * n + nu], acc);
+                    int yy = ty * m + i, xx = tx * m + j;
+                    if (yy < H && xx < W) out[(((size_t)img * H + yy) * W + xx) * Cout + co] = acc;
+                }
+        }
+    }
+    return 0;
+}
+
 // Stage 4b: dequantise and output transform, o = A^T (sY * Yq) A, cropped to
 // the image.  Z[i][nu] = fmaf-chain over xi of AT[i][xi] * Yd[xi][nu];
 // o[i][j] = fmaf-chain over nu of Z[i][nu] * AT[j][nu].

@@ -312,6 +312,41 @@ def test_y_groups_span_taps():
 
 
 @pytest.mark.parametrize("m,pts", [(4, P4), (6, P6)])
+def test_y_tap_reading_absorbs_per_tap_powers_of_two(m, pts):
+    """The per-tap Y reading (Y_TAP): a per-tap power-of-two profile on S_B scales
+    V, Y and sY of each tap (i, j) by d_i d_j exactly and A^T's column xi by 1/d_xi,
+    so the per-tap groups give bit-identical codes and output.  With the default
+    tile-spanning groups the same profile changes the codes (test_y_groups_span_taps)."""
+    n, G = m + 2, 16
+    x, w = rand_case(72, N=1, H=13, W=11, Cin=32, Cout=32)
+    sb, sg = dyadic_scales(17, n), dyadic_scales(18, n)
+    k = np.array([0, 1, -1, 2, 0, -2, 1, 0][:n], np.float32)
+    base = oracle.run_pipeline(oracle.Plan(m, pts, sb, sg), x, w, G, per_tap=True)
+    prof = oracle.run_pipeline(oracle.Plan(m, pts, sb * 2.0 ** k, sg), x, w, G, per_tap=True)
+    assert np.array_equal(base["Vq"], prof["Vq"]) and np.array_equal(base["Yq"], prof["Yq"])
+    d = 2.0 ** k.astype(np.float64)
+    ratio = (d[:, None] * d[None, :]).reshape(-1)                # tap (i, j) -> d_i d_j
+    assert np.array_equal(prof["sY"].astype(np.float64), base["sY"].astype(np.float64) * ratio[None, :, None])
+    assert np.array_equal(base["out"], prof["out"])
+
+
+def test_y_tap_scales_are_per_tap_group_maxima():
+    """sY[t][tap][j] = max |Y[t][tap][jG:(j+1)G]| / 127 (IEEE division), codes = rne(Y / sY)."""
+    r = np.random.default_rng(5)
+    T, n2, Cout, G = 3, 16, 64, 32
+    Y = (r.standard_normal((T, n2, Cout)) * np.exp(r.standard_normal((T, n2, 1)))).astype(np.float32)
+    Y[1, 3, :G] = 0.0                                              # an all-zero group
+    Yq, sY = oracle.y_requant(n2, Y, G, per_tap=True)
+    amax = np.abs(Y.reshape(T, n2, Cout // G, G)).max(axis=-1)
+    assert np.array_equal(sY, (amax / np.float32(127.0)).astype(np.float32))
+    assert sY[1, 3, 0] == 0.0 and not Yq[1, 3, :G].any()
+    assert np.abs(Yq.astype(np.int32)).max() == 127
+    q = Yq.reshape(T, n2, Cout // G, G).astype(np.float64) * sY[..., None]
+    err = np.abs(q - Y.reshape(T, n2, Cout // G, G))
+    assert np.all(err <= 0.5 * sY[..., None] * (1 + 1e-6) + 1e-30)
+
+
+@pytest.mark.parametrize("m,pts", [(4, P4), (6, P6)])
 def test_standard_scales_collapse_and_row_norm_scales_recover(m, pts):
     """The pages: with standard scales fully quantized Winograd collapses (FID > 300),
     and rescaling the rows of B^T and G (their row norms) removes Y's per-tap
