@@ -38,7 +38,7 @@ struct Layout {
     int TH = 0, TW = 0, n2 = 0, ng = 0, ngo = 0;
     long T = 0, T_pad = 0;
     int y_path = 0, gemm = 0;
-    bool dbg_yq = false, dbg_acc = false;
+    bool dbg_yq = false, dbg_acc = false, ytap = false;
     size_t off_vq = 0, off_sv = 0, off_amax = 0, off_yq = 0, off_y32 = 0, off_sy = 0, off_acc = 0, off_err = 0;
     size_t total = 0;
 };
@@ -88,7 +88,9 @@ Layout make_layout(const wino_plan_s* p, int N, int H, int W, int Cin, int Cout)
     L.ngo = Cout / p->G;
     L.gemm = p->opts.gemm == WINO_GEMM_AUTO ? WINO_GEMM_TCGEN05 : p->opts.gemm;
     if (L.gemm == WINO_GEMM_TCGEN05 && tc_block_n(Cout, p->G) == 0) L.gemm = WINO_GEMM_SIMT;
-    L.y_path = p->opts.y_path == WINO_YPATH_AUTO ? choose_y_path(p, L.T, Cin, Cout, L.n2) : p->opts.y_path;
+    L.ytap = p->opts.y_groups == WINO_YGROUPS_TAP;
+    L.y_path = L.ytap ? WINO_YPATH_Y32
+                      : (p->opts.y_path == WINO_YPATH_AUTO ? choose_y_path(p, L.T, Cin, Cout, L.n2) : p->opts.y_path);
     L.dbg_yq = (p->opts.debug & WINO_DEBUG_YQ) != 0;
     L.dbg_acc = (p->opts.debug & WINO_DEBUG_ACC32) != 0;
     size_t off = 0;
@@ -108,7 +110,7 @@ Layout make_layout(const wino_plan_s* p, int N, int H, int W, int Cin, int Cout)
     }
     if (L.dbg_yq) {
         L.off_sy = off;
-        off = up(off + sizeof(float) * (size_t)L.T * L.ngo, kAlign);
+        off = up(off + sizeof(float) * (size_t)L.T * (L.ytap ? L.n2 : 1) * L.ngo, kAlign);
     }
     if (L.dbg_acc) {
         L.off_acc = off;
@@ -226,6 +228,7 @@ int run_conv(wino_plan_s* p, const void* x, int x_dtype, int N, int H, int W, in
     oa.Yq_dbg = (L.y_path == WINO_YPATH_Y32 && L.dbg_yq) ? Yq : nullptr;
     oa.sY_dbg = sYd;
     oa.out = y;
+    oa.ytap = L.ytap ? 1 : 0;
     prof_mark(p, slot++, st);
     e = launch_output_transform(oa, p->tf, p->mat.m, p->at_masked, L.y_path == WINO_YPATH_Y32, y_dtype == WINO_BF16,
                                 st);
@@ -269,7 +272,8 @@ int wino_plan(wino_plan_t* out, int m, const double* points, const float* S_B, c
     p->G = group;
     std::memset(&p->opts, 0, sizeof(p->opts));
     if (opts) p->opts = *opts;
-    if (p->opts.y_path < 0 || p->opts.y_path > 2 || p->opts.gemm < 0 || p->opts.gemm > 2) {
+    if (p->opts.y_path < 0 || p->opts.y_path > 2 || p->opts.gemm < 0 || p->opts.gemm > 2 || p->opts.y_groups < 0 ||
+        p->opts.y_groups > 1 || (p->opts.y_groups == WINO_YGROUPS_TAP && p->opts.y_path == WINO_YPATH_RECOMPUTE)) {
         delete p;
         return WINO_ERR_INVALID_ARG;
     }
@@ -405,7 +409,7 @@ int wino_debug_dump(wino_plan_t p, const void* ws, int N, int H, int W, int Cin,
             need = (size_t)L.T * L.n2 * Cout; off = L.off_yq; break;
         case WINO_DUMP_SY:
             if (!L.dbg_yq) return WINO_ERR_UNSUPPORTED;
-            need = sizeof(float) * (size_t)L.T * L.ngo; off = L.off_sy; break;
+            need = sizeof(float) * (size_t)L.T * (L.ytap ? L.n2 : 1) * L.ngo; off = L.off_sy; break;
         case WINO_DUMP_Y32:
             if (!L.off_y32) return WINO_ERR_UNSUPPORTED;
             need = sizeof(float) * (size_t)L.T * L.n2 * Cout; off = L.off_y32; break;

@@ -110,11 +110,135 @@ __global__ void __launch_bounds__(128, 4) output_transform_kernel(OutputArgs p, 
     }
 }
 
+// Per-tap Y groups (the Y_TAP reading): Y is requantised with one scale per
+// (tile, tap, G couts).  Same thread layout as output_transform_kernel, fp32 Y
+// source only.  Pass 1 reduces each tap's |Y| over the group -- the G/2 lanes of
+// a warp segment by shuffles, or (G >= 128) the G/64 warps of the CTA through
+// shared memory -- and one thread per (group, tap) stores the scale; pass 2 is
+// the fp32-Y path of output_transform_kernel with the tap's own scale.
+template <int M, uint64_t MASK, bool BF16_OUT>
+__global__ void __launch_bounds__(128) output_transform_ytap_kernel(OutputArgs p, TransformArgs tf) {
+    constexpr int N = M + 2, N2 = N * N;
+    __shared__ QScale qsm[4][2][N2];     // [warp][segment][tap] (G <= 64) or [group in CTA][0][tap]
+    __shared__ float red[4][N2];         // per-warp maxima (G >= 128)
+    grid_dependents_launch();
+    grid_dependency_wait();
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const long i = (long)blockIdx.x * blockDim.x + threadIdx.x;
+    const int cpairs = p.Cout >> 1;
+    const long t = i / cpairs;
+    const int co = 2 * (int)(i - t * cpairs);
+    const bool live = t < p.T;           // a CTA covers whole groups; dead threads still join the reductions
+    const int G = p.G;
+    const int cg = co / G;
+    const size_t base = (size_t)(live ? t : 0) * p.Cout + co;
+    const size_t tstride = (size_t)p.T * p.Cout;
+
+    // ---- pass 1: per-tap group scales
+    if (G <= 64) {
+        const int seg_w = G / 2;                   // lanes per group
+        const int seg = lane / seg_w, sl = lane % seg_w;
+        for (int tap = 0; tap < N2; ++tap) {
+            float a = 0.0f;
+            if (live) {
+                const float2 y = *reinterpret_cast<const float2*>(p.Y32 + base + (size_t)tap * tstride);
+                a = fmaxf(fabsf(y.x), fabsf(y.y));
+            }
+            for (int o = seg_w / 2; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
+            if (sl == tap % seg_w) {
+                qsm[warp][seg][tap] = make_qscale(a);
+                if (p.sY_dbg && live) p.sY_dbg[((size_t)t * N2 + tap) * p.ngo + cg] = qsm[warp][seg][tap].s;
+            }
+        }
+        __syncwarp();
+    } else {
+        for (int tap = 0; tap < N2; ++tap) {
+            float a = 0.0f;
+            if (live) {
+                const float2 y = *reinterpret_cast<const float2*>(p.Y32 + base + (size_t)tap * tstride);
+                a = fmaxf(fabsf(y.x), fabsf(y.y));
+            }
+            for (int o = 16; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
+            if (lane == 0) red[warp][tap] = a;
+        }
+        __syncthreads();
+        const int wpg = G / 64;                    // warps per group
+        const int ngc = 4 / wpg;                   // groups in the CTA
+        for (int k = threadIdx.x; k < ngc * N2; k += blockDim.x) {
+            const int gi = k / N2, tap = k % N2;
+            float a = 0.0f;
+            for (int w = 0; w < wpg; ++w) a = fmaxf(a, red[gi * wpg + w][tap]);
+            qsm[gi][0][tap] = make_qscale(a);
+            const long i0 = (long)blockIdx.x * blockDim.x + gi * (G / 2);   // first thread of the group
+            const long tg = i0 / cpairs;
+            if (p.sY_dbg && tg < p.T)
+                p.sY_dbg[((size_t)tg * N2 + tap) * p.ngo + (int)(i0 - tg * cpairs) * 2 / G] = qsm[gi][0][tap].s;
+        }
+        __syncthreads();
+    }
+    if (!live) return;
+    const QScale* myq = G <= 64 ? qsm[warp][lane / (G / 2)] : qsm[warp / (G / 64)][0];
+
+    // ---- pass 2: requantise with the tap's scale, then A^T . A
+    uint64_t Z[M][N];
+#pragma unroll
+    for (int nu = 0; nu < N; ++nu) {
+        uint64_t Yc[N];
+#pragma unroll
+        for (int xi = 0; xi < N; ++xi) {
+            const int tap = xi * N + nu;
+            const QScale q = myq[tap];
+            const float2 y = *reinterpret_cast<const float2*>(p.Y32 + base + (size_t)tap * tstride);
+            const Quad qd = quant4(y.x, y.y, y.x, y.y, q);
+            Yc[xi] = f2_mul(f2_pack(q.s, q.s), qd.k01);
+            if (p.Yq_dbg)
+                *reinterpret_cast<uint16_t*>(p.Yq_dbg + base + (size_t)tap * tstride) = (uint16_t)(qd.packed & 0xffffu);
+        }
+#pragma unroll
+        for (int r = 0; r < M; ++r) {
+            uint64_t acc = 0ull;
+#pragma unroll
+            for (int xi = 0; xi < N; ++xi)
+                if ((MASK >> (r * N + xi)) & 1ull) acc = f2_fma(tf.ATd[r * N + xi], Yc[xi], acc);
+            Z[r][nu] = acc;
+        }
+    }
+    const int TT = p.TH * p.TW;
+    const int img = (int)(t / TT);
+    const int rem = (int)(t - (long)img * TT);
+    const int ty = rem / p.TW, tx = rem - ty * p.TW;
+#pragma unroll
+    for (int r = 0; r < M; ++r) {
+        const int yy = ty * M + r;
+        if (yy >= p.H) break;
+#pragma unroll
+        for (int c = 0; c < M; ++c) {
+            const int xx = tx * M + c;
+            if (xx >= p.W) break;
+            uint64_t acc = 0ull;
+#pragma unroll
+            for (int nu = 0; nu < N; ++nu)
+                if ((MASK >> (c * N + nu)) & 1ull) acc = f2_fma(Z[r][nu], tf.ATd[c * N + nu], acc);
+            float o0, o1;
+            f2_unpack(acc, o0, o1);
+            const size_t o = (((size_t)img * p.H + yy) * p.W + xx) * p.Cout + co;
+            if (BF16_OUT)
+                *reinterpret_cast<__nv_bfloat162*>(reinterpret_cast<__nv_bfloat16*>(p.out) + o) =
+                    __floats2bfloat162_rn(o0, o1);
+            else
+                *reinterpret_cast<float2*>(reinterpret_cast<float*>(p.out) + o) = make_float2(o0, o1);
+        }
+    }
+}
+
 template <int M, uint64_t MASK>
 cudaError_t launch_m(const OutputArgs& a, const TransformArgs& tf, bool src_y32, bool bf16_out, bool debug,
                      cudaStream_t st) {
     const long threads = a.T * (long)(a.Cout / 2);
     const dim3 grid((unsigned)((threads + 127) / 128));
+    if (a.ytap)
+        return bf16_out ? launch_dependent(output_transform_ytap_kernel<M, MASK, true>, grid, dim3(128), 0, st, a, tf)
+                        : launch_dependent(output_transform_ytap_kernel<M, MASK, false>, grid, dim3(128), 0, st, a, tf);
 #define WINO_OUT_LAUNCH(Y32, BF, DBG) \
     return launch_dependent(output_transform_kernel<M, MASK, Y32, BF, DBG>, grid, dim3(128), 0, st, a, tf)
     if (src_y32) {

@@ -31,6 +31,7 @@ BF16 = 1
 YPATH_AUTO, YPATH_RECOMPUTE, YPATH_Y32 = 0, 1, 2
 GEMM_AUTO, GEMM_TCGEN05, GEMM_SIMT = 0, 1, 2
 DEBUG_YQ, DEBUG_ACC32, DEBUG_FORCE_TIMEOUT = 1, 2, 4
+YGROUPS_TILE, YGROUPS_TAP = 0, 1
 DUMP_VQ, DUMP_SV, DUMP_YQ, DUMP_SY, DUMP_Y32, DUMP_ACC32 = range(6)
 
 EXPORTED = [
@@ -52,7 +53,7 @@ class WinoError(RuntimeError):
 
 class Opts(ctypes.Structure):
     _fields_ = [("y_path", ctypes.c_int), ("gemm", ctypes.c_int), ("debug", ctypes.c_int),
-                ("reserved", ctypes.c_int * 5)]
+                ("y_groups", ctypes.c_int), ("reserved", ctypes.c_int * 4)]
 
 
 _lib = None
@@ -124,19 +125,19 @@ class Plan:
     """A wino_plan: transforms of F(m,3) for the given points and scales."""
 
     def __init__(self, m: int, points: Sequence[float], S_B=None, S_G=None, group: int = 32,
-                 y_path: int = YPATH_AUTO, gemm: int = GEMM_AUTO, debug: int = 0):
+                 y_path: int = YPATH_AUTO, gemm: int = GEMM_AUTO, debug: int = 0, y_groups: int = YGROUPS_TILE):
         L = load_library()
         n = m + 2
         pts = (ctypes.c_double * n)(*[float(p) for p in points])
         sb = None if S_B is None else (ctypes.c_float * n)(*[float(v) for v in S_B])
         sg = None if S_G is None else (ctypes.c_float * n)(*[float(v) for v in S_G])
-        opts = Opts(y_path, gemm, debug)
+        opts = Opts(y_path, gemm, debug, y_groups)
         h = _vp()
         rc = L.wino_plan(ctypes.byref(h), m, pts, sb, sg, group, ctypes.byref(opts))
         if rc != OK:
             raise WinoError(rc, "wino_plan")
         self._h = h
-        self.m, self.n, self.group = m, n, group
+        self.m, self.n, self.group, self.y_groups = m, n, group, y_groups
 
     def __del__(self):
         h = getattr(self, "_h", None)
@@ -248,7 +249,8 @@ class Plan:
         m, n2, G = self.m, self.n * self.n, self.group
         T = N * math.ceil(H / m) * math.ceil(W / m)
         shapes = {DUMP_VQ: ((T, n2, Cin), np.int8), DUMP_SV: ((T, n2, Cin // G), np.float32),
-                  DUMP_YQ: ((T, n2, Cout), np.int8), DUMP_SY: ((T, Cout // G), np.float32),
+                  DUMP_YQ: ((T, n2, Cout), np.int8),
+                  DUMP_SY: (((T, n2, Cout // G) if self.y_groups == YGROUPS_TAP else (T, Cout // G)), np.float32),
                   DUMP_Y32: ((T, n2, Cout), np.float32), DUMP_ACC32: ((n2, T, Cout, Cin // G), np.int32)}
         shape, dt = shapes[what]
         a = np.zeros(shape, dt)

@@ -82,8 +82,17 @@ typedef struct wino_opts {
                              bounded wait expires, every CTA returns early and
                              wino_check_device_error reports
                              WINO_ERR_DEVICE_TIMEOUT (output undefined) */
-    int reserved[5];
+    int y_groups;  /* WINO_YGROUPS_*: how Y is grouped for its requantisation */
+    int reserved[4];
 } wino_opts;
+
+/* Y groups (the input of the output transform).  TILE (default, the reading the
+ * method needs): one scale per (tile, G consecutive couts) spanning all n*n taps.
+ * TAP (alternative reading): one scale per (tile, tap, G couts); it needs the
+ * fp32-Y path (y_path AUTO resolves to Y32, RECOMPUTE is rejected) and
+ * WINO_DUMP_SY is then [T][n*n][Cout/G]. */
+#define WINO_YGROUPS_TILE 0
+#define WINO_YGROUPS_TAP 1
 
 #define WINO_DEBUG_YQ 1
 #define WINO_DEBUG_ACC32 2
@@ -94,7 +103,7 @@ typedef struct wino_opts {
 #define WINO_DUMP_VQ 0    /* int8  [T][n*n][Cin]        quantised input transform */
 #define WINO_DUMP_SV 1    /* fp32  [T][n*n][Cin/G]      its scales */
 #define WINO_DUMP_YQ 2    /* int8  [T][n*n][Cout]       requantised Y (needs WINO_DEBUG_YQ on the Y32 path) */
-#define WINO_DUMP_SY 3    /* fp32  [T][Cout/G]          Y scales (needs WINO_DEBUG_YQ) */
+#define WINO_DUMP_SY 3    /* fp32  [T][Cout/G]          Y scales (needs WINO_DEBUG_YQ); [T][n*n][Cout/G] with WINO_YGROUPS_TAP */
 #define WINO_DUMP_Y32 4   /* fp32  [T][n*n][Cout]       dequantised Y (Y32 path only) */
 #define WINO_DUMP_ACC32 5 /* int32 [n*n][T][Cout][Cin/G] per-K-group accumulators (WINO_DEBUG_ACC32) */
 

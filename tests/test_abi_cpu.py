@@ -90,6 +90,15 @@ def test_plan_rejects_invalid_arguments(lib, bad):
     assert e.value.status == wino.ERR_INVALID_ARG
 
 
+def test_y_groups_option(lib):
+    tap = wino.Plan(6, synth.POINTS_F6, None, None, 32, y_groups=wino.YGROUPS_TAP)
+    assert tap.resolved_config(32, 56, 56, 64, 64)[0] == wino.YPATH_Y32     # the per-tap reading needs fp32 Y
+    for bad in (dict(y_groups=2), dict(y_groups=wino.YGROUPS_TAP, y_path=wino.YPATH_RECOMPUTE)):
+        with pytest.raises(wino.WinoError) as e:
+            wino.Plan(6, synth.POINTS_F6, None, None, 32, **bad)
+        assert e.value.status == wino.ERR_INVALID_ARG
+
+
 def test_workspace_and_weight_sizes(lib):
     p = wino.Plan(6, synth.POINTS_F6, None, None, 32)
     N, H, W, C = 32, 56, 56, 64

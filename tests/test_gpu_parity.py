@@ -80,6 +80,33 @@ def test_stagewise_bit_exact(cuda_dev, name, y_path, gemm):
     assert abs(s_gpu - s_orc) <= 0.01
 
 
+_oracle_tap_cache = {}
+
+
+@pytest.mark.parametrize("gemm", [wino.GEMM_TCGEN05, wino.GEMM_SIMT])
+@pytest.mark.parametrize("name", ["ragged_f6_cout96", "f4_g64_outliers", "f6_g256", "f6_single_partial_tile",
+                                  "f2_ragged", "f4_permuted_points"])
+def test_y_tap_reading_bit_exact(cuda_dev, name, gemm):
+    """The per-tap Y groups (WINO_YGROUPS_TAP): Yq and the [T][n2][Cout/G] scales bit for bit,
+    the output within the fp32 tolerance, on the fp32-Y path it forces."""
+    m, pts, G, x_f32, x_bits, w, sb, sg = make_case(name)
+    if name not in _oracle_tap_cache:
+        _oracle_tap_cache[name] = run_oracle(m, pts, sb, sg, G, x_f32, w, per_tap=True)
+    ref = _oracle_tap_cache[name]
+    got = run_gpu(m, pts, sb, sg, G, x_f32, x_bits, w, out_dtype=torch.float32, gemm=gemm,
+                  debug=wino.DEBUG_YQ, y_groups=wino.YGROUPS_TAP)
+    assert got["y_path"] == wino.YPATH_Y32
+    for k in ("Vq", "sV", "Y", "Yq", "sY"):
+        assert_bits_equal(k, got[k], ref[k])
+    assert rel_l2(got["out"], ref["out"]) <= 1e-5
+    assert abs(oracle.sqnr_db(ref["ref"], got["out"]) - oracle.sqnr_db(ref["ref"], ref["out"])) <= 0.01
+
+
+def test_y_tap_rejects_recompute_path(cuda_dev):
+    with pytest.raises(wino.WinoError):
+        wino.Plan(6, P6, None, None, 32, y_path=wino.YPATH_RECOMPUTE, y_groups=wino.YGROUPS_TAP)
+
+
 @pytest.mark.parametrize("name", ["ragged_f6_cout96", "f6_g64_cout128", "f4_two_row_blocks"])
 def test_default_path_bf16_output(cuda_dev, name):
     """Default options (AUTO path and kernel) with bf16 output, as the benchmark runs them."""
