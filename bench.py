@@ -67,6 +67,8 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=200)
+    ap.add_argument("--y-groups", default="tile", choices=["tile", "tap"],
+                    help="Y quantisation groups: tile (default reading) or tap (the per-tap option)")
     return ap.parse_args()
 
 
@@ -194,7 +196,8 @@ def run_ours(args, layer, rank, world):
     x_f32, x_bits = synth.make_input(layer)
     w = synth.make_weights(layer)
     sb, sg = synth.make_scales(layer)
-    plan = wino.Plan(layer.m, layer.points, sb, sg, layer.group)
+    y_groups = wino.YGROUPS_TAP if getattr(args, "y_groups", "tile") == "tap" else wino.YGROUPS_TILE
+    plan = wino.Plan(layer.m, layer.points, sb, sg, layer.group, y_groups=y_groups)
     N, H, W, Cin, Cout = layer.N, layer.H, layer.W, layer.Cin, layer.Cout
     if x_bits is not None:
         x = torch.from_numpy(x_bits.view(np.int16).copy()).view(torch.bfloat16).to(dev)
@@ -322,23 +325,23 @@ def oracle_sample(layer: synth.Layer, rows: int, images: int):
     return plan, xs, Uq, sU, flops
 
 
-def oracle_step(plan, xs, Uq, sU, G):
+def oracle_step(plan, xs, Uq, sU, G, per_tap=False):
     import oracle
     n2 = plan.n * plan.n
     N, H, W, _ = xs.shape
     Vq, sV, _ = oracle.input_transform(plan, xs, G)
     Y, _ = oracle.hadamard(n2, Vq, sV, Uq, sU, G)
-    Yq, sY = oracle.y_requant(n2, Y, G)
-    oracle.output_transform(plan, Yq, sY, N, H, W, G)
+    Yq, sY = oracle.y_requant(n2, Y, G, per_tap)
+    oracle.output_transform(plan, Yq, sY, N, H, W, G, per_tap)
 
 
-def cpu_baseline(layer: synth.Layer, budget_s: float = 12.0):
+def cpu_baseline(layer: synth.Layer, budget_s: float = 12.0, per_tap: bool = False):
     import oracle
     threads = oracle.set_threads(0)
     rows, images = 1, 1
     plan, xs, Uq, sU, flops = oracle_sample(layer, rows, images)
     t0 = time.perf_counter()
-    oracle_step(plan, xs, Uq, sU, layer.group)
+    oracle_step(plan, xs, Uq, sU, layer.group, per_tap)
     dt = time.perf_counter() - t0
     # grow the sample (whole images first) while it stays within the budget
     TH = -(-layer.H // layer.m)
@@ -349,12 +352,12 @@ def cpu_baseline(layer: synth.Layer, budget_s: float = 12.0):
             images = min(layer.N, images * 2)
         plan, xs, Uq, sU, flops = oracle_sample(layer, rows, images)
         t0 = time.perf_counter()
-        oracle_step(plan, xs, Uq, sU, layer.group)
+        oracle_step(plan, xs, Uq, sU, layer.group, per_tap)
         dt = time.perf_counter() - t0
     reps = max(1, int(budget_s / 2 / max(dt, 1e-3)))
     t0 = time.perf_counter()
     for _ in range(reps):
-        oracle_step(plan, xs, Uq, sU, layer.group)
+        oracle_step(plan, xs, Uq, sU, layer.group, per_tap)
     dt = (time.perf_counter() - t0) / reps
     return {"value": flops / dt / 1e12, "unit": UNIT, "cores": threads, "kind": "oracle",
             "sample": "%d image(s) x %d of %d tile rows of %s; input transform, Hadamard, Y requant, output "
@@ -362,6 +365,7 @@ def cpu_baseline(layer: synth.Layer, budget_s: float = 12.0):
 
 
 def run_reference(args, layer):
+    per_tap = args.y_groups == "tap"
     import oracle
     threads = oracle.set_threads(0)
     TH = -(-layer.H // layer.m)
@@ -369,19 +373,19 @@ def run_reference(args, layer):
     rows = 1
     plan, xs, Uq, sU, flops = oracle_sample(layer, rows, 1)
     t0 = time.perf_counter()
-    oracle_step(plan, xs, Uq, sU, layer.group)
+    oracle_step(plan, xs, Uq, sU, layer.group, per_tap)
     dt = time.perf_counter() - t0
     while dt * 2 <= budget and rows < TH:
         rows = min(TH, rows * 2)
         plan, xs, Uq, sU, flops = oracle_sample(layer, rows, 1)
         t0 = time.perf_counter()
-        oracle_step(plan, xs, Uq, sU, layer.group)
+        oracle_step(plan, xs, Uq, sU, layer.group, per_tap)
         dt = time.perf_counter() - t0
     for _ in range(args.warmup):
-        oracle_step(plan, xs, Uq, sU, layer.group)
+        oracle_step(plan, xs, Uq, sU, layer.group, per_tap)
     t0 = time.perf_counter()
     for _ in range(args.steps):
-        oracle_step(plan, xs, Uq, sU, layer.group)
+        oracle_step(plan, xs, Uq, sU, layer.group, per_tap)
     total = time.perf_counter() - t0
     value = args.steps * flops / total / 1e12
     sample = "1 image x %d of %d tile rows of %s per step" % (rows, TH, layer.describe())
@@ -397,7 +401,8 @@ def main():
     config = {"workload": "%s[%d]: %s" % (layer.workload, layer.index, layer.describe()), "model": layer.workload,
               "global_batch": layer.N * world, "seq_len": None, "H": layer.H, "W": layer.W, "Cin": layer.Cin,
               "Cout": layer.Cout, "m": layer.m, "group": layer.group, "parallelism": "dp%d" % world,
-              "l2": "flushed before every timed step (256 MiB write)", "output": "bf16 NHWC"}
+              "l2": "flushed before every timed step (256 MiB write)", "output": "bf16 NHWC",
+              "y_groups": args.y_groups}
     line = {"metric": METRIC, "unit": UNIT, "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int8 (fp32 transforms)",
             "data": "synthetic (seeded)", "config": config}
@@ -428,7 +433,7 @@ def main():
         return
     cpu = None
     if not args.no_cpu_baseline and world == 1:
-        cpu = cpu_baseline(layer)
+        cpu = cpu_baseline(layer, per_tap=args.y_groups == "tap")
     line.update(value=r["value"], ms_per_step=r["ms_per_step"], e2e=r["e2e"], roofline=r["roofline"],
                 cpu_baseline=cpu, clocks=r["clocks"], gpu_launches=r["gpu_launches"],
                 kernels=r["per_kernel"], y_path=r["y_path"], gemm=r["gemm"], impl="ours")

@@ -16,12 +16,13 @@
 // fp32 instruction per step (the per-channel chains are unchanged).  One 4-D
 // TMA box brings the CTA's halo patch (n rows x TX*m+2 columns x G channels;
 // outside the image the box reads zeros, which is the pad-1 border) into
-// shared memory.  V goes to shared memory half the taps at a time, a
-// [tap][64 channels] block per warp (rows padded to 68 words: conflict-free
-// 16-byte reads), where lane l owns one tap of each 32-channel chunk: its
-// absmax (the chunks of one group combine in registers, or in shared memory
-// across warps for G > 64), the group scale, and the 32 codes (quant4),
-// written as two 16-byte stores of the tap-major Vq.
+// shared memory.  V goes to shared memory in batches of taps (half of them for
+// F(6,3), all of them for the smaller tiles), a [tap][64 channels] block per
+// warp (rows padded to 68 words: conflict-free 16-byte reads); the lanes then
+// take the batch's (tap, 32-channel chunk) items in turn: the chunk's absmax
+// (the two chunks of a G=64 group combine across a lane pair, G >= 128 across
+// warps in shared memory), the group scale, and 32 codes (quant4), written as
+// two 16-byte stores of the tap-major Vq.
 #include <algorithm>
 
 #include "kernels.h"
@@ -46,16 +47,17 @@ struct Pair<float> {
 
 template <int M, typename Tin, int G>
 struct InCfg {
-    static constexpr int N = M + 2, N2 = N * N, H2 = N2 / 2;   // taps per half
+    static constexpr int N = M + 2, N2 = N * N;
+    static constexpr int NB = M == 6 ? 2 : 1;          // batches of taps staged in shared memory
+    static constexpr int TB = N2 / NB, RB = N / NB;    // taps and transform rows per batch
     static constexpr int kMaxThreads = 256;
     static constexpr int kPitch = 68;                   // words per V row in shared memory (64 channels + pad)
     static constexpr int kMaxWarps = kMaxThreads / 32;
-    static constexpr size_t kVbufBytes = sizeof(float) * kMaxWarps * H2 * kPitch;
     __host__ __device__ static size_t patch_bytes(int tx) { return sizeof(Tin) * N * (size_t)(tx * M + 2) * G; }
     __host__ __device__ static int threads(int tx) { return (tx * (G / 2) + 31) / 32 * 32; }
     // the V blocks reuse the patch's shared memory once every thread holds its patch values
     __host__ __device__ static size_t smem(int tx) {
-        const size_t v = sizeof(float) * (threads(tx) / 32) * H2 * kPitch;
+        const size_t v = sizeof(float) * (threads(tx) / 32) * TB * kPitch;
         return patch_bytes(tx) > v ? patch_bytes(tx) : v;
     }
 };
@@ -65,12 +67,12 @@ template <int M, uint64_t MASK, typename Tin, int G>
 __global__ void __maxnreg__(MASK == kMaskAll ? 255 : 168)
     input_transform_kernel(const __grid_constant__ CUtensorMap tmX, InputArgs p, TransformArgs tf, int TX) {
     using Cfg = InCfg<M, Tin, G>;
-    constexpr int N = M + 2, N2 = N * N, H2 = Cfg::H2, P = Cfg::kPitch;
+    constexpr int N = M + 2, P = Cfg::kPitch, NB = Cfg::NB, TB = Cfg::TB, RB = Cfg::RB;
     constexpr int CPW = G <= 64 ? 1 : G / 64;    // warps per group (G > 64)
     extern __shared__ __align__(128) unsigned char smem[];
     const Tin* patch = reinterpret_cast<const Tin*>(smem);   // [N][PW][G]
-    float* vbuf = reinterpret_cast<float*>(smem);             // [warps][H2][P], after the patch is consumed
-    __shared__ float red[Cfg::kMaxWarps][32];
+    float* vbuf = reinterpret_cast<float*>(smem);             // [warps][TB][P], after the patch is consumed
+    __shared__ float red[Cfg::kMaxWarps][TB];
     __shared__ uint64_t bar;
     __shared__ int load_ok;
 
@@ -132,65 +134,61 @@ __global__ void __maxnreg__(MASK == kMaskAll ? 255 : 168)
 #pragma unroll
         for (int i = 0; i < N; ++i) v[i][l] = tcol[i];
     }
-    float* vw = vbuf + (size_t)warp * H2 * P;
+    float* vw = vbuf + (size_t)warp * TB * P;
 #pragma unroll
-    for (int h = 0; h < 2; ++h) {
-        // 3. V = T1 B for the rows of this half: taps h*H2 .. h*H2 + H2 - 1
-        if (h) __syncwarp();   // the previous half's codes are written
+    for (int h = 0; h < NB; ++h) {
+        // 3. V = T1 B for the rows of this batch: taps h*TB .. h*TB + TB - 1
+        if (h) __syncwarp();   // the previous batch's codes are written
 #pragma unroll
-        for (int i = h * N / 2; i < (h + 1) * N / 2; ++i) {
+        for (int i = h * RB; i < (h + 1) * RB; ++i) {
 #pragma unroll
             for (int j = 0; j < N; ++j) {
                 uint64_t acc = 0ull;
 #pragma unroll
                 for (int l = 0; l < N; ++l)
                     if ((MASK >> (j * N + l)) & 1ull) acc = f2_fma(v[i][l], tf.BTd[j * N + l], acc);
-                *reinterpret_cast<uint64_t*>(vw + (i * N + j - h * H2) * P + 2 * lane) = acc;
+                *reinterpret_cast<uint64_t*>(vw + (i * N + j - h * TB) * P + 2 * lane) = acc;
             }
         }
         __syncwarp();
 
-        // 4. absmax of this lane's tap over each 32-channel chunk of the warp
-        const bool own = lane < H2;
-        const int tap = h * H2 + lane;
-        const float* vrow = vw + (own ? lane : 0) * P;
-        float am[2] = {0.0f, 0.0f};
+        // 4.-5. items (tap, chunk) of the batch, one per lane and round: absmax of the chunk's
+        // 32 channels, the group maximum (G = 64: the two chunks of a tap sit on lanes 2k and
+        // 2k+1; G > 64: across CPW warps in shared memory), the scale and 32 codes
 #pragma unroll
-        for (int c = 0; c < 2; ++c) {
-            const float4* row = reinterpret_cast<const float4*>(vrow + 32 * c);
+        for (int r0 = 0; r0 < 2 * TB; r0 += 32) {
+            const int k = r0 + lane;
+            const bool own = k < 2 * TB;
+            const int tl_ = own ? k >> 1 : 0, c = k & 1;
+            const int tap = h * TB + tl_;
+            const float4* row = reinterpret_cast<const float4*>(vw + tl_ * P + 32 * c);
+            float am = 0.0f;
 #pragma unroll
             for (int j = 0; j < 8; ++j) {
                 const float4 x4 = row[j];
-                am[c] = max_abs3(am[c], x4.x, x4.y);
-                am[c] = max_abs3(am[c], x4.z, x4.w);
+                am = max_abs3(am, x4.x, x4.y);
+                am = max_abs3(am, x4.z, x4.w);
             }
-        }
-        // group maxima: G = 32: one chunk; G = 64: the warp's two chunks; G > 64: CPW warps
-        if (G == 64) {
-            am[0] = am[1] = fmaxf(am[0], am[1]);
-        } else if (G > 64) {
-            red[warp][lane] = fmaxf(am[0], am[1]);
-            __syncthreads();
-            const int leader = warp - warp % CPW;
-            float a = 0.0f;
+            if (!own) am = 0.0f;
+            if (G >= 64) am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, 1));
+            if (G > 64) {
+                if (c == 0 && own) red[warp][tl_] = am;
+                __syncthreads();
+                const int leader = warp - warp % CPW;
+                float a = 0.0f;
 #pragma unroll
-            for (int i = 0; i < CPW; ++i) a = fmaxf(a, red[leader + i][lane]);
-            am[0] = am[1] = a;
-            __syncthreads();   // red is reused by the next half
-        }
-
-        // 5. scales and codes, chunk by chunk
-#pragma unroll
-        for (int c = 0; c < 2; ++c) {
+                for (int i = 0; i < CPW; ++i) a = fmaxf(a, red[leader + i][tl_]);
+                am = a;
+                __syncthreads();   // red is reused by the next round
+            }
             const int th = warp * 32 + 16 * c;     // first thread of the chunk
             const int ctl = th / (G / 2);          // its tile
             const int ch = 2 * (th % (G / 2));     // its first channel within the group
             const int tx = tx0 + ctl;
             if (!own || ctl >= TX || tx >= p.TW) continue;
             const long t = (long)row_id * p.TW + tx;
-            const QScale q = make_qscale(am[c]);
+            const QScale q = make_qscale(am);
             if (ch == 0) p.sV[((size_t)tap * (p.Cin / G) + g) * p.T_pad + t] = q.s;
-            const float4* row = reinterpret_cast<const float4*>(vrow + 32 * c);
             uint32_t w[8];
 #pragma unroll
             for (int j = 0; j < 8; ++j) {

@@ -165,8 +165,9 @@ def workload(name: str, seed: int = 0) -> List[Layer]:
     if name == "tiny":
         return [Layer("tiny", 0, 4, 1, 16, 16, 32, 32, 32, "f32", "normal", 1.0, "identity", seed)]
     if name == "resnet18":
-        return [Layer("resnet18", 0, 6, 32, 56, 56, 64, 64, 32, "bf16", "relu_normal", 2.0,
-                      "loguniform", seed)]
+        # [0] the F(6,3) layer; [1] the same layer as F(2,3) and [2] as F(4,3) (tile-size comparison)
+        return [Layer("resnet18", i, m, 32, 56, 56, 64, 64, 32, "bf16", "relu_normal", 2.0, "loguniform", seed)
+                for i, m in enumerate((6, 2, 4))]
     if name == "resnet34":
         shapes = [(64, 56), (128, 28), (256, 14), (512, 7)]
         return [Layer("resnet34", i, 6, 64, hw, hw, c, c, 32, "bf16", "relu_normal", 2.0,
