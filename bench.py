@@ -50,9 +50,6 @@ NCU_TRAFFIC = {
     # (workload, layer, kernel) -> dram read+write bytes per launch from one ncu capture of the
     # CURRENT kernel (profiles/resnet18_f63_g32_launches_and_full.md); entries are removed
     # whenever that kernel changes.
-    ("resnet18", 0, "input_transform"): 25461248,
-    ("resnet18", 0, "hadamard_absmax"): 15272960,
-    ("resnet18", 0, "hadamard_quant"): 15283200,
     ("resnet18", 0, "output_transform"): 13175040,
 }
 
