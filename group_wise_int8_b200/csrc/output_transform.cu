@@ -31,7 +31,8 @@ __device__ __forceinline__ uint64_t codes2_to_f2(uint32_t x) {
 }
 
 template <int M, uint64_t MASK, bool SRC_Y32, bool BF16_OUT, bool DEBUG>
-__global__ void __launch_bounds__(128, 4) output_transform_kernel(OutputArgs p, TransformArgs tf) {
+// fp32-Y source: six CTAs per SM (measured faster despite spills: the loads dominate)
+__global__ void __launch_bounds__(128, SRC_Y32 ? 6 : 4) output_transform_kernel(OutputArgs p, TransformArgs tf) {
     constexpr int N = M + 2;
     grid_dependents_launch();
     grid_dependency_wait();
