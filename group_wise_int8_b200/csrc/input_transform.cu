@@ -63,8 +63,9 @@ struct InCfg {
 };
 
 template <int M, uint64_t MASK, typename Tin, int G>
-// at most 168 registers: two CTAs of a 10-tile row (160 threads) share an SM
-__global__ void __maxnreg__(MASK == kMaskAll ? 255 : 168)
+// at most 128 registers: three CTAs of a 10-tile row (160 threads) share an SM (measured best;
+// the few spilled bytes cost less than the lost occupancy)
+__global__ void __maxnreg__(MASK == kMaskAll ? 255 : 128)
     input_transform_kernel(const __grid_constant__ CUtensorMap tmX, InputArgs p, TransformArgs tf, int TX) {
     using Cfg = InCfg<M, Tin, G>;
     constexpr int N = M + 2, P = Cfg::kPitch, NB = Cfg::NB, TB = Cfg::TB, RB = Cfg::RB;
