@@ -50,7 +50,7 @@ struct InCfg {
     static constexpr int N = M + 2, N2 = N * N;
     static constexpr int NB = M == 6 ? 2 : 1;          // batches of taps staged in shared memory
     static constexpr int TB = N2 / NB, RB = N / NB;    // taps and transform rows per batch
-    static constexpr int kMaxThreads = 256;
+    static constexpr int kMaxThreads = 160;   // measured: up to 10 tiles of G=32 per CTA
     static constexpr int kPitch = 68;                   // words per V row in shared memory (64 channels + pad)
     static constexpr int kMaxWarps = kMaxThreads / 32;
     __host__ __device__ static size_t patch_bytes(int tx) { return sizeof(Tin) * N * (size_t)(tx * M + 2) * G; }
