@@ -167,6 +167,46 @@ __device__ __forceinline__ Quad quant4(float v0, float v1, float v2, float v3, c
     return o;
 }
 
+// Codes of NV values of one group (NV a multiple of 4), packed four per word,
+// by the argument of quant4 with a single check for all NV values (the
+// fallback, taken when any of them lies near a half-integer, is quant_code_fast
+// for all of them).
+template <int NV>
+__device__ __forceinline__ void quant_chunk(const float (&v)[NV], const QScale& q, uint32_t (&w)[NV / 4]) {
+    const uint64_t magic2 = f2_pack(kRoundMagic, kRoundMagic);
+    if (q.r != 0.0f || q.s == 0.0f) {
+        const uint64_t r2 = f2_pack(q.r, q.r);
+        uint64_t a[NV / 2];
+        float dmax = 0.0f;
+#pragma unroll
+        for (int i = 0; i < NV / 2; ++i) {
+            const uint64_t t = f2_mul(f2_pack(v[2 * i], v[2 * i + 1]), r2);
+            a[i] = f2_add(t, magic2);
+            float d0, d1;
+            f2_unpack(f2_sub(t, f2_sub(a[i], magic2)), d0, d1);
+            dmax = max_abs3(dmax, d0, d1);
+        }
+        if (dmax < 0.5f - 0x1p-12f) {
+#pragma unroll
+            for (int i = 0; i < NV / 4; ++i) {
+                float a0, a1, a2, a3;
+                f2_unpack(a[2 * i], a0, a1);
+                f2_unpack(a[2 * i + 1], a2, a3);
+                w[i] = __byte_perm(__byte_perm(__float_as_uint(a0), __float_as_uint(a1), 0x0040),
+                                   __byte_perm(__float_as_uint(a2), __float_as_uint(a3), 0x0040), 0x5410);
+            }
+            return;
+        }
+    }
+#pragma unroll
+    for (int i = 0; i < NV / 4; ++i) {
+        const int c0 = quant_code_fast(v[4 * i], q), c1 = quant_code_fast(v[4 * i + 1], q);
+        const int c2 = quant_code_fast(v[4 * i + 2], q), c3 = quant_code_fast(v[4 * i + 3], q);
+        w[i] = (uint32_t)(c0 & 0xff) | ((uint32_t)(c1 & 0xff) << 8) | ((uint32_t)(c2 & 0xff) << 16) |
+               ((uint32_t)(c3 & 0xff) << 24);
+    }
+}
+
 // Recursive-halving max over the 32 lanes of a warp for 64 values per lane.
 // a[0..63] holds this lane's values; on return a[0], a[1] hold the maxima
 // over all lanes of entries 2*lane and 2*lane + 1.

@@ -429,9 +429,7 @@ __global__ void __launch_bounds__(TcCfg<BN>::kThreads, 1)
                         if (MODE == kModeQuant) {
                             if (valid) {
                                 uint32_t q[CPT / 4];
-#pragma unroll
-                                for (int e = 0; e < CPT / 4; ++e)
-                                    q[e] = quant4(y[4 * e], y[4 * e + 1], y[4 * e + 2], y[4 * e + 3], qy[h]).packed;
+                                quant_chunk<CPT>(y, qy[h], q);
                                 int8_t* dst = p.Yq + ((size_t)tap * p.T + row) * p.Cout + colg[h];
                                 if (CPT == 8) {
                                     *reinterpret_cast<uint2*>(dst) = make_uint2(q[0], q[1 % (CPT / 4)]);

@@ -192,9 +192,20 @@ __global__ void __maxnreg__(MASK == kMaskAll ? 255 : 128)
             if (ch == 0) p.sV[((size_t)tap * (p.Cin / G) + g) * p.T_pad + t] = q.s;
             uint32_t w[8];
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                const float4 x4 = row[j];
-                w[j] = quant4(x4.x, x4.y, x4.z, x4.w, q).packed;
+            for (int hh = 0; hh < 2; ++hh) {   // two 16-value halves of the chunk, one exactness check each
+                float xv[16];
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const float4 x4 = row[4 * hh + j];
+                    xv[4 * j] = x4.x;
+                    xv[4 * j + 1] = x4.y;
+                    xv[4 * j + 2] = x4.z;
+                    xv[4 * j + 3] = x4.w;
+                }
+                uint32_t wh[4];
+                quant_chunk<16>(xv, q, wh);
+#pragma unroll
+                for (int j = 0; j < 4; ++j) w[4 * hh + j] = wh[j];
             }
             uint4* dst = reinterpret_cast<uint4*>(p.Vq + ((size_t)tap * p.T_pad + t) * p.Cin + g * G + ch);
             dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
