@@ -229,6 +229,7 @@ int run_conv(wino_plan_s* p, const void* x, int x_dtype, int N, int H, int W, in
     oa.sY_dbg = sYd;
     oa.out = y;
     oa.ytap = L.ytap ? 1 : 0;
+    oa.err = err;
     prof_mark(p, slot++, st);
     e = launch_output_transform(oa, p->tf, p->mat.m, p->at_masked, L.y_path == WINO_YPATH_Y32, y_dtype == WINO_BF16,
                                 st);

@@ -96,6 +96,7 @@ struct OutputArgs {
     float* sY_dbg;         // debug copy of sY [T][ngo], or null
     void* out;             // [N][H][W][Cout] fp32 or bf16
     int ytap;              // per-tap Y groups (Y32 source; sY_dbg is then [T][n2][ngo])
+    int* err;              // device error word (bounded waits)
 };
 cudaError_t launch_output_transform(const OutputArgs& a, const TransformArgs& tf, int m, bool masked, bool src_y32,
                                     bool bf16_out, cudaStream_t st);

@@ -14,7 +14,10 @@
 // the per-cout chains and their order unchanged).  Lanes run along cout
 // pairs: every tap load and output store of a warp is contiguous.  Z is built
 // one column of Y at a time, so only Z and one Y column are live.
+#include <cstring>
+
 #include "kernels.h"
+#include "sm100.cuh"
 
 namespace wino {
 namespace {
@@ -32,10 +35,33 @@ __device__ __forceinline__ uint64_t codes2_to_f2(uint32_t x) {
 
 template <int M, uint64_t MASK, bool SRC_Y32, bool BF16_OUT, bool DEBUG>
 // fp32-Y source: six CTAs per SM (measured faster despite spills: the loads dominate)
-__global__ void __launch_bounds__(128, SRC_Y32 ? 6 : 4) output_transform_kernel(OutputArgs p, TransformArgs tf) {
-    constexpr int N = M + 2;
+__global__ void __launch_bounds__(128, SRC_Y32 ? 6 : 4)
+    output_transform_kernel(const __grid_constant__ CUtensorMap tmYq, OutputArgs p, TransformArgs tf) {
+    constexpr int N = M + 2, N2 = N * N;
+    // int8 source: the CTA's 256 contiguous bytes of every tap, one 2-D TMA box
+    __shared__ __align__(128) uint8_t ysm[SRC_Y32 ? 16 : 256 * N2];
+    __shared__ uint64_t bar;
+    __shared__ int load_ok;
     grid_dependents_launch();
     grid_dependency_wait();
+    if (!SRC_Y32) {
+        if (threadIdx.x == 0) {
+            sm100::mbar_init(&bar, 1);
+            sm100::fence_mbar_init();
+            sm100::mbar_arrive_expect_tx(&bar, 256u * N2);
+            sm100::tma_load_2d(ysm, &tmYq, &bar, (int)(blockIdx.x * 256u), 0);
+            load_ok = 1;
+            const unsigned long long t0 = sm100::globaltimer();
+            while (!sm100::mbar_try_wait(&bar, 0))
+                if (sm100::globaltimer() - t0 > sm100::kWaitLimitNs) {
+                    load_ok = 0;
+                    atomicCAS(p.err, 0, sm100::kDevErrTimeout);
+                    break;
+                }
+        }
+        __syncthreads();
+        if (!load_ok) return;   // uniform; the host reads the error word
+    }
     const long i = (long)blockIdx.x * blockDim.x + threadIdx.x;
     const int cpairs = p.Cout >> 1;
     const long t = i / cpairs;
@@ -70,7 +96,7 @@ __global__ void __launch_bounds__(128, SRC_Y32 ? 6 : 4) output_transform_kernel(
         } else {
 #pragma unroll
             for (int xi = 0; xi < N; ++xi) {
-                const uint32_t x = *reinterpret_cast<const uint16_t*>(p.Yq + base + (size_t)(xi * N + nu) * tstride);
+                const uint32_t x = *reinterpret_cast<const uint16_t*>(ysm + (xi * N + nu) * 256 + 2 * threadIdx.x);
                 Yc[xi] = f2_mul(s2, codes2_to_f2(x));
             }
         }
@@ -237,11 +263,21 @@ cudaError_t launch_m(const OutputArgs& a, const TransformArgs& tf, bool src_y32,
                      cudaStream_t st) {
     const long threads = a.T * (long)(a.Cout / 2);
     const dim3 grid((unsigned)((threads + 127) / 128));
+    CUtensorMap tm;
+    std::memset(&tm, 0, sizeof(tm));
+    if (!src_y32) {   // Yq [n2][T*Cout] bytes; box 256 x n2 (a CTA's 128 cout pairs, every tap)
+        const cuuint64_t dims[2] = {(cuuint64_t)a.T * a.Cout, (cuuint64_t)a.n2};
+        const cuuint64_t strides[1] = {(cuuint64_t)a.T * a.Cout};
+        const cuuint32_t box[2] = {256u, (cuuint32_t)a.n2};
+        if (!make_tensor_map(&tm, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, a.Yq, dims, strides, box,
+                             CU_TENSOR_MAP_SWIZZLE_NONE))
+            return cudaErrorInvalidValue;
+    }
     if (a.ytap)
         return bf16_out ? launch_dependent(output_transform_ytap_kernel<M, MASK, true>, grid, dim3(128), 0, st, a, tf)
                         : launch_dependent(output_transform_ytap_kernel<M, MASK, false>, grid, dim3(128), 0, st, a, tf);
 #define WINO_OUT_LAUNCH(Y32, BF, DBG) \
-    return launch_dependent(output_transform_kernel<M, MASK, Y32, BF, DBG>, grid, dim3(128), 0, st, a, tf)
+    return launch_dependent(output_transform_kernel<M, MASK, Y32, BF, DBG>, grid, dim3(128), 0, st, tm, a, tf)
     if (src_y32) {
         if (bf16_out) {
             if (debug) WINO_OUT_LAUNCH(true, true, true); else WINO_OUT_LAUNCH(true, true, false);
