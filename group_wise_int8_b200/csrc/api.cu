@@ -25,6 +25,10 @@ struct wino_plan_s {
     // per-kernel timing (wino_profile_begin / wino_profile_end)
     std::vector<cudaEvent_t> prof_events;
     int prof_max_calls = 0, prof_calls = 0, prof_launches = 0;
+    // pipelined host entry point: plan-owned copy streams and events on device host_dev
+    int host_dev = -1;
+    cudaStream_t copy_in = nullptr, copy_out = nullptr;
+    std::vector<cudaEvent_t> host_events;
 };
 
 namespace {
@@ -126,6 +130,40 @@ int cuda_status(wino_plan_s* p, cudaError_t e) {
     if (e == cudaSuccess) return WINO_OK;
     p->last_cuda = (int)e;
     return WINO_ERR_CUDA;
+}
+
+constexpr int kMaxHostChunks = 4;
+
+// The host entry point's copy streams and events, created on the current device.
+int ensure_host_streams(wino_plan_s* p) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_status(p, e);
+    if (p->copy_in && p->host_dev == dev) return WINO_OK;
+    for (cudaEvent_t ev : p->host_events) cudaEventDestroy(ev);
+    p->host_events.clear();
+    if (p->copy_in) cudaStreamDestroy(p->copy_in);
+    if (p->copy_out) cudaStreamDestroy(p->copy_out);
+    p->copy_in = p->copy_out = nullptr;
+    if ((e = cudaStreamCreateWithFlags(&p->copy_in, cudaStreamNonBlocking)) != cudaSuccess ||
+        (e = cudaStreamCreateWithFlags(&p->copy_out, cudaStreamNonBlocking)) != cudaSuccess)
+        return cuda_status(p, e);
+    p->host_events.assign(1 + 3 * kMaxHostChunks, nullptr);
+    for (cudaEvent_t& ev : p->host_events)
+        if ((e = cudaEventCreateWithFlags(&ev, cudaEventDisableTiming)) != cudaSuccess) return cuda_status(p, e);
+    p->host_dev = dev;
+    return WINO_OK;
+}
+
+// Folds a chunk's device error word into the call's (first error wins).
+__global__ void error_merge_kernel(int* dst, const int* src) {
+    const int v = *src;
+    if (v) atomicCAS(dst, 0, v);
+}
+
+cudaError_t launch_error_merge(int* dst, const int* src, cudaStream_t st) {
+    error_merge_kernel<<<1, 1, 0, st>>>(dst, src);
+    return cudaGetLastError();
 }
 
 constexpr int kMaxLaunches = 4;
@@ -302,8 +340,12 @@ int wino_plan(wino_plan_t* out, int m, const double* points, const float* S_B, c
 }
 
 int wino_plan_destroy(wino_plan_t p) {
-    if (p)
+    if (p) {
         for (cudaEvent_t ev : p->prof_events) cudaEventDestroy(ev);
+        for (cudaEvent_t ev : p->host_events) cudaEventDestroy(ev);
+        if (p->copy_in) cudaStreamDestroy(p->copy_in);
+        if (p->copy_out) cudaStreamDestroy(p->copy_out);
+    }
     delete p;
     return WINO_OK;
 }
@@ -366,19 +408,65 @@ int wino_conv2d_int8_host(wino_plan_t p, const void* x_host, int x_dtype, int N,
     if (!p || !x_host || !y_host || !ws) return WINO_ERR_INVALID_ARG;
     int rc = check_shape(p, N, H, W, Cin, Cout);
     if (rc) return rc;
-    const size_t need = make_layout(p, N, H, W, Cin, Cout).total;
+    const Layout L = make_layout(p, N, H, W, Cin, Cout);
+    const size_t need = L.total;
     const size_t stage = wino_host_staging_bytes(p, N, H, W, Cin, Cout, x_dtype, y_dtype);
     if (ws_bytes < need + stage) return WINO_ERR_WORKSPACE;
     const size_t xs = x_dtype == WINO_BF16 ? 2 : 4, ys = y_dtype == WINO_BF16 ? 2 : 4;
-    const size_t xbytes = xs * N * H * W * Cin, ybytes = ys * N * H * W * Cout;
+    const size_t xrow = xs * H * W * Cin, yrow = ys * H * W * Cout;   // bytes per image
     unsigned char* xd = static_cast<unsigned char*>(ws) + need;
-    unsigned char* yd = xd + up(xbytes, kAlign);
+    unsigned char* yd = xd + up(xrow * N, kAlign);
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    cudaError_t e = cudaMemcpyAsync(xd, x_host, xbytes, cudaMemcpyHostToDevice, st);
-    if (e != cudaSuccess) return cuda_status(p, e);
-    rc = run_conv(p, xd, x_dtype, N, H, W, Cin, wt, Cout, yd, y_dtype, ws, need, st);
-    if (rc) return rc;
-    return cuda_status(p, cudaMemcpyAsync(y_host, yd, ybytes, cudaMemcpyDeviceToHost, st));
+    cudaError_t e;
+
+    // Chunks of images: every tile, and so every result, belongs to one image, so the
+    // chunks give the same bytes as one call.  Two chunk workspaces must fit below the
+    // whole call's error word (which collects the chunks' errors).
+    int K = std::min(N, kMaxHostChunks), Nc = N;
+    size_t need_c = need;
+    for (; K > 1; --K) {
+        Nc = (N + K - 1) / K;
+        need_c = up(make_layout(p, Nc, H, W, Cin, Cout).total, kAlign);
+        if (2 * need_c <= L.off_err) break;
+    }
+    if (K <= 1) {
+        if ((e = cudaMemcpyAsync(xd, x_host, xrow * N, cudaMemcpyHostToDevice, st)) != cudaSuccess)
+            return cuda_status(p, e);
+        rc = run_conv(p, xd, x_dtype, N, H, W, Cin, wt, Cout, yd, y_dtype, ws, need, st);
+        if (rc) return rc;
+        return cuda_status(p, cudaMemcpyAsync(y_host, yd, yrow * N, cudaMemcpyDeviceToHost, st));
+    }
+    K = (N + Nc - 1) / Nc;
+    if ((rc = ensure_host_streams(p)) != WINO_OK) return rc;
+    cudaEvent_t* ev = p->host_events.data();   // [0]: start, [1 + 3k ..]: in, compute, out of chunk k
+    int* err = reinterpret_cast<int*>(static_cast<unsigned char*>(ws) + L.off_err);
+    if ((e = cudaMemsetAsync(err, 0, sizeof(int), st)) != cudaSuccess) return cuda_status(p, e);
+    cudaEventRecord(ev[0], st);
+    cudaStreamWaitEvent(p->copy_in, ev[0], 0);
+    cudaStreamWaitEvent(p->copy_out, ev[0], 0);
+    const unsigned char* xh = static_cast<const unsigned char*>(x_host);
+    unsigned char* yh = static_cast<unsigned char*>(y_host);
+    for (int k = 0; k < K; ++k) {
+        const int n0 = k * Nc, nk = std::min(Nc, N - n0);
+        unsigned char* buf = static_cast<unsigned char*>(ws) + (size_t)(k & 1) * need_c;
+        if ((e = cudaMemcpyAsync(xd + xrow * n0, xh + xrow * n0, xrow * nk, cudaMemcpyHostToDevice, p->copy_in)) !=
+            cudaSuccess)
+            return cuda_status(p, e);
+        cudaEventRecord(ev[1 + 3 * k], p->copy_in);
+        cudaStreamWaitEvent(st, ev[1 + 3 * k], 0);
+        rc = run_conv(p, xd + xrow * n0, x_dtype, nk, H, W, Cin, wt, Cout, yd + yrow * n0, y_dtype, buf, need_c, st);
+        if (rc) return rc;
+        const Layout Lk = make_layout(p, nk, H, W, Cin, Cout);
+        if ((e = launch_error_merge(err, reinterpret_cast<const int*>(buf + Lk.off_err), st)) != cudaSuccess)
+            return cuda_status(p, e);
+        cudaEventRecord(ev[2 + 3 * k], st);
+        cudaStreamWaitEvent(p->copy_out, ev[2 + 3 * k], 0);
+        if ((e = cudaMemcpyAsync(yh + yrow * n0, yd + yrow * n0, yrow * nk, cudaMemcpyDeviceToHost, p->copy_out)) !=
+            cudaSuccess)
+            return cuda_status(p, e);
+        cudaEventRecord(ev[3 + 3 * k], p->copy_out);
+    }
+    return cuda_status(p, cudaStreamWaitEvent(st, ev[3 * K], 0));
 }
 
 int wino_check_device_error(wino_plan_t p, const void* ws, int N, int H, int W, int Cin, int Cout, void* stream) {

@@ -203,11 +203,15 @@ size_t wino_host_staging_bytes(wino_plan_t plan, int N, int H, int W, int Cin, i
 
 /*
  * wino_conv2d_int8_host -- same convolution with HOST input and output
- * buffers: copies x_host to the device, runs wino_conv2d_int8, copies the
- * result to y_host, all asynchronously on stream (pinned host memory gives
- * truly asynchronous copies).  ws_dev must hold wino_workspace_bytes() +
- * wino_host_staging_bytes().  The caller synchronises the stream before
- * reading y_host.
+ * buffers: copies x_host to the device, runs the convolution, copies the
+ * result to y_host, all asynchronously with respect to stream (pinned host
+ * memory gives truly asynchronous copies).  When N >= 2 the batch is cut into
+ * up to 4 chunks of images, pipelined: the copy of chunk k+1 in and of chunk
+ * k-1 out overlap the convolution of chunk k (the copies run on two streams
+ * the plan owns, ordered after and before `stream` by events; results are
+ * identical to one call, every tile belonging to one image).  ws_dev must hold
+ * wino_workspace_bytes() + wino_host_staging_bytes().  The caller synchronises
+ * `stream` before reading y_host.  Calls on one plan must not run concurrently.
  */
 int wino_conv2d_int8_host(wino_plan_t plan, const void* x_host, int x_dtype, int N, int H, int W, int Cin,
                            const void* wt_dev, int Cout, void* y_host, int y_dtype, void* ws_dev, size_t ws_bytes,

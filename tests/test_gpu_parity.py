@@ -136,6 +136,31 @@ def test_host_entry_point_matches_device_call(cuda_dev):
     assert torch.equal(y_host, y_dev.cpu())
 
 
+@pytest.mark.parametrize("N", [3, 5, 9])
+def test_host_entry_point_chunks_match_device_call(cuda_dev, N):
+    """The host entry point pipelines chunks of images; its bytes equal one device call."""
+    layer = synth.random_layer(4, 6, N, 14, 13, 64, 64, 32, dtype="f32", act="relu_normal",
+                               scales="loguniform", workload="host_chunks")
+    x_f32, _ = synth.make_input(layer)
+    w = synth.make_weights(layer)
+    sb, sg = synth.make_scales(layer)
+    plan = wino.Plan(6, P6, sb, sg, 32)
+    H, W, Cin, Cout = 14, 13, 64, 64
+    wt = plan.transform_weights(torch.from_numpy(w).cuda())
+    x_host = torch.from_numpy(x_f32).pin_memory()
+    y_host = torch.empty((N, H, W, Cout), dtype=torch.float32).pin_memory()
+    ws = torch.empty(plan.workspace_bytes(N, H, W, Cin, Cout) +
+                     plan.host_staging_bytes(N, H, W, Cin, Cout, torch.float32, torch.float32),
+                     dtype=torch.uint8, device="cuda")
+    ws.fill_(0x5A)
+    plan.conv2d_host(x_host, wt, Cout, y_host, ws)
+    torch.cuda.synchronize()
+    assert plan.check_device_error(ws, N, H, W, Cin, Cout) == wino.OK
+    y_dev = plan.conv2d(x_host.cuda(), wt, Cout, out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    assert torch.equal(y_host, y_dev.cpu())
+
+
 def test_repeated_calls_reuse_workspace(cuda_dev):
     """The workspace carries nothing between calls: a second call on a dirty
     workspace gives the same bits."""
