@@ -18,7 +18,7 @@
 // outside the image the box reads zeros, which is the pad-1 border) into
 // shared memory.  V goes to shared memory in batches of taps (half of them for
 // F(6,3), all of them for the smaller tiles), a [tap][64 channels] block per
-// warp (rows padded to 68 words: conflict-free 16-byte reads); the lanes then
+// warp (rows of 72 words, the second chunk at word 36: conflict-free 16-byte reads); the lanes then
 // take the batch's (tap, 32-channel chunk) items in turn: the chunk's absmax
 // (the two chunks of a G=64 group combine across a lane pair, G >= 128 across
 // warps in shared memory), the group scale, and 32 codes (quant4), written as
@@ -51,7 +51,10 @@ struct InCfg {
     static constexpr int NB = M == 6 ? 2 : 1;          // batches of taps staged in shared memory
     static constexpr int TB = N2 / NB, RB = N / NB;    // taps and transform rows per batch
     static constexpr int kMaxThreads = 160;   // measured: up to 10 tiles of G=32 per CTA
-    static constexpr int kPitch = 68;                   // words per V row in shared memory (64 channels + pad)
+    // words per V row in shared memory: chunk 0 at word 0, chunk 1 at word 36 (so the two chunk
+    // rows of one tap start on different banks), pitch 72 (8 taps x 2 chunks of float4 reads per
+    // quarter warp hit 32 distinct banks)
+    static constexpr int kPitch = 72, kChunk1 = 36;
     static constexpr int kMaxWarps = kMaxThreads / 32;
     __host__ __device__ static size_t patch_bytes(int tx) { return sizeof(Tin) * N * (size_t)(tx * M + 2) * G; }
     __host__ __device__ static int threads(int tx) { return (tx * (G / 2) + 31) / 32 * 32; }
@@ -68,7 +71,7 @@ template <int M, uint64_t MASK, typename Tin, int G>
 __global__ void __maxnreg__(MASK == kMaskAll ? 255 : 128)
     input_transform_kernel(const __grid_constant__ CUtensorMap tmX, InputArgs p, TransformArgs tf, int TX) {
     using Cfg = InCfg<M, Tin, G>;
-    constexpr int N = M + 2, P = Cfg::kPitch, NB = Cfg::NB, TB = Cfg::TB, RB = Cfg::RB;
+    constexpr int N = M + 2, P = Cfg::kPitch, C1 = Cfg::kChunk1, NB = Cfg::NB, TB = Cfg::TB, RB = Cfg::RB;
     constexpr int CPW = G <= 64 ? 1 : G / 64;    // warps per group (G > 64)
     extern __shared__ __align__(128) unsigned char smem[];
     const Tin* patch = reinterpret_cast<const Tin*>(smem);   // [N][PW][G]
@@ -148,7 +151,7 @@ __global__ void __maxnreg__(MASK == kMaskAll ? 255 : 128)
 #pragma unroll
                 for (int l = 0; l < N; ++l)
                     if ((MASK >> (j * N + l)) & 1ull) acc = f2_fma(v[i][l], tf.BTd[j * N + l], acc);
-                *reinterpret_cast<uint64_t*>(vw + (i * N + j - h * TB) * P + 2 * lane) = acc;
+                *reinterpret_cast<uint64_t*>(vw + (i * N + j - h * TB) * P + 2 * lane + (lane >= 16 ? C1 - 32 : 0)) = acc;
             }
         }
         __syncwarp();
@@ -162,7 +165,7 @@ __global__ void __maxnreg__(MASK == kMaskAll ? 255 : 128)
             const bool own = k < 2 * TB;
             const int tl_ = own ? k >> 1 : 0, c = k & 1;
             const int tap = h * TB + tl_;
-            const float4* row = reinterpret_cast<const float4*>(vw + tl_ * P + 32 * c);
+            const float4* row = reinterpret_cast<const float4*>(vw + tl_ * P + C1 * c);
             float am = 0.0f;
 #pragma unroll
             for (int j = 0; j < 8; ++j) {
