@@ -19,7 +19,7 @@ CSRC = os.path.join(HERE, "csrc")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(HERE, "libwino_b200.so")
 SOURCES = ["plan.cpp", "api.cu", "weight_transform.cu", "input_transform.cu", "hadamard_tc.cu",
-           "hadamard_simt.cu", "output_transform.cu", "noalloc.cu"]
+           "hadamard_simt.cu", "output_transform.cu", "input_quant.cu", "noalloc.cu"]
 HEADERS = ["plan.h", "common.cuh", "sm100.cuh", "kernels.h"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 

@@ -42,8 +42,8 @@ struct Layout {
     int TH = 0, TW = 0, n2 = 0, ng = 0, ngo = 0;
     long T = 0, T_pad = 0;
     int y_path = 0, gemm = 0;
-    bool dbg_yq = false, dbg_acc = false, ytap = false;
-    size_t off_vq = 0, off_sv = 0, off_amax = 0, off_yq = 0, off_y32 = 0, off_sy = 0, off_acc = 0, off_err = 0;
+    bool dbg_yq = false, dbg_acc = false, ytap = false, xq = false;
+    size_t off_xq = 0, off_vq = 0, off_sv = 0, off_amax = 0, off_yq = 0, off_y32 = 0, off_sy = 0, off_acc = 0, off_err = 0;
     size_t total = 0;
 };
 
@@ -97,7 +97,12 @@ Layout make_layout(const wino_plan_s* p, int N, int H, int W, int Cin, int Cout)
                       : (p->opts.y_path == WINO_YPATH_AUTO ? choose_y_path(p, L.T, Cin, Cout, L.n2) : p->opts.y_path);
     L.dbg_yq = (p->opts.debug & WINO_DEBUG_YQ) != 0;
     L.dbg_acc = (p->opts.debug & WINO_DEBUG_ACC32) != 0;
+    L.xq = p->opts.x_int8 != 0;
     size_t off = 0;
+    if (L.xq) {  // fp32 copy of x after its group-wise int8 round trip
+        L.off_xq = off;
+        off = up(off + sizeof(float) * (size_t)N * H * W * Cin, kAlign);
+    }
     L.off_vq = off;
     off = up(off + (size_t)L.T_pad * L.n2 * Cin, kAlign);
     L.off_sv = off;
@@ -166,7 +171,7 @@ cudaError_t launch_error_merge(int* dst, const int* src, cudaStream_t st) {
     return cudaGetLastError();
 }
 
-constexpr int kMaxLaunches = 4;
+constexpr int kMaxLaunches = 5;
 
 // Records profiling event `slot` of the current call (no-op unless profiling).
 void prof_mark(wino_plan_s* p, int slot, cudaStream_t st) {
@@ -197,6 +202,16 @@ int run_conv(wino_plan_s* p, const void* x, int x_dtype, int N, int H, int W, in
     const float* sU = reinterpret_cast<const float*>(static_cast<const unsigned char*>(wt) +
                                                      up((size_t)L.n2 * Cout * Cin, kAlign));
 
+    int slot = 0;
+    bool x_bf16 = x_dtype == WINO_BF16;
+    if (L.xq) {
+        float* xq = reinterpret_cast<float*>(base + L.off_xq);
+        prof_mark(p, slot++, st);
+        cudaError_t e = launch_input_quant(x, x_bf16, (long)N * H * W * Cin, p->G, xq, num_sms(), st);
+        if (e != cudaSuccess) return cuda_status(p, e);
+        x = xq;
+        x_bf16 = false;
+    }
     InputArgs ia;
     ia.x = x;
     ia.N = N;
@@ -213,9 +228,8 @@ int run_conv(wino_plan_s* p, const void* x, int x_dtype, int N, int H, int W, in
     ia.sV = sV;
     ia.amax = amax;
     ia.err = err;
-    int slot = 0;
     prof_mark(p, slot++, st);
-    cudaError_t e = launch_input_transform(ia, p->tf, p->mat.m, p->bt_masked, x_dtype == WINO_BF16, st);
+    cudaError_t e = launch_input_transform(ia, p->tf, p->mat.m, p->bt_masked, x_bf16, st);
     if (e != cudaSuccess) return cuda_status(p, e);
 
     GemmArgs ga;
@@ -312,10 +326,12 @@ int wino_plan(wino_plan_t* out, int m, const double* points, const float* S_B, c
     std::memset(&p->opts, 0, sizeof(p->opts));
     if (opts) p->opts = *opts;
     if (p->opts.y_path < 0 || p->opts.y_path > 2 || p->opts.gemm < 0 || p->opts.gemm > 2 || p->opts.y_groups < 0 ||
-        p->opts.y_groups > 1 || (p->opts.y_groups == WINO_YGROUPS_TAP && p->opts.y_path == WINO_YPATH_RECOMPUTE)) {
+        p->opts.y_groups > 1 || (p->opts.y_groups == WINO_YGROUPS_TAP && p->opts.y_path == WINO_YPATH_RECOMPUTE) ||
+        (p->opts.x_int8 != 0 && p->opts.x_int8 != 1) || (p->opts.int8_transforms != 0 && p->opts.int8_transforms != 1)) {
         delete p;
         return WINO_ERR_INVALID_ARG;
     }
+    if (p->opts.int8_transforms) quantize_transforms_int8(&p->mat);
     const int n = p->mat.n;
     std::memset(&p->tf, 0, sizeof(p->tf));
     std::memcpy(p->tf.BT, p->mat.BT, sizeof(float) * n * n);
@@ -547,7 +563,7 @@ int wino_resolved_config(wino_plan_t p, int N, int H, int W, int Cin, int Cout, 
 int wino_launches_per_call(wino_plan_t p, int N, int H, int W, int Cin, int Cout) {
     if (check_shape(p, N, H, W, Cin, Cout)) return 0;
     const Layout L = make_layout(p, N, H, W, Cin, Cout);
-    return L.y_path == WINO_YPATH_RECOMPUTE ? 4 : 3;
+    return (L.y_path == WINO_YPATH_RECOMPUTE ? 4 : 3) + (L.xq ? 1 : 0);
 }
 
 int wino_profile_begin(wino_plan_t p, int max_calls) {

@@ -61,6 +61,11 @@ struct InputArgs {
 cudaError_t launch_input_transform(const InputArgs& a, const TransformArgs& tf, int m, bool masked, bool bf16_in,
                                    cudaStream_t st);
 
+// Group-wise int8 on x itself: xq = s * Q(x) per G consecutive channels of a pixel
+// (elems = N*H*W*Cin values, x bf16 or fp32, xq fp32; both 16-byte aligned).
+cudaError_t launch_input_quant(const void* x, bool bf16_in, long elems, int G, float* xq, int num_sms,
+                               cudaStream_t st);
+
 // ------------------------------------------------------------ Hadamard GEMM
 enum GemmMode { kModeAbsmax = 0, kModeQuant = 1, kModeY32 = 2 };
 

@@ -198,4 +198,27 @@ int build_matrices(int m, const double* points, const float* S_B, const float* S
     return WINO_OK;
 }
 
+namespace {
+
+// One matrix of `len` fp32 entries through the symmetric int8 quantiser, in place.
+void quantize_matrix(float* a, int len, uint64_t* nonzero) {
+    float amax = 0.0f;
+    for (int i = 0; i < len; ++i) amax = std::fmax(amax, std::fabs(a[i]));
+    const float s = amax / 127.0f;
+    *nonzero = 0;
+    for (int i = 0; i < len; ++i) {
+        float q = 0.0f;
+        if (s != 0.0f) q = std::fmin(127.0f, std::fmax(-127.0f, std::nearbyint(a[i] / s)));
+        a[i] = s * q;
+        if (a[i] != 0.0f) *nonzero |= 1ull << i;
+    }
+}
+
+}  // namespace
+
+void quantize_transforms_int8(Matrices* M) {
+    quantize_matrix(M->BT, M->n * M->n, &M->bt_nonzero);
+    quantize_matrix(M->AT, M->m * M->n, &M->at_nonzero);
+}
+
 }  // namespace wino

@@ -21,4 +21,9 @@ struct Matrices {
 // Returns WINO_OK, WINO_ERR_INVALID_ARG or WINO_ERR_NOT_EXACT.
 int build_matrices(int m, const double* points, const float* S_B, const float* S_G, Matrices* out);
 
+// Int8 transforms with one scale per matrix: B^T and A^T each become s * q, where
+// s = max|entry| / 127 (fp32 division), q = clamp(rne(entry / s), +-127), the product
+// rounded to fp32.  The nonzero masks are recomputed from the quantised entries.
+void quantize_transforms_int8(Matrices* M);
+
 }  // namespace wino

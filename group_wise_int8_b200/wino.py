@@ -53,7 +53,8 @@ class WinoError(RuntimeError):
 
 class Opts(ctypes.Structure):
     _fields_ = [("y_path", ctypes.c_int), ("gemm", ctypes.c_int), ("debug", ctypes.c_int),
-                ("y_groups", ctypes.c_int), ("reserved", ctypes.c_int * 4)]
+                ("y_groups", ctypes.c_int), ("x_int8", ctypes.c_int), ("int8_transforms", ctypes.c_int),
+                ("reserved", ctypes.c_int * 2)]
 
 
 _lib = None
@@ -125,13 +126,14 @@ class Plan:
     """A wino_plan: transforms of F(m,3) for the given points and scales."""
 
     def __init__(self, m: int, points: Sequence[float], S_B=None, S_G=None, group: int = 32,
-                 y_path: int = YPATH_AUTO, gemm: int = GEMM_AUTO, debug: int = 0, y_groups: int = YGROUPS_TILE):
+                 y_path: int = YPATH_AUTO, gemm: int = GEMM_AUTO, debug: int = 0, y_groups: int = YGROUPS_TILE,
+                 x_int8: bool = False, int8_transforms: bool = False):
         L = load_library()
         n = m + 2
         pts = (ctypes.c_double * n)(*[float(p) for p in points])
         sb = None if S_B is None else (ctypes.c_float * n)(*[float(v) for v in S_B])
         sg = None if S_G is None else (ctypes.c_float * n)(*[float(v) for v in S_G])
-        opts = Opts(y_path, gemm, debug, y_groups)
+        opts = Opts(y_path, gemm, debug, y_groups, int(x_int8), int(int8_transforms))
         h = _vp()
         rc = L.wino_plan(ctypes.byref(h), m, pts, sb, sg, group, ctypes.byref(opts))
         if rc != OK:

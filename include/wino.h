@@ -83,7 +83,16 @@ typedef struct wino_opts {
                              wino_check_device_error reports
                              WINO_ERR_DEVICE_TIMEOUT (output undefined) */
     int y_groups;  /* WINO_YGROUPS_*: how Y is grouped for its requantisation */
-    int reserved[4];
+    int x_int8;    /* 0 or 1.  1: group-wise int8 on x itself before the input transform
+                      (alternative reading of the input side, Eqs. (14)-(16)): per pixel, G
+                      consecutive channels share s = absmax/127 and x becomes
+                      s * clamp(rne(x/s), +-127) in fp32; one extra kernel per call, and the
+                      workspace holds that fp32 copy of x */
+    int int8_transforms; /* 0 or 1.  1: B^T and A^T held as int8 with one scale per matrix
+                      (same passage): each entry becomes s * clamp(rne(M/s), +-127) in fp32,
+                      s = max|M|/127, at plan time; G stays fp64 (the weights are quantised
+                      after their transform) */
+    int reserved[2];
 } wino_opts;
 
 /* Y groups (the input of the output transform).  TILE (default, the reading the
@@ -130,8 +139,9 @@ int wino_plan(wino_plan_t* out, int m, const double* points, const float* S_B, c
               const wino_opts* opts);
 int wino_plan_destroy(wino_plan_t plan);
 
-/* Host copies of the fp32 transforms the kernels use: BT [n][n], AT [m][n],
- * and the fp64 G [n][3] of the weight transform.  Any pointer may be NULL. */
+/* Host copies of the fp32 transforms the kernels use: BT [n][n], AT [m][n]
+ * (after int8_transforms, when set), and the fp64 G [n][3] of the weight
+ * transform.  Any pointer may be NULL. */
 int wino_plan_matrices(wino_plan_t plan, float* BT_host, double* G_host, float* AT_host);
 
 /* m, n, G of a plan; any pointer may be NULL. */
@@ -163,8 +173,8 @@ size_t wino_workspace_bytes(wino_plan_t plan, int N, int H, int W, int Cin, int 
  *            Cin, Cout).
  *   y_dev    [N][H][W][Cout] in y_dtype (WINO_F32 or WINO_BF16, RNE), device.
  *   ws_dev   device workspace of ws_bytes >= wino_workspace_bytes().
- * Launches the input transform, the Hadamard GEMM (one or two passes) and the
- * output transform on stream; returns after the launches (asynchronous).
+ * Launches (with x_int8: the quantisation of x, then) the input transform, the
+ * Hadamard GEMM (one or two passes) and the output transform on stream; returns after the launches (asynchronous).
  * A bounded device wait that expires makes a later call on the same
  * workspace return WINO_ERR_DEVICE_TIMEOUT (see wino_check_device_error).
  * Errors: INVALID_ARG, UNSUPPORTED, WORKSPACE, CUDA, DEVICE_TIMEOUT.

@@ -35,6 +35,10 @@ def lib():
         L.orc_plan.restype = ctypes.c_int
         L.orc_quantize.argtypes = [_f32p, ctypes.c_int, _i8p, _f32p]
         L.orc_quantize.restype = None
+        L.orc_quantize_matrix.argtypes = [_f32p, ctypes.c_int]
+        L.orc_quantize_matrix.restype = None
+        L.orc_quantize_input.argtypes = [_f32p, ctypes.c_long, ctypes.c_int, ctypes.c_int, _f32p]
+        L.orc_quantize_input.restype = ctypes.c_int
         L.orc_weight_transform.argtypes = [ctypes.c_int, _f64p, _f32p, ctypes.c_int, ctypes.c_int,
                                            ctypes.c_int, _f32p, _i8p, _f32p]
         L.orc_input_transform.argtypes = [ctypes.c_int, _f32p, _f32p, ctypes.c_int, ctypes.c_int,
@@ -73,9 +77,10 @@ def set_threads(t: int) -> int:
 
 
 class Plan:
-    """Transform matrices of F(m,3) (see orc_plan)."""
+    """Transform matrices of F(m,3) (see orc_plan).  int8_transforms: the alternative reading
+    in which the fp32 B^T and A^T are each held as int8 with one scale (orc_quantize_matrix)."""
 
-    def __init__(self, m: int, points: Sequence[float], S_B=None, S_G=None):
+    def __init__(self, m: int, points: Sequence[float], S_B=None, S_G=None, int8_transforms: bool = False):
         n = m + 2
         self.m, self.n = m, n
         pts = np.ascontiguousarray(np.array(points, dtype=np.float64))
@@ -92,6 +97,9 @@ class Plan:
                             _p(self.AT_f, _f32p))
         if rc != 0:
             raise ValueError("orc_plan failed: %d" % rc)
+        if int8_transforms:
+            lib().orc_quantize_matrix(_p(self.BT_f, _f32p), n * n)
+            lib().orc_quantize_matrix(_p(self.AT_f, _f32p), m * n)
 
 
 def quantize(v: np.ndarray):
@@ -100,6 +108,16 @@ def quantize(v: np.ndarray):
     s = np.zeros(1, np.float32)
     lib().orc_quantize(_p(v, _f32p), v.size, _p(q, _i8p), _p(s, _f32p))
     return q, float(s[0])
+
+
+def quantize_input(x: np.ndarray, G: int) -> np.ndarray:
+    """x [..., C] with each pixel's G consecutive channels through Q, returned as s * q (fp32)."""
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    C = x.shape[-1]
+    xq = np.zeros_like(x)
+    rc = lib().orc_quantize_input(_p(x, _f32p), x.size // C, C, G, _p(xq, _f32p))
+    assert rc == 0
+    return xq
 
 
 def weight_transform(plan: Plan, w: np.ndarray, G: int, want_float: bool = False):
@@ -198,11 +216,13 @@ def conv_wino_f32(plan: Plan, x: np.ndarray, w: np.ndarray) -> np.ndarray:
 
 
 def run_pipeline(plan: Plan, x: np.ndarray, w: np.ndarray, G: int, want_acc: bool = False,
-                 per_tap: bool = False) -> Dict[str, np.ndarray]:
+                 per_tap: bool = False, x_int8: bool = False) -> Dict[str, np.ndarray]:
     """The full quantised pipeline, every stage kept for comparison (per_tap: the Y_TAP
-    reading of the Y groups)."""
+    reading of the Y groups; x_int8: x itself group-quantised before the input transform)."""
     N, H, W, _ = x.shape
     n2 = plan.n * plan.n
+    if x_int8:
+        x = quantize_input(x, G)
     Uq, sU, _ = weight_transform(plan, w, G)
     Vq, sV, _ = input_transform(plan, x, G)
     Y, acc = hadamard(n2, Vq, sV, Uq, sU, G, want_acc=want_acc)

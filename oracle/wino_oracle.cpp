@@ -27,6 +27,11 @@
 //    single or per-row scale cannot absorb, "Core claim" / Fig. 3).
 //  * Fixed fp32 evaluation order (fmaf chains, ascending index, from +0) so that
 //    every int8 code is a well-defined function of the inputs.
+//  * Alternative readings, selectable (the scales "sqB sqB sqx" of Eqs. (14)-(16),
+//    review "Referee Report", minor comment): x through Q per pixel and G
+//    consecutive channels (orc_quantize_input); B^T and A^T through Q as one
+//    group each (orc_quantize_matrix).  Both leave dequantised fp32 values that
+//    the unchanged stages consume.
 //
 // Parity status: pinned by the CPU tests (exact Winograd identity with
 // quantisation off, scale invariance, textbook F(4,3) special case, quantiser
@@ -301,6 +306,38 @@ int orc_plan(int m, const double* points, const float* S_B, const float* S_G, do
 
 // Q on one contiguous group of len values.
 void orc_quantize(const float* v, int len, signed char* q, float* s) { quantize_group(v, 1, len, q, 1, s); }
+
+// Alternative reading of the transforms (Eqs. (14)-(16): the input transform
+// carries two scales of B): the matrix of len entries as ONE group of Q, each
+// entry replaced, in place, by s * q in fp32.
+void orc_quantize_matrix(float* a, int len) {
+    std::vector<signed char> q(len);
+    float s = 0.0f;
+    quantize_group(a, 1, len, q.data(), 1, &s);
+    for (int i = 0; i < len; ++i) a[i] = s * (float)q[i];
+}
+
+// Alternative reading of the input side (same passage: a scale of x): x
+// [P][C] (P pixels, NHWC order) through Q per pixel and G consecutive channels,
+// each value replaced by s * q in fp32 (xq may alias nothing).
+int orc_quantize_input(const float* x, long P, int C, int G, float* xq) {
+    if (G <= 0 || C % G != 0) return -1;
+    const int ng = C / G;
+    set_omp();
+#pragma omp parallel
+    {
+        std::vector<signed char> q(G);
+#pragma omp for schedule(static)
+        for (long p = 0; p < P; ++p)
+            for (int j = 0; j < ng; ++j) {
+                const float* v = &x[(size_t)p * C + (size_t)j * G];
+                float s = 0.0f;
+                quantize_group(v, 1, G, q.data(), 1, &s);
+                for (int i = 0; i < G; ++i) xq[(size_t)p * C + (size_t)j * G + i] = s * (float)q[i];
+            }
+    }
+    return 0;
+}
 
 // Stage 1: weight transform U = G g G^T per (cout, cin) in fp64 (fma chains,
 // ascending index, from +0), U_f = (float)U; then Q over G consecutive input

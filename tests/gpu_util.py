@@ -27,10 +27,11 @@ def weight_dumps(plan, wt: torch.Tensor, Cin: int, Cout: int):
 
 
 def run_gpu(m, pts, sb, sg, G, x_f32, x_bits, w, out_dtype=torch.float32, y_path=wino.YPATH_AUTO,
-            gemm=wino.GEMM_AUTO, debug=0, y_groups=wino.YGROUPS_TILE):
+            gemm=wino.GEMM_AUTO, debug=0, y_groups=wino.YGROUPS_TILE, x_int8=False, int8_transforms=False):
     N, H, W, Cin = x_f32.shape
     Cout = w.shape[0]
-    plan = wino.Plan(m, pts, sb, sg, G, y_path=y_path, gemm=gemm, debug=debug, y_groups=y_groups)
+    plan = wino.Plan(m, pts, sb, sg, G, y_path=y_path, gemm=gemm, debug=debug, y_groups=y_groups,
+                     x_int8=x_int8, int8_transforms=int8_transforms)
     x = to_device_input(x_f32, x_bits)
     wt = plan.transform_weights(torch.from_numpy(w).cuda())
     ws = torch.empty(plan.workspace_bytes(N, H, W, Cin, Cout), dtype=torch.uint8, device="cuda")
@@ -54,8 +55,9 @@ def run_gpu(m, pts, sb, sg, G, x_f32, x_bits, w, out_dtype=torch.float32, y_path
     return res
 
 
-def run_oracle(m, pts, sb, sg, G, x_f32, w, want_acc=False, per_tap=False):
-    res = oracle.run_pipeline(oracle.Plan(m, pts, sb, sg), x_f32, w, G, want_acc=want_acc, per_tap=per_tap)
+def run_oracle(m, pts, sb, sg, G, x_f32, w, want_acc=False, per_tap=False, x_int8=False, int8_transforms=False):
+    res = oracle.run_pipeline(oracle.Plan(m, pts, sb, sg, int8_transforms=int8_transforms), x_f32, w, G,
+                              want_acc=want_acc, per_tap=per_tap, x_int8=x_int8)
     res["ref"] = oracle.conv_direct_f64(x_f32, w)
     return res
 

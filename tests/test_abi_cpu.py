@@ -75,6 +75,34 @@ def test_plan_f23_matches_oracle(lib, pts):
     assert np.array_equal(BT, op.BT_f) and np.array_equal(G, op.G_d) and np.array_equal(AT, op.AT_f)
 
 
+@pytest.mark.parametrize("m,pts,scaled", [(2, synth.POINTS_F2, False), (4, synth.POINTS_F4, True),
+                                          (6, synth.POINTS_F6, False), (6, synth.POINTS_F6, True)])
+def test_plan_int8_transforms_match_oracle(lib, m, pts, scaled):
+    """The int8-transform reading is applied at plan time on the host: the library's B^T
+    and A^T equal the oracle's quantised matrices bit for bit, G is untouched."""
+    n = m + 2
+    r = np.random.default_rng(m)
+    sb = (r.integers(32, 129, n) / 64.0).astype(np.float32) if scaled else None
+    sg = (r.integers(32, 129, n) / 64.0).astype(np.float32) if scaled else None
+    op = oracle.Plan(m, pts, sb, sg, int8_transforms=True)
+    BT, G, AT = wino.Plan(m, pts, sb, sg, 32, int8_transforms=True).matrices()
+    assert np.array_equal(BT, op.BT_f) and np.array_equal(G, op.G_d) and np.array_equal(AT, op.AT_f)
+    BT0, _, AT0 = wino.Plan(m, pts, sb, sg, 32).matrices()
+    assert not np.array_equal(BT0, BT)
+
+
+def test_x_int8_option_adds_a_launch_and_workspace(lib):
+    shape = (2, 20, 20, 64, 64)
+    p0 = wino.Plan(6, synth.POINTS_F6, None, None, 32)
+    p1 = wino.Plan(6, synth.POINTS_F6, None, None, 32, x_int8=True)
+    assert p1.launches_per_call(*shape) == p0.launches_per_call(*shape) + 1
+    assert p1.workspace_bytes(*shape) >= p0.workspace_bytes(*shape) + 4 * 2 * 20 * 20 * 64
+    for bad in (dict(x_int8=2), dict(int8_transforms=-1)):
+        with pytest.raises(wino.WinoError) as e:
+            wino.Plan(6, synth.POINTS_F6, None, None, 32, **bad)
+        assert e.value.status == wino.ERR_INVALID_ARG
+
+
 @pytest.mark.parametrize("bad", [
     dict(m=5), dict(group=48), dict(points=(0.0, 1.0, 1.0, 2.0, -2.0, math.inf)),
     dict(points=(0.0, 1.0, -1.0, math.inf, -2.0, math.inf)), dict(points=(0.0, 1.0, -1.0, 2.0, float("nan"), math.inf)),

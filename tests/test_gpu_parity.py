@@ -102,6 +102,33 @@ def test_y_tap_reading_bit_exact(cuda_dev, name, gemm):
     assert abs(oracle.sqnr_db(ref["ref"], got["out"]) - oracle.sqnr_db(ref["ref"], ref["out"])) <= 0.01
 
 
+_oracle_alt_cache = {}
+_ALT = {"x_int8": dict(x_int8=True), "int8_transforms": dict(int8_transforms=True),
+        "both": dict(x_int8=True, int8_transforms=True)}
+
+
+@pytest.mark.parametrize("y_path", [wino.YPATH_RECOMPUTE, wino.YPATH_Y32])
+@pytest.mark.parametrize("reading", list(_ALT))
+@pytest.mark.parametrize("name", ["tiny_f4", "ragged_f6_cout96", "f4_g64_outliers", "f6_g256", "f2_ragged",
+                                  "f6_one_pixel"])
+def test_alternative_input_readings_bit_exact(cuda_dev, name, reading, y_path):
+    """x group-quantised per pixel before the transform (x_int8) and/or int8 B^T and A^T with
+    one scale per matrix (int8_transforms): every code and scale bit for bit, the output
+    within the fp32 tolerance, on both Y paths."""
+    m, pts, G, x_f32, x_bits, w, sb, sg = make_case(name)
+    key = (name, reading)
+    if key not in _oracle_alt_cache:
+        _oracle_alt_cache[key] = run_oracle(m, pts, sb, sg, G, x_f32, w, **_ALT[reading])
+    ref = _oracle_alt_cache[key]
+    got = run_gpu(m, pts, sb, sg, G, x_f32, x_bits, w, out_dtype=torch.float32, y_path=y_path,
+                  debug=wino.DEBUG_YQ, **_ALT[reading])
+    keys = ("Uq", "sU", "Vq", "sV", "Yq", "sY") + (("Y",) if y_path == wino.YPATH_Y32 else ())
+    for k in keys:
+        assert_bits_equal(k, got[k], ref[k])
+    assert rel_l2(got["out"], ref["out"]) <= 1e-5
+    assert abs(oracle.sqnr_db(ref["ref"], got["out"]) - oracle.sqnr_db(ref["ref"], ref["out"])) <= 0.01
+
+
 def test_y_tap_rejects_recompute_path(cuda_dev):
     with pytest.raises(wino.WinoError):
         wino.Plan(6, P6, None, None, 32, y_path=wino.YPATH_RECOMPUTE, y_groups=wino.YGROUPS_TAP)

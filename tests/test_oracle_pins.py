@@ -364,3 +364,119 @@ def test_standard_scales_collapse_and_row_norm_scales_recover(m, pts):
     assert s_std < 0.0
     assert s_bal > 10.0
     assert s_bal > s_std + 20.0
+
+
+# ------------------------------------------- alternative input-side readings
+# Eqs. (14)-(16) give the quantised input transform the scales "sqB sqB sqx": an
+# int8 B^T (one scale per matrix, applied on both sides) and an int8 x.  The
+# library offers both as plan options (x_int8, int8_transforms); these pins fix
+# the oracle's side of them.
+
+def _exact_code(v, amax):
+    """rne(127 v / amax) in exact rationals, clamped to +-127, and whether it sits within
+    1e-4 of a tie (where the fp32 division may decide either way)."""
+    t = Fraction(float(v)) * 127 / Fraction(float(amax))
+    frac = t - math.floor(t)
+    return max(-127, min(127, round(t))), abs(frac - Fraction(1, 2)) < Fraction(1, 10 ** 4)
+
+
+def _check_int8_matrix(got, exact):
+    """got = s * q entrywise with s = max|exact| / 127 (fp32) and q the exact-rational
+    rne codes of exact (either neighbour at a tie)."""
+    amax = float(np.abs(exact).max())
+    s = np.float32(amax) / np.float32(127.0)
+    for v, g in zip(np.asarray(exact, np.float64).ravel(), np.asarray(got).ravel()):
+        q, tie = _exact_code(v, amax)
+        want = {np.float32(s * np.float32(c)) for c in ((q - 1, q, q + 1) if tie else (q,))}
+        assert np.float32(g) in want, (v, g, q, want)
+
+
+def test_int8_transforms_lavin_gray_codes():
+    """Int8 transforms on the Lavin-Gray F(4,3) matrices: B^T's largest entry is 5, so its
+    codes are rne(127 v / 5) (4 -> 102, 1 -> 25, 2 -> 51, -5 -> -127); A^T's is 8 (1 -> 16,
+    2 -> 32, 8 -> 127; 4 lands on the tie 63.5, decided by the fp32 division)."""
+    sb = np.array([4, -6, -6, 24, 24, 1], np.float32)
+    sg = np.array([1 / 4, -1 / 6, -1 / 6, 1 / 24, 1 / 24, 1], np.float32)
+    BT = np.array([[4, 0, -5, 0, 1, 0], [0, -4, -4, 1, 1, 0], [0, 4, -4, -1, 1, 0],
+                   [0, -2, -1, 2, 1, 0], [0, 2, -1, -2, 1, 0], [0, 4, 0, -5, 0, 1]], np.float64)
+    AT = np.array([[1, 1, 1, 1, 1, 0], [0, 1, -1, 2, -2, 0], [0, 1, 1, 4, 4, 0],
+                   [0, 1, -1, 8, -8, 1]], np.float64)
+    p = oracle.Plan(4, P4, sb, sg, int8_transforms=True)
+    exact = oracle.Plan(4, P4, sb, sg)
+    assert _exact_code(4, 5) == (102, False) and _exact_code(4, 8) == (64, True)
+    _check_int8_matrix(p.BT_f, BT)
+    _check_int8_matrix(p.AT_f, exact.AT_d)        # A^T = AT up to the fp32 scales S_A
+    assert np.array_equal(p.G_d, exact.G_d) and np.array_equal(p.BT_d, exact.BT_d)
+    s = np.float32(5.0) / np.float32(127.0)
+    assert p.BT_f[0, 0] == np.float32(s * np.float32(102)) and p.BT_f[0, 2] == -np.float32(s * np.float32(127))
+
+
+@pytest.mark.parametrize("m,pts", [(4, P4), (6, P6)])
+def test_int8_transforms_error_bound_and_zeros(m, pts):
+    """Every entry moves by at most half a step of its matrix's scale, zeros stay zero, the
+    largest entry maps to +-127 steps, and no entry exceeds 127 steps."""
+    n = m + 2
+    sb, sg = dyadic_scales(31, n), dyadic_scales(32, n)
+    p = oracle.Plan(m, pts, sb, sg, int8_transforms=True)
+    exact = oracle.Plan(m, pts, sb, sg)
+    for got, ref in ((p.BT_f, exact.BT_f), (p.AT_f, exact.AT_f)):
+        s = float(np.float32(np.abs(ref).max()) / np.float32(127.0))
+        err = np.abs(got.astype(np.float64) - ref.astype(np.float64))
+        assert np.all(err <= 0.5 * s * (1 + 1e-5))
+        assert np.all(got[ref == 0] == 0)
+        codes = got.astype(np.float64) / s
+        assert np.allclose(codes, np.round(codes), rtol=0, atol=1e-4) and np.abs(codes).max() <= 127 + 1e-4
+        assert abs(abs(codes.ravel()[np.argmax(np.abs(ref))]) - 127) < 1e-4
+
+
+def test_int8_transforms_change_nothing_on_the_int8_grid():
+    """The textbook F(2,3) matrices hold only 0 and +-1, so each becomes 127 steps of 1/127:
+    in fp32 (1/127) * 127 rounds back to 1, the plan is unchanged and so is every stage."""
+    sb = np.array([1, 2, 2, -1], np.float32)
+    sg = np.array([1, 0.5, 0.5, 1], np.float32)
+    p0, p1 = oracle.Plan(2, P2, sb, sg), oracle.Plan(2, P2, sb, sg, int8_transforms=True)
+    assert np.array_equal(p0.BT_f, p1.BT_f) and np.array_equal(p0.AT_f, p1.AT_f)
+    x, w = rand_case(81, N=1, H=9, W=10, Cin=32, Cout=32)
+    a, b = oracle.run_pipeline(p0, x, w, 32), oracle.run_pipeline(p1, x, w, 32)
+    for k in ("Vq", "sV", "Yq", "sY", "out"):
+        assert np.array_equal(a[k], b[k])
+
+
+def test_x_int8_codes_per_pixel_group_brute_force():
+    """x through Q per pixel and G consecutive channels: s = absmax / 127 of that group
+    only (fp32 division) and codes rne(127 x / absmax) in exact rationals (either neighbour
+    at a tie); an outlier in one group leaves every other group untouched."""
+    r = np.random.default_rng(9)
+    G = 16
+    x = (r.standard_normal((2, 3, 2, 48)) * np.exp(r.standard_normal((2, 3, 2, 3)).repeat(G, axis=-1)))
+    x = x.astype(np.float32)
+    x[1, 2, 0, G:2 * G] = 0.0                                   # an all-zero group
+    xq = oracle.quantize_input(x, G)
+    assert not xq[1, 2, 0, G:2 * G].any()
+    for idx in np.ndindex(*x.shape[:3]):
+        for j in range(3):
+            grp, got = x[idx][j * G:(j + 1) * G], xq[idx][j * G:(j + 1) * G]
+            if not grp.any():
+                continue
+            _check_int8_matrix(got, grp.astype(np.float64))
+    y = x.copy()
+    y[0, 1, 1, 5] = 1e4                                          # outlier in group 0 of one pixel
+    yq = oracle.quantize_input(y, G)
+    changed = np.argwhere(np.any((yq != xq).reshape(2, 3, 2, 3, G), axis=-1))
+    assert changed.tolist() == [[0, 1, 1, 0]]
+
+
+def test_x_int8_changes_nothing_on_the_int8_grid():
+    """Values k / 8 with integer |k| <= 127 and a +-127 in every group are their own codes
+    (s = 1/8 exactly): the quantised input equals x and the whole pipeline is unchanged."""
+    r = np.random.default_rng(10)
+    N, H, W, C, G = 1, 11, 9, 64, 32
+    k = r.integers(-127, 128, (N, H, W, C))
+    k[..., 0], k[..., G] = 127, -127
+    x = (k / 8.0).astype(np.float32)
+    assert np.array_equal(oracle.quantize_input(x, G), x)
+    w = (r.standard_normal((32, 3, 3, C)) / 24).astype(np.float32)
+    p = oracle.Plan(4, P4, dyadic_scales(3, 6), dyadic_scales(4, 6))
+    a, b = oracle.run_pipeline(p, x, w, G), oracle.run_pipeline(p, x, w, G, x_int8=True)
+    for key in ("Vq", "sV", "Yq", "sY", "out"):
+        assert np.array_equal(a[key], b[key])
