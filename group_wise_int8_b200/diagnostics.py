@@ -62,13 +62,15 @@ def reference_conv_f64(x: torch.Tensor, w: np.ndarray) -> np.ndarray:
 
 
 def diagnose(m: int, points: Sequence[float], S_B, S_G, G: int, x: torch.Tensor, w: np.ndarray,
-             y_groups: int = wino.YGROUPS_TILE, gemm: int = wino.GEMM_AUTO) -> Dict[str, object]:
-    """x: device NHWC (bf16 or fp32), w: host [Cout][3][3][Cin] fp32."""
+             y_groups: int = wino.YGROUPS_TILE, gemm: int = wino.GEMM_AUTO, x_int8: bool = False,
+             int8_transforms: bool = False) -> Dict[str, object]:
+    """x: device NHWC (bf16 or fp32), w: host [Cout][3][3][Cin] fp32.  x_int8 / int8_transforms:
+    the alternative readings of the input side (int8 x per pixel group, int8 B^T and A^T)."""
     N, H, W, Cin = x.shape
     Cout = w.shape[0]
     n = m + 2
     plan = wino.Plan(m, points, S_B, S_G, G, y_path=wino.YPATH_Y32, gemm=gemm, debug=wino.DEBUG_YQ,
-                     y_groups=y_groups)
+                     y_groups=y_groups, x_int8=x_int8, int8_transforms=int8_transforms)
     wt = plan.transform_weights(torch.from_numpy(np.ascontiguousarray(w, np.float32)).to(x.device))
     ws = torch.empty(plan.workspace_bytes(N, H, W, Cin, Cout), dtype=torch.uint8, device=x.device)
     out = plan.conv2d(x, wt, Cout, out_dtype=torch.float32, workspace=ws)
@@ -124,6 +126,11 @@ def main(argv: Optional[Sequence[str]] = None):
             if yg == wino.YGROUPS_TILE:
                 for row in d["rel_std_Y"]:
                     print("      " + " ".join("%6.2f" % v for v in row))
+    sb, sg = presets["rownorm"]
+    for xi, it in ((True, False), (False, True), (True, True)):
+        d = diagnose(layer.m, layer.points, sb, sg, layer.group, x, w, x_int8=xi, int8_transforms=it)
+        print("tile groups     rownorm       SQNR %7.2f dB   x_int8=%d int8_transforms=%d"
+              % (d["sqnr_db"], xi, it))
 
 
 if __name__ == "__main__":
