@@ -48,8 +48,8 @@ UNIT = "TFLOP/s"
 # current kernel exists.
 NCU_TRAFFIC = {
     # (workload, layer, kernel) -> dram read+write bytes per launch from one ncu capture of the
-    # CURRENT kernel (profiles/resnet18_f63_g32_launches_and_full.md); entries are removed
-    # whenever that kernel changes.
+    # CURRENT kernel (summarised under profiles/); entries are removed whenever that kernel changes.
+    ("resnet18", 0, "input_transform"): 14695168,
     ("resnet18", 0, "hadamard_absmax"): 15109120,
     ("resnet18", 0, "hadamard_quant"): 19476480,
     ("resnet18", 0, "output_transform"): 13168640,
