@@ -42,7 +42,7 @@ struct Layout {
     int TH = 0, TW = 0, n2 = 0, ng = 0, ngo = 0;
     long T = 0, T_pad = 0;
     int y_path = 0, gemm = 0;
-    bool dbg_yq = false, dbg_acc = false, ytap = false, xq = false;
+    bool dbg_yq = false, dbg_acc = false, ytap = false, xq = false, swap = false;
     size_t off_xq = 0, off_vq = 0, off_sv = 0, off_amax = 0, off_yq = 0, off_y32 = 0, off_sy = 0, off_acc = 0, off_err = 0;
     size_t total = 0;
 };
@@ -93,8 +93,13 @@ Layout make_layout(const wino_plan_s* p, int N, int H, int W, int Cin, int Cout)
     L.gemm = p->opts.gemm == WINO_GEMM_AUTO ? WINO_GEMM_TCGEN05 : p->opts.gemm;
     if (L.gemm == WINO_GEMM_TCGEN05 && tc_block_n(Cout, p->G) == 0) L.gemm = WINO_GEMM_SIMT;
     L.ytap = p->opts.y_groups == WINO_YGROUPS_TAP;
-    L.y_path = L.ytap ? WINO_YPATH_Y32
-                      : (p->opts.y_path == WINO_YPATH_AUTO ? choose_y_path(p, L.T, Cin, Cout, L.n2) : p->opts.y_path);
+    // at most 32 tiles: the fp32-Y pass runs with swapped operands (output channels on the MMA's
+    // 128 rows), unless the recompute path was asked for
+    L.swap = L.gemm == WINO_GEMM_TCGEN05 && tc_swap_ok((int)std::min<long>(L.T, 1 << 30), Cout) &&
+             p->opts.y_path != WINO_YPATH_RECOMPUTE;
+    L.y_path = (L.ytap || L.swap) ? WINO_YPATH_Y32
+                                  : (p->opts.y_path == WINO_YPATH_AUTO ? choose_y_path(p, L.T, Cin, Cout, L.n2)
+                                                                       : p->opts.y_path);
     L.dbg_yq = (p->opts.debug & WINO_DEBUG_YQ) != 0;
     L.dbg_acc = (p->opts.debug & WINO_DEBUG_ACC32) != 0;
     L.xq = p->opts.x_int8 != 0;
@@ -250,6 +255,7 @@ int run_conv(wino_plan_s* p, const void* x, int x_dtype, int N, int H, int W, in
     ga.acc = acc;
     ga.err = err;
     ga.force_timeout = (p->opts.debug & WINO_DEBUG_FORCE_TIMEOUT) != 0 && L.gemm == WINO_GEMM_TCGEN05;
+    ga.swap_ab = L.swap ? 1 : 0;
     auto gemm = [&](int mode) -> cudaError_t {
         prof_mark(p, slot++, st);
         if (L.gemm == WINO_GEMM_SIMT) return launch_hadamard_simt(ga, Vq, Uq, mode, st);

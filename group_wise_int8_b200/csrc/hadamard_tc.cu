@@ -150,7 +150,33 @@ struct Walk {
     }
 };
 
-template <int BN, int MODE, bool DUMP>
+// Publishes a block's running |Y| maxima into amax [T_pad][Cout/G] (atomicMax on the float bits).
+// Rows are tiles: one entry per chunk (its columns lie in one group).  SWAP (rows are output
+// channels, columns tiles): per column the maximum over the warp's 32 channels (one group, as
+// G >= 32 and a warp's channels start at a multiple of 32), published by lane 0.
+template <int NP, int CPT, bool SWAP>
+__device__ __forceinline__ void publish_amax(const GemmArgs& p, int row, int lane, const int (&cgrp)[NP],
+                                             const int (&colg)[NP], const float (&gmax)[NP],
+                                             const float (&gcol)[NP][CPT]) {
+#pragma unroll
+    for (int h = 0; h < NP; ++h) {
+        if (SWAP) {
+            const int grp = (row - lane) / p.G;
+#pragma unroll
+            for (int c = 0; c < CPT; ++c) {
+                float v = gcol[h][c];
+#pragma unroll
+                for (int off = 16; off > 0; off >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, off));
+                const int tt = colg[h] + c;
+                if (lane == 0 && tt < p.T) atomicMax(&p.amax[(size_t)tt * p.ngo + grp], __float_as_uint(v));
+            }
+        } else {
+            atomicMax(&p.amax[(size_t)row * p.ngo + cgrp[h]], __float_as_uint(gmax[h]));
+        }
+    }
+}
+
+template <int BN, int MODE, bool DUMP, bool SWAP>
 __global__ void __launch_bounds__(TcCfg<BN>::kThreads, 1)
     hadamard_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                        const __grid_constant__ CUtensorMap tmSV, const __grid_constant__ CUtensorMap tmSU, GemmArgs p) {
@@ -170,8 +196,9 @@ __global__ void __launch_bounds__(TcCfg<BN>::kThreads, 1)
     const uint32_t stage_bytes = a_bytes + b_bytes;
     const int S = p.stages;
     float* sv_ring = reinterpret_cast<float*>(smem + (size_t)S * stage_bytes);   // [S][TPS][GPS][128]
-    float* su_ring = sv_ring + (size_t)S * TPS * GPS * kBM;                      // [S][TPS][GPS][BN]
-    SmemTail* tail = reinterpret_cast<SmemTail*>(su_ring + (size_t)S * TPS * GPS * BN);
+    const int su_stride = (TPS * GPS * BN + 31) / 32 * 32;                         // 128-byte stage slices
+    float* su_ring = sv_ring + (size_t)S * TPS * GPS * kBM;                      // [S][su_stride]: [TPS][GPS][BN]
+    SmemTail* tail = reinterpret_cast<SmemTail*>(su_ring + (size_t)S * su_stride);
     volatile int* abort_flag = &tail->abort_flag;
     const uint32_t scale_bytes = (uint32_t)TPS * GPS * (kBM + BN) * 4;
 
@@ -232,7 +259,7 @@ __global__ void __launch_bounds__(TcCfg<BN>::kThreads, 1)
                         tma_load_3d(sa + a_bytes + (size_t)c * TPS * b_tile, &tmB, bar, k0, w.nb * BN, w.tap);
                     }
                     tma_load_3d(sv_ring + (size_t)st.idx * TPS * GPS * kBM, &tmSV, bar, w.mb * kBM, ks * GPS, w.tap);
-                    tma_load_3d(su_ring + (size_t)st.idx * TPS * GPS * BN, &tmSU, bar, w.nb * BN, ks * GPS, w.tap);
+                    tma_load_3d(su_ring + (size_t)st.idx * su_stride, &tmSU, bar, w.nb * BN, ks * GPS, w.tap);
                     ++issued;
                     st.next(S);
                 }
@@ -328,11 +355,14 @@ __global__ void __launch_bounds__(TcCfg<BN>::kThreads, 1)
         bool valid = false;
         int colg[NP], cgrp[NP];
         float gmax[NP];
+        float gcol[NP][CPT];   // SWAP: running |Y| maximum per column (tile) of this thread's cout
         QScale qy[NP];
 #pragma unroll
         for (int h = 0; h < NP; ++h) {
             colg[h] = cgrp[h] = 0;
             gmax[h] = 0.0f;
+#pragma unroll
+            for (int c = 0; c < CPT; ++c) gcol[h][c] = 0.0f;
             qy[h].s = qy[h].r = 0.0f;
             qy[h].rd = 0.0;
         }
@@ -343,19 +373,17 @@ __global__ void __launch_bounds__(TcCfg<BN>::kThreads, 1)
             const int b_id = w.mb * p.num_nb + w.nb;
             if (b_id != blk) {
                 // a new (row block, column block): publish the running |Y| maxima of the previous one
-#pragma unroll
-                for (int h = 0; h < NP; ++h) {
-                    if (MODE != kModeQuant && valid && blk >= 0)
-                        atomicMax(&p.amax[(size_t)row * p.ngo + cgrp[h]], __float_as_uint(gmax[h]));
-                }
+                if (MODE != kModeQuant && valid && blk >= 0) publish_amax<NP, CPT, SWAP>(p, row, lane, cgrp, colg, gmax, gcol);
                 blk = b_id;
                 row = w.mb * kBM + rloc;
-                valid = row < p.T;
+                valid = row < (SWAP ? p.Cout : p.T);
 #pragma unroll
                 for (int h = 0; h < NP; ++h) {
                     colg[h] = w.nb * BN + col0[h];
                     cgrp[h] = colg[h] / p.G;          // CPT <= G: a chunk's columns lie in one Y group
                     gmax[h] = 0.0f;
+#pragma unroll
+                    for (int c = 0; c < CPT; ++c) gcol[h][c] = 0.0f;
                     if (MODE == kModeQuant && valid)
                         qy[h] = make_qscale(__uint_as_float(p.amax[(size_t)row * p.ngo + cgrp[h]]));
                 }
@@ -366,7 +394,7 @@ __global__ void __launch_bounds__(TcCfg<BN>::kThreads, 1)
                     break;
                 }
                 const float* svs = sv_ring + (size_t)st.idx * TPS * GPS * kBM + rloc;
-                const float* sus = su_ring + (size_t)st.idx * TPS * GPS * BN;
+                const float* sus = su_ring + (size_t)st.idx * su_stride;
                 for (int t = 0; t < nt; ++t) {
                     const int tap = w.tap + t;
                     if (!warp_wait(&tail->acc_full[sl.idx], sl.phase, abort_flag, p.err)) {
@@ -413,8 +441,14 @@ __global__ void __launch_bounds__(TcCfg<BN>::kThreads, 1)
                             if (DUMP && valid) {
                                 const int jg = ks * GPS + j;
 #pragma unroll
-                                for (int c = 0; c < CPT; ++c)
-                                    p.acc[(((size_t)tap * p.T + row) * p.Cout + colg[h] + c) * p.ng + jg] = (int)r[h][c];
+                                for (int c = 0; c < CPT; ++c) {
+                                    if (SWAP) {   // row = output channel, column = tile
+                                        if (colg[h] + c < p.T)
+                                            p.acc[(((size_t)tap * p.T + colg[h] + c) * p.Cout + row) * p.ng + jg] = (int)r[h][c];
+                                    } else {
+                                        p.acc[(((size_t)tap * p.T + row) * p.Cout + colg[h] + c) * p.ng + jg] = (int)r[h][c];
+                                    }
+                                }
                             }
                         }
                     }
@@ -440,6 +474,15 @@ __global__ void __launch_bounds__(TcCfg<BN>::kThreads, 1)
                                             make_uint4(q[4 * c], q[4 * c + 1], q[4 * c + 2], q[4 * c + 3]);
                                 }
                             }
+                        } else if (SWAP) {
+                            // one output channel, CPT tiles: lanes hold consecutive channels, so each
+                            // store instruction writes 32 consecutive floats of one tile and tap
+#pragma unroll
+                            for (int c = 0; c < CPT; ++c) {
+                                const int tt = colg[h] + c;
+                                gcol[h][c] = fmaxf(gcol[h][c], fabsf(y[c]));
+                                if (tt < p.T) p.Y32[((size_t)tap * p.T + tt) * p.Cout + row] = y[c];
+                            }
                         } else {
 #pragma unroll
                             for (int c = 0; c < CPT; c += 2) gmax[h] = max_abs3(gmax[h], y[c], y[c + 1]);
@@ -459,10 +502,7 @@ __global__ void __launch_bounds__(TcCfg<BN>::kThreads, 1)
             }
             w.advance(nt, p);
         }
-#pragma unroll
-        for (int h = 0; h < NP; ++h)
-            if (ok && MODE != kModeQuant && valid && blk >= 0)
-                atomicMax(&p.amax[(size_t)row * p.ngo + cgrp[h]], __float_as_uint(gmax[h]));
+        if (ok && MODE != kModeQuant && valid && blk >= 0) publish_amax<NP, CPT, SWAP>(p, row, lane, cgrp, colg, gmax, gcol);
     }
 
     tc_fence_before();
@@ -500,20 +540,30 @@ struct Maps {
 };
 
 size_t smem_bytes(const GemmArgs& a, int BN) {
-    const size_t per_stage = (size_t)a.tps * a.SK * (kBM + BN) + (size_t)a.tps * (a.SK / a.G) * (kBM + BN) * 4;
+    const size_t gps = (size_t)(a.SK / a.G);
+    const size_t per_stage = (size_t)a.tps * a.SK * (kBM + BN) + (size_t)a.tps * gps * kBM * 4 +
+                             ((size_t)a.tps * gps * BN + 31) / 32 * 32 * 4;
     return 1024 + (size_t)a.stages * per_stage + sizeof(SmemTail);
 }
 
-template <int BN, int MODE, bool DUMP>
+template <int BN, int MODE, bool DUMP, bool SWAP = false>
 cudaError_t launch_cfg(const GemmArgs& a, const Maps& m, int num_sms, cudaStream_t st) {
     using Cfg = TcCfg<BN>;
     // at least half the SM's shared memory, so one CTA owns the SM and its TMEM
     const size_t smem = std::max<size_t>(smem_bytes(a, BN), 116 * 1024);
-    auto kern = hadamard_tc_kernel<BN, MODE, DUMP>;
+    auto kern = hadamard_tc_kernel<BN, MODE, DUMP, SWAP>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     const int grid = a.num_units < num_sms ? a.num_units : num_sms;   // every CTA gets at least one tap-unit
     return launch_dependent(kern, dim3(grid), dim3(Cfg::kThreads), smem, st, m.a, m.b, m.sv, m.su, a);
+}
+
+// Swapped operands: the fp32-Y pass only.
+template <int BN>
+cudaError_t launch_swap(const GemmArgs& a, const Maps& m, int mode, int num_sms, cudaStream_t st) {
+    if (mode != kModeY32) return cudaErrorInvalidValue;
+    return a.acc ? launch_cfg<BN, kModeY32, true, true>(a, m, num_sms, st)
+                 : launch_cfg<BN, kModeY32, false, true>(a, m, num_sms, st);
 }
 
 template <int BN>
@@ -581,47 +631,62 @@ static void choose_stage(GemmArgs& a, int BN) {
     a.stages = stages > kMaxStages ? kMaxStages : (stages < 2 ? 2 : stages);
 }
 
+bool tc_swap_ok(int T, int Cout) { return T <= 32 && Cout % kBM == 0; }
+
 cudaError_t launch_hadamard_tc(GemmArgs a, const int8_t* Vq, const int8_t* Uq, int mode, int num_sms,
                                cudaStream_t st, int* launches) {
-    const int BN = tc_block_n(a.Cout, a.G);
+    const bool swap = a.swap_ab != 0;
+    if (swap && (!tc_swap_ok(a.T, a.Cout) || mode != kModeY32)) return cudaErrorInvalidValue;
+    // swapped: 128 output channels per row block, the tiles (at most 32) as the MMA's N
+    const int BN = swap ? (a.T <= 16 ? 16 : 32) : tc_block_n(a.Cout, a.G);
     if (BN == 0) return cudaErrorInvalidValue;
     EncodeTiledFn enc = get_encode_fn();
     if (!enc) return cudaErrorNotSupported;
-    a.num_mb = (a.T + kBM - 1) / kBM;
-    a.num_nb = a.Cout / BN;
+    a.num_mb = swap ? a.Cout / kBM : (a.T + kBM - 1) / kBM;
+    a.num_nb = swap ? (a.T + BN - 1) / BN : a.Cout / BN;
     choose_stage(a, BN);
     a.num_units = a.num_mb * a.num_nb * a.n2;   // tap-units, split evenly over the CTAs
 
     Maps m;
     const CUtensorMapSwizzle sw = swizzle_for(a.BK);
     const int gps = a.SK / a.G;
-    {   // Vq [n2][T_pad][Cin] int8, box BK x 128 x TPS
-        const cuuint64_t dims[3] = {(cuuint64_t)a.Cin, (cuuint64_t)a.T_pad, (cuuint64_t)a.n2};
-        const cuuint64_t strides[2] = {(cuuint64_t)a.Cin, (cuuint64_t)a.T_pad * a.Cin};
+    // operand A: 128 rows (tiles of Vq, or output channels of Uq when swapped) per row block;
+    // operand B: BN rows (output channels of Uq, or tiles of Vq when swapped); the row scales
+    // (128 per K-group) and column scales (BN per K-group) follow their operands
+    const int8_t* a_src = swap ? Uq : Vq;
+    const int8_t* b_src = swap ? Vq : Uq;
+    const float* ra_src = swap ? a.sU : a.sV;
+    const float* cb_src = swap ? a.sV : a.sU;
+    const cuuint64_t rows_v = (cuuint64_t)a.T_pad, rows_u = (cuuint64_t)a.Cout;
+    const cuuint64_t a_rows = swap ? rows_u : rows_v, b_rows = swap ? rows_v : rows_u;
+    {   // A [n2][a_rows][Cin] int8, box BK x 128 x TPS
+        const cuuint64_t dims[3] = {(cuuint64_t)a.Cin, a_rows, (cuuint64_t)a.n2};
+        const cuuint64_t strides[2] = {(cuuint64_t)a.Cin, a_rows * a.Cin};
         const cuuint32_t box[3] = {(cuuint32_t)a.BK, (cuuint32_t)kBM, (cuuint32_t)a.tps};
-        if (!encode(enc, &m.a, CU_TENSOR_MAP_DATA_TYPE_UINT8, Vq, dims, strides, box, sw)) return cudaErrorInvalidValue;
+        if (!encode(enc, &m.a, CU_TENSOR_MAP_DATA_TYPE_UINT8, a_src, dims, strides, box, sw)) return cudaErrorInvalidValue;
     }
-    {   // Uq [n2][Cout][Cin] int8, box BK x BN x TPS
-        const cuuint64_t dims[3] = {(cuuint64_t)a.Cin, (cuuint64_t)a.Cout, (cuuint64_t)a.n2};
-        const cuuint64_t strides[2] = {(cuuint64_t)a.Cin, (cuuint64_t)a.Cout * a.Cin};
+    {   // B [n2][b_rows][Cin] int8, box BK x BN x TPS
+        const cuuint64_t dims[3] = {(cuuint64_t)a.Cin, b_rows, (cuuint64_t)a.n2};
+        const cuuint64_t strides[2] = {(cuuint64_t)a.Cin, b_rows * a.Cin};
         const cuuint32_t box[3] = {(cuuint32_t)a.BK, (cuuint32_t)BN, (cuuint32_t)a.tps};
-        if (!encode(enc, &m.b, CU_TENSOR_MAP_DATA_TYPE_UINT8, Uq, dims, strides, box, sw)) return cudaErrorInvalidValue;
+        if (!encode(enc, &m.b, CU_TENSOR_MAP_DATA_TYPE_UINT8, b_src, dims, strides, box, sw)) return cudaErrorInvalidValue;
     }
-    {   // sV [n2][ng][T_pad] fp32, box 128 x gps x TPS
-        const cuuint64_t dims[3] = {(cuuint64_t)a.T_pad, (cuuint64_t)a.ng, (cuuint64_t)a.n2};
-        const cuuint64_t strides[2] = {(cuuint64_t)a.T_pad * 4, (cuuint64_t)a.ng * a.T_pad * 4};
+    {   // row scales [n2][ng][a_rows] fp32, box 128 x gps x TPS
+        const cuuint64_t dims[3] = {a_rows, (cuuint64_t)a.ng, (cuuint64_t)a.n2};
+        const cuuint64_t strides[2] = {a_rows * 4, (cuuint64_t)a.ng * a_rows * 4};
         const cuuint32_t box[3] = {(cuuint32_t)kBM, (cuuint32_t)gps, (cuuint32_t)a.tps};
-        if (!encode(enc, &m.sv, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, a.sV, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_NONE))
+        if (!encode(enc, &m.sv, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, ra_src, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_NONE))
             return cudaErrorInvalidValue;
     }
-    {   // sU [n2][ng][Cout] fp32, box BN x gps x TPS
-        const cuuint64_t dims[3] = {(cuuint64_t)a.Cout, (cuuint64_t)a.ng, (cuuint64_t)a.n2};
-        const cuuint64_t strides[2] = {(cuuint64_t)a.Cout * 4, (cuuint64_t)a.ng * a.Cout * 4};
+    {   // column scales [n2][ng][b_rows] fp32, box BN x gps x TPS
+        const cuuint64_t dims[3] = {b_rows, (cuuint64_t)a.ng, (cuuint64_t)a.n2};
+        const cuuint64_t strides[2] = {b_rows * 4, (cuuint64_t)a.ng * b_rows * 4};
         const cuuint32_t box[3] = {(cuuint32_t)BN, (cuuint32_t)gps, (cuuint32_t)a.tps};
-        if (!encode(enc, &m.su, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, a.sU, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_NONE))
+        if (!encode(enc, &m.su, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, cb_src, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_NONE))
             return cudaErrorInvalidValue;
     }
     if (launches) ++*launches;
+    if (swap) return BN == 16 ? launch_swap<16>(a, m, mode, num_sms, st) : launch_swap<32>(a, m, mode, num_sms, st);
     if (BN == 64) return launch_bn<64>(a, m, mode, num_sms, st);
     return launch_bn<32>(a, m, mode, num_sms, st);
 }
