@@ -68,6 +68,10 @@ def parse():
     ap.add_argument("--e2e-steps", type=int, default=200)
     ap.add_argument("--y-groups", default="tile", choices=["tile", "tap"],
                     help="Y quantisation groups: tile (default reading) or tap (the per-tap option)")
+    ap.add_argument("--x-int8", action="store_true",
+                    help="alternative reading: x group-quantised per pixel before the input transform")
+    ap.add_argument("--int8-transforms", action="store_true",
+                    help="alternative reading: B^T and A^T held as int8 with one scale per matrix")
     return ap.parse_args()
 
 
@@ -89,7 +93,7 @@ def load_peaks():
 
 
 # ----------------------------------------------------------------- byte model
-def stage_model(layer: synth.Layer, y_path: int):
+def stage_model(layer: synth.Layer, y_path: int, x_int8: bool = False):
     """Algorithmic bytes and int8 ops of each launch of one call, by launch index."""
     from group_wise_int8_b200 import wino
     n2 = layer.n * layer.n
@@ -103,7 +107,12 @@ def stage_model(layer: synth.Layer, y_path: int):
     amax = 4 * T * (layer.Cout // G)
     yq = T * n2 * layer.Cout
     ops = 2.0 * T * n2 * layer.Cin * layer.Cout
-    stages = [("input_transform", x + v + amax, 0.0)]
+    stages = []
+    if x_int8:   # reads x, writes its fp32 round trip, which the input transform then reads
+        xq = layer.N * layer.H * layer.W * layer.Cin * 4
+        stages.append(("input_quant", x + xq, 0.0))
+        x = xq
+    stages.append(("input_transform", x + v + amax, 0.0))
     if y_path == wino.YPATH_RECOMPUTE:
         stages.append(("hadamard_absmax", v + u + amax, ops))
         stages.append(("hadamard_quant", v + u + amax + yq, ops))
@@ -196,7 +205,8 @@ def run_ours(args, layer, rank, world):
     w = synth.make_weights(layer)
     sb, sg = synth.make_scales(layer)
     y_groups = wino.YGROUPS_TAP if getattr(args, "y_groups", "tile") == "tap" else wino.YGROUPS_TILE
-    plan = wino.Plan(layer.m, layer.points, sb, sg, layer.group, y_groups=y_groups)
+    plan = wino.Plan(layer.m, layer.points, sb, sg, layer.group, y_groups=y_groups, x_int8=args.x_int8,
+                     int8_transforms=args.int8_transforms)
     N, H, W, Cin, Cout = layer.N, layer.H, layer.W, layer.Cin, layer.Cout
     if x_bits is not None:
         x = torch.from_numpy(x_bits.view(np.int16).copy()).view(torch.bfloat16).to(dev)
@@ -284,7 +294,7 @@ def run_ours(args, layer, rank, world):
 
     # roofline of the dominant kernel
     peaks = load_peaks()
-    model = stage_model(layer, y_path)
+    model = stage_model(layer, y_path, args.x_int8)
     avg_ms = [t / calls for t in stage_ms]
     dom = int(np.argmax(avg_ms))
     name, nbytes, ops = model[dom]
@@ -310,7 +320,7 @@ def run_ours(args, layer, rank, world):
 
 
 # ------------------------------------------------------------- CPU oracle timing
-def oracle_sample(layer: synth.Layer, rows: int, images: int):
+def oracle_sample(layer: synth.Layer, rows: int, images: int, int8_transforms: bool = False):
     """The layer cropped to `rows` tile rows of `images` images (same weights)."""
     import oracle
     x_f32, _ = synth.make_input(layer)
@@ -318,29 +328,32 @@ def oracle_sample(layer: synth.Layer, rows: int, images: int):
     sb, sg = synth.make_scales(layer)
     H = min(layer.H, rows * layer.m)
     xs = np.ascontiguousarray(x_f32[:images, :H])
-    plan = oracle.Plan(layer.m, layer.points, sb, sg)
+    plan = oracle.Plan(layer.m, layer.points, sb, sg, int8_transforms=int8_transforms)
     Uq, sU, _ = oracle.weight_transform(plan, w, layer.group)
     flops = 2.0 * images * H * layer.W * layer.Cin * layer.Cout * 9
     return plan, xs, Uq, sU, flops
 
 
-def oracle_step(plan, xs, Uq, sU, G, per_tap=False):
+def oracle_step(plan, xs, Uq, sU, G, per_tap=False, x_int8=False):
     import oracle
     n2 = plan.n * plan.n
     N, H, W, _ = xs.shape
+    if x_int8:
+        xs = oracle.quantize_input(xs, G)
     Vq, sV, _ = oracle.input_transform(plan, xs, G)
     Y, _ = oracle.hadamard(n2, Vq, sV, Uq, sU, G)
     Yq, sY = oracle.y_requant(n2, Y, G, per_tap)
     oracle.output_transform(plan, Yq, sY, N, H, W, G, per_tap)
 
 
-def cpu_baseline(layer: synth.Layer, budget_s: float = 12.0, per_tap: bool = False):
+def cpu_baseline(layer: synth.Layer, budget_s: float = 12.0, per_tap: bool = False, x_int8: bool = False,
+                 int8_transforms: bool = False):
     import oracle
     threads = oracle.set_threads(0)
     rows, images = 1, 1
-    plan, xs, Uq, sU, flops = oracle_sample(layer, rows, images)
+    plan, xs, Uq, sU, flops = oracle_sample(layer, rows, images, int8_transforms)
     t0 = time.perf_counter()
-    oracle_step(plan, xs, Uq, sU, layer.group, per_tap)
+    oracle_step(plan, xs, Uq, sU, layer.group, per_tap, x_int8)
     dt = time.perf_counter() - t0
     # grow the sample (whole images first) while it stays within the budget
     TH = -(-layer.H // layer.m)
@@ -349,14 +362,14 @@ def cpu_baseline(layer: synth.Layer, budget_s: float = 12.0, per_tap: bool = Fal
             rows = min(TH, rows * 2)
         else:
             images = min(layer.N, images * 2)
-        plan, xs, Uq, sU, flops = oracle_sample(layer, rows, images)
+        plan, xs, Uq, sU, flops = oracle_sample(layer, rows, images, int8_transforms)
         t0 = time.perf_counter()
-        oracle_step(plan, xs, Uq, sU, layer.group, per_tap)
+        oracle_step(plan, xs, Uq, sU, layer.group, per_tap, x_int8)
         dt = time.perf_counter() - t0
     reps = max(1, int(budget_s / 2 / max(dt, 1e-3)))
     t0 = time.perf_counter()
     for _ in range(reps):
-        oracle_step(plan, xs, Uq, sU, layer.group, per_tap)
+        oracle_step(plan, xs, Uq, sU, layer.group, per_tap, x_int8)
     dt = (time.perf_counter() - t0) / reps
     return {"value": flops / dt / 1e12, "unit": UNIT, "cores": threads, "kind": "oracle",
             "sample": "%d image(s) x %d of %d tile rows of %s; input transform, Hadamard, Y requant, output "
@@ -365,26 +378,27 @@ def cpu_baseline(layer: synth.Layer, budget_s: float = 12.0, per_tap: bool = Fal
 
 def run_reference(args, layer):
     per_tap = args.y_groups == "tap"
+    x_int8 = args.x_int8
     import oracle
     threads = oracle.set_threads(0)
     TH = -(-layer.H // layer.m)
     budget = 150.0 / max(1, args.steps + args.warmup)   # seconds per step: whole run within a few minutes
     rows = 1
-    plan, xs, Uq, sU, flops = oracle_sample(layer, rows, 1)
+    plan, xs, Uq, sU, flops = oracle_sample(layer, rows, 1, args.int8_transforms)
     t0 = time.perf_counter()
-    oracle_step(plan, xs, Uq, sU, layer.group, per_tap)
+    oracle_step(plan, xs, Uq, sU, layer.group, per_tap, x_int8)
     dt = time.perf_counter() - t0
     while dt * 2 <= budget and rows < TH:
         rows = min(TH, rows * 2)
-        plan, xs, Uq, sU, flops = oracle_sample(layer, rows, 1)
+        plan, xs, Uq, sU, flops = oracle_sample(layer, rows, 1, args.int8_transforms)
         t0 = time.perf_counter()
-        oracle_step(plan, xs, Uq, sU, layer.group, per_tap)
+        oracle_step(plan, xs, Uq, sU, layer.group, per_tap, x_int8)
         dt = time.perf_counter() - t0
     for _ in range(args.warmup):
-        oracle_step(plan, xs, Uq, sU, layer.group, per_tap)
+        oracle_step(plan, xs, Uq, sU, layer.group, per_tap, x_int8)
     t0 = time.perf_counter()
     for _ in range(args.steps):
-        oracle_step(plan, xs, Uq, sU, layer.group, per_tap)
+        oracle_step(plan, xs, Uq, sU, layer.group, per_tap, x_int8)
     total = time.perf_counter() - t0
     value = args.steps * flops / total / 1e12
     sample = "1 image x %d of %d tile rows of %s per step" % (rows, TH, layer.describe())
@@ -401,7 +415,7 @@ def main():
               "global_batch": layer.N * world, "seq_len": None, "H": layer.H, "W": layer.W, "Cin": layer.Cin,
               "Cout": layer.Cout, "m": layer.m, "group": layer.group, "parallelism": "dp%d" % world,
               "l2": "flushed before every timed step (256 MiB write)", "output": "bf16 NHWC",
-              "y_groups": args.y_groups}
+              "y_groups": args.y_groups, "x_int8": args.x_int8, "int8_transforms": args.int8_transforms}
     line = {"metric": METRIC, "unit": UNIT, "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int8 (fp32 transforms)",
             "data": "synthetic (seeded)", "config": config}
@@ -432,7 +446,8 @@ def main():
         return
     cpu = None
     if not args.no_cpu_baseline and world == 1:
-        cpu = cpu_baseline(layer, per_tap=args.y_groups == "tap")
+        cpu = cpu_baseline(layer, per_tap=args.y_groups == "tap", x_int8=args.x_int8,
+                           int8_transforms=args.int8_transforms)
     line.update(value=r["value"], ms_per_step=r["ms_per_step"], e2e=r["e2e"], roofline=r["roofline"],
                 cpu_baseline=cpu, clocks=r["clocks"], gpu_launches=r["gpu_launches"],
                 kernels=r["per_kernel"], y_path=r["y_path"], gemm=r["gemm"], impl="ours")

@@ -10,7 +10,9 @@
 //
 // Each lane owns 8 consecutive values (one 16-byte bf16 load or two 16-byte fp32
 // loads), so G / 8 lanes share a group and combine their absmax with xor
-// shuffles; a warp covers 256 values per step of its grid-stride loop.
+// shuffles; a warp covers 256 values per step of its grid-stride loop.  The codes
+// come from the division-free exact quantiser (quant4) and s * q is one fp32
+// multiply per value.
 #include <algorithm>
 
 #include "common.cuh"
@@ -64,14 +66,14 @@ __global__ void __launch_bounds__(256) input_quant_kernel(const Tin* __restrict_
         for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(v[i]));
 #pragma unroll
         for (int off = 1; off < kLanes; off <<= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
-        const float s = group_scale(amax);
-        float o[8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) o[i] = __fmul_rn(s, (float)quant_code(v[i], s));
+        // codes without a division (quant4: exact, with its own fallback), then s * q in fp32
+        const QScale q = make_qscale(amax);
+        const uint64_t s2 = f2_pack(q.s, q.s);
+        const Quad a = quant4(v[0], v[1], v[2], v[3], q), b = quant4(v[4], v[5], v[6], v[7], q);
         if (live) {
-            float4* dst = reinterpret_cast<float4*>(xq + e);
-            dst[0] = make_float4(o[0], o[1], o[2], o[3]);
-            dst[1] = make_float4(o[4], o[5], o[6], o[7]);
+            ulonglong2* dst = reinterpret_cast<ulonglong2*>(xq + e);
+            dst[0] = make_ulonglong2(f2_mul(s2, a.k01), f2_mul(s2, a.k23));
+            dst[1] = make_ulonglong2(f2_mul(s2, b.k01), f2_mul(s2, b.k23));
         }
     }
 }

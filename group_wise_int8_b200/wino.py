@@ -237,10 +237,10 @@ class Plan:
 
     def profile_end(self):
         """-> (summed ms per launch index, calls recorded)."""
-        ms = (ctypes.c_float * 4)()
+        ms = (ctypes.c_float * 8)()
         nl, nc = _i(), _i()
-        self._check(_lib.wino_profile_end(self._h, ms, 4, ctypes.byref(nl), ctypes.byref(nc)), "wino_profile_end")
-        return [ms[i] for i in range(nl.value)], nc.value
+        self._check(_lib.wino_profile_end(self._h, ms, 8, ctypes.byref(nl), ctypes.byref(nc)), "wino_profile_end")
+        return [ms[i] for i in range(min(nl.value, 8))], nc.value
 
     def check_device_error(self, workspace: torch.Tensor, N, H, W, Cin, Cout, stream=None) -> int:
         return _lib.wino_check_device_error(self._h, workspace.data_ptr(), N, H, W, Cin, Cout, _stream_handle(stream))
