@@ -144,10 +144,10 @@ __global__ void __launch_bounds__(128, SRC_Y32 ? 6 : 4)
 // shared memory -- and one thread per (group, tap) stores the scale; pass 2 is
 // the fp32-Y path of output_transform_kernel with the tap's own scale.
 template <int M, uint64_t MASK, bool BF16_OUT>
-__global__ void __launch_bounds__(128) output_transform_ytap_kernel(OutputArgs p, TransformArgs tf) {
+__global__ void __launch_bounds__(128, 6) output_transform_ytap_kernel(OutputArgs p, TransformArgs tf) {
     constexpr int N = M + 2, N2 = N * N;
     __shared__ QScale qsm[4][2][N2];     // [warp][segment][tap] (G <= 64) or [group in CTA][0][tap]
-    __shared__ float red[4][N2];         // per-warp maxima (G >= 128)
+    __shared__ float red[4][2][N2];      // per-warp (and segment) maxima
     grid_dependents_launch();
     grid_dependency_wait();
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -161,40 +161,44 @@ __global__ void __launch_bounds__(128) output_transform_ytap_kernel(OutputArgs p
     const size_t base = (size_t)(live ? t : 0) * p.Cout + co;
     const size_t tstride = (size_t)p.T * p.Cout;
 
-    // ---- pass 1: per-tap group scales
+    // ---- pass 1: per-tap group scales.  Eight taps at a time: their loads in flight together
+    // and their lane reductions interleaved; the segment's first lane keeps the maxima.
+    const int seg_w = G <= 64 ? G / 2 : 32;        // lanes of the warp reduced together
+    const int seg = lane / seg_w, sl = lane % seg_w;
+    for (int t0 = 0; t0 < N2; t0 += 8) {
+        float a[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+            a[k] = 0.0f;
+            if (live && t0 + k < N2) {
+                const float2 y = *reinterpret_cast<const float2*>(p.Y32 + base + (size_t)(t0 + k) * tstride);
+                a[k] = fmaxf(fabsf(y.x), fabsf(y.y));
+            }
+        }
+        for (int o = seg_w / 2; o > 0; o >>= 1)
+#pragma unroll
+            for (int k = 0; k < 8; ++k) a[k] = fmaxf(a[k], __shfl_xor_sync(0xffffffffu, a[k], o));
+        if (sl == 0)
+#pragma unroll
+            for (int k = 0; k < 8; ++k)
+                if (t0 + k < N2) red[warp][seg][t0 + k] = a[k];
+    }
     if (G <= 64) {
-        const int seg_w = G / 2;                   // lanes per group
-        const int seg = lane / seg_w, sl = lane % seg_w;
-        for (int tap = 0; tap < N2; ++tap) {
-            float a = 0.0f;
-            if (live) {
-                const float2 y = *reinterpret_cast<const float2*>(p.Y32 + base + (size_t)tap * tstride);
-                a = fmaxf(fabsf(y.x), fabsf(y.y));
-            }
-            for (int o = seg_w / 2; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
-            if (sl == tap % seg_w) {
-                qsm[warp][seg][tap] = make_qscale(a);
-                if (p.sY_dbg && live) p.sY_dbg[((size_t)t * N2 + tap) * p.ngo + cg] = qsm[warp][seg][tap].s;
-            }
+        __syncwarp();
+        // each lane of the segment derives the scales of every seg_w-th tap
+        for (int tap = sl; tap < N2; tap += seg_w) {
+            qsm[warp][seg][tap] = make_qscale(red[warp][seg][tap]);
+            if (p.sY_dbg && live) p.sY_dbg[((size_t)t * N2 + tap) * p.ngo + cg] = qsm[warp][seg][tap].s;
         }
         __syncwarp();
     } else {
-        for (int tap = 0; tap < N2; ++tap) {
-            float a = 0.0f;
-            if (live) {
-                const float2 y = *reinterpret_cast<const float2*>(p.Y32 + base + (size_t)tap * tstride);
-                a = fmaxf(fabsf(y.x), fabsf(y.y));
-            }
-            for (int o = 16; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
-            if (lane == 0) red[warp][tap] = a;
-        }
         __syncthreads();
         const int wpg = G / 64;                    // warps per group
         const int ngc = 4 / wpg;                   // groups in the CTA
         for (int k = threadIdx.x; k < ngc * N2; k += blockDim.x) {
             const int gi = k / N2, tap = k % N2;
             float a = 0.0f;
-            for (int w = 0; w < wpg; ++w) a = fmaxf(a, red[gi * wpg + w][tap]);
+            for (int w = 0; w < wpg; ++w) a = fmaxf(a, red[gi * wpg + w][0][tap]);
             qsm[gi][0][tap] = make_qscale(a);
             const long i0 = (long)blockIdx.x * blockDim.x + gi * (G / 2);   // first thread of the group
             const long tg = i0 / cpairs;
