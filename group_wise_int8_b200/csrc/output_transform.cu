@@ -262,6 +262,88 @@ __global__ void __launch_bounds__(128, 6) output_transform_ytap_kernel(OutputArg
     }
 }
 
+// Layers with few (tile, channel pair) items -- too few for one thread each to fill the GPU --
+// on the fp32-Y path: N threads per item, one per column nu of Y.  Thread nu requantises its
+// column's N taps and forms column nu of Z = A^T Yd; after a warp barrier thread r < M forms
+// output row r from row r of Z.  The arithmetic and every chain order are those of
+// output_transform_kernel; each thread's chain is an N-th as long.
+template <int M, uint64_t MASK, bool BF16_OUT, bool DEBUG>
+__global__ void __launch_bounds__(128) output_transform_split_kernel(OutputArgs p, TransformArgs tf) {
+    constexpr int N = M + 2;
+    constexpr int IPW = 32 / N;                   // items per warp (F(4,3): lanes 30, 31 idle)
+    __shared__ uint64_t zs[4][IPW][M][N];         // Z of each item, (co, co + 1) pairs
+    grid_dependents_launch();
+    grid_dependency_wait();
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int slot = lane / N, nu = lane - slot * N;
+    const long item = ((long)blockIdx.x * 4 + warp) * IPW + slot;   // (tile, channel pair)
+    const int cpairs = p.Cout >> 1;
+    const long t = item / cpairs;
+    const int co = 2 * (int)(item - t * cpairs);
+    const bool live = slot < IPW && t < p.T;
+    if (live) {
+        const int cg = co / p.G;
+        const QScale qs = make_qscale(__uint_as_float(p.amax[(size_t)t * p.ngo + cg]));
+        if (DEBUG && nu == 0 && co % p.G == 0) p.sY_dbg[(size_t)t * p.ngo + cg] = qs.s;
+        const uint64_t s2 = f2_pack(qs.s, qs.s);
+        const size_t base = (size_t)t * p.Cout + co;
+        const size_t tstride = (size_t)p.T * p.Cout;
+        uint64_t Yc[N];                           // column nu of Yd: taps xi * N + nu
+#pragma unroll
+        for (int xi = 0; xi < N; xi += 2) {
+            const float2 a = *reinterpret_cast<const float2*>(p.Y32 + base + (size_t)(xi * N + nu) * tstride);
+            const float2 b = *reinterpret_cast<const float2*>(p.Y32 + base + (size_t)((xi + 1) * N + nu) * tstride);
+            const Quad qd = quant4(a.x, a.y, b.x, b.y, qs);
+            Yc[xi] = f2_mul(s2, qd.k01);
+            Yc[xi + 1] = f2_mul(s2, qd.k23);
+            if (DEBUG) {
+                *reinterpret_cast<uint16_t*>(p.Yq_dbg + base + (size_t)(xi * N + nu) * tstride) =
+                    (uint16_t)(qd.packed & 0xffffu);
+                *reinterpret_cast<uint16_t*>(p.Yq_dbg + base + (size_t)((xi + 1) * N + nu) * tstride) =
+                    (uint16_t)(qd.packed >> 16);
+            }
+        }
+#pragma unroll
+        for (int r = 0; r < M; ++r) {
+            uint64_t acc = 0ull;
+#pragma unroll
+            for (int xi = 0; xi < N; ++xi)
+                if ((MASK >> (r * N + xi)) & 1ull) acc = f2_fma(tf.ATd[r * N + xi], Yc[xi], acc);
+            zs[warp][slot][r][nu] = acc;
+        }
+    }
+    __syncwarp();
+    if (!live || nu >= M) return;
+    const int r = nu;                             // this thread's output row
+    const int TT = p.TH * p.TW;
+    const int img = (int)(t / TT);
+    const int rem = (int)(t - (long)img * TT);
+    const int ty = rem / p.TW, tx = rem - ty * p.TW;
+    const int yy = ty * M + r;
+    if (yy >= p.H) return;
+#pragma unroll
+    for (int c = 0; c < M; ++c) {
+        const int xx = tx * M + c;
+        if (xx >= p.W) break;
+        uint64_t acc = 0ull;
+#pragma unroll
+        for (int k = 0; k < N; ++k)
+            if ((MASK >> (c * N + k)) & 1ull) acc = f2_fma(zs[warp][slot][r][k], tf.ATd[c * N + k], acc);
+        float o0, o1;
+        f2_unpack(acc, o0, o1);
+        const size_t o = (((size_t)img * p.H + yy) * p.W + xx) * p.Cout + co;
+        if (BF16_OUT)
+            *reinterpret_cast<__nv_bfloat162*>(reinterpret_cast<__nv_bfloat16*>(p.out) + o) =
+                __floats2bfloat162_rn(o0, o1);
+        else
+            *reinterpret_cast<float2*>(reinterpret_cast<float*>(p.out) + o) = make_float2(o0, o1);
+    }
+}
+
+// Below this many (tile, channel pair) items (two CTAs of 128 per SM), the fp32-Y path splits
+// each item over N threads.
+constexpr long kSplitItems = 148L * 2 * 128;
+
 template <int M, uint64_t MASK>
 cudaError_t launch_m(const OutputArgs& a, const TransformArgs& tf, bool src_y32, bool bf16_out, bool debug,
                      cudaStream_t st) {
@@ -280,6 +362,18 @@ cudaError_t launch_m(const OutputArgs& a, const TransformArgs& tf, bool src_y32,
     if (a.ytap)
         return bf16_out ? launch_dependent(output_transform_ytap_kernel<M, MASK, true>, grid, dim3(128), 0, st, a, tf)
                         : launch_dependent(output_transform_ytap_kernel<M, MASK, false>, grid, dim3(128), 0, st, a, tf);
+    if (src_y32 && threads < kSplitItems) {   // too few items for one thread each: split them
+        constexpr int IPW = 32 / (M + 2);
+        const dim3 sgrid((unsigned)((threads + 4 * IPW - 1) / (4 * IPW)));
+#define WINO_SPLIT_LAUNCH(BF, DBG) \
+    return launch_dependent(output_transform_split_kernel<M, MASK, BF, DBG>, sgrid, dim3(128), 0, st, a, tf)
+        if (bf16_out) {
+            if (debug) WINO_SPLIT_LAUNCH(true, true); else WINO_SPLIT_LAUNCH(true, false);
+        } else {
+            if (debug) WINO_SPLIT_LAUNCH(false, true); else WINO_SPLIT_LAUNCH(false, false);
+        }
+#undef WINO_SPLIT_LAUNCH
+    }
 #define WINO_OUT_LAUNCH(Y32, BF, DBG) \
     return launch_dependent(output_transform_kernel<M, MASK, Y32, BF, DBG>, grid, dim3(128), 0, st, tm, a, tf)
     if (src_y32) {

@@ -39,6 +39,9 @@ CASES = {
     "f2_ragged": (2, P2, 2, 13, 11, 64, 64, 32, "bf16", "relu_normal", "loguniform"),
     "f2_g64_cout128_f32": (2, P2, 1, 30, 30, 128, 128, 64, "f32", "student_t_outliers", "loguniform"),
     "f2_permuted_points": (2, (math.inf, -1.0, 0.0, 1.0), 1, 9, 10, 32, 64, 32, "bf16", "normal", "loguniform"),
+    # enough (tile, channel pair) items for the one-thread-per-item fp32-Y output kernel; the
+    # smaller cases take the split kernel on that path
+    "f6_many_items": (6, P6, 4, 60, 59, 64, 256, 64, "bf16", "relu_normal", "loguniform"),
 }
 
 
