@@ -42,6 +42,9 @@ CASES = {
     # enough (tile, channel pair) items for the one-thread-per-item fp32-Y output kernel; the
     # smaller cases take the split kernel on that path
     "f6_many_items": (6, P6, 4, 60, 59, 64, 256, 64, "bf16", "relu_normal", "loguniform"),
+    # enough tiles per channel group for the one-thread-per-item input transform (the smaller
+    # cases take its split kernel)
+    "f6_many_tiles": (6, P6, 24, 56, 56, 64, 32, 32, "bf16", "relu_normal", "loguniform"),
 }
 
 
