@@ -233,6 +233,7 @@ int run_conv(wino_plan_s* p, const void* x, int x_dtype, int N, int H, int W, in
     ia.sV = sV;
     ia.amax = amax;
     ia.err = err;
+    ia.num_sms = num_sms();
     prof_mark(p, slot++, st);
     cudaError_t e = launch_input_transform(ia, p->tf, p->mat.m, p->bt_masked, x_bf16, st);
     if (e != cudaSuccess) return cuda_status(p, e);
@@ -288,6 +289,7 @@ int run_conv(wino_plan_s* p, const void* x, int x_dtype, int N, int H, int W, in
     oa.out = y;
     oa.ytap = L.ytap ? 1 : 0;
     oa.err = err;
+    oa.num_sms = num_sms();
     prof_mark(p, slot++, st);
     e = launch_output_transform(oa, p->tf, p->mat.m, p->at_masked, L.y_path == WINO_YPATH_Y32, y_dtype == WINO_BF16,
                                 st);

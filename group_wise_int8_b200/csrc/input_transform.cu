@@ -354,9 +354,8 @@ __global__ void __launch_bounds__(InSplitCfg<M, Tin, G>::kMaxThreads)
     quant_batch<G, TB, Cfg::kMaxWarps>(vw, lane, warp, lwarp, h * TB, TX, tx0, row_id, g, p, red);
 }
 
-// Below this many threads in the grid above (a resident wave of three 160-thread CTAs per SM),
-// the split kernel runs instead.
-constexpr long kSplitInThreads = 148L * 3 * 160;
+// Below a resident wave of the grid above (three 160-thread CTAs per SM) the split kernel runs.
+inline long split_in_threads(int num_sms) { return (long)num_sms * 3 * 160; }
 
 template <int M, uint64_t MASK, typename Tin, int G>
 cudaError_t launch_split_g(const InputArgs& a, const TransformArgs& tf, cudaStream_t st) {
@@ -387,7 +386,7 @@ cudaError_t launch_g(const InputArgs& a, const TransformArgs& tf, cudaStream_t s
     const int max_tx = std::min(Cfg::kMaxThreads / (G / 2), (256 - 2) / M);
     const int nblk = (a.TW + max_tx - 1) / max_tx;
     const int TX = (a.TW + nblk - 1) / nblk;
-    if ((long)nblk * a.N * a.TH * (a.Cin / G) * Cfg::threads(TX) < kSplitInThreads)
+    if ((long)nblk * a.N * a.TH * (a.Cin / G) * Cfg::threads(TX) < split_in_threads(a.num_sms))
         return launch_split_g<M, MASK, Tin, G>(a, tf, st);
     // x [N][H][W][Cin] as a 4-D tensor (Cin, W, H, N); box G x (TX*m+2) x n x 1
     CUtensorMap tm;

@@ -57,6 +57,7 @@ struct InputArgs {
     float* sV;       // [n*n][Cin/G][T_pad]
     unsigned* amax;  // [T_pad][Cout/G], cleared here
     int* err;        // device error word, cleared here
+    int num_sms;     // SMs of the device (sizes the choice of the split kernel)
 };
 cudaError_t launch_input_transform(const InputArgs& a, const TransformArgs& tf, int m, bool masked, bool bf16_in,
                                    cudaStream_t st);
@@ -105,6 +106,7 @@ struct OutputArgs {
     void* out;             // [N][H][W][Cout] fp32 or bf16
     int ytap;              // per-tap Y groups (Y32 source; sY_dbg is then [T][n2][ngo])
     int* err;              // device error word (bounded waits)
+    int num_sms;           // SMs of the device (sizes the choice of the split kernel)
 };
 cudaError_t launch_output_transform(const OutputArgs& a, const TransformArgs& tf, int m, bool masked, bool src_y32,
                                     bool bf16_out, cudaStream_t st);

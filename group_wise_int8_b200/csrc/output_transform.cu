@@ -340,9 +340,9 @@ __global__ void __launch_bounds__(128) output_transform_split_kernel(OutputArgs 
     }
 }
 
-// Below this many (tile, channel pair) items (two CTAs of 128 per SM), the fp32-Y path splits
+// Below two 128-thread CTAs' worth of (tile, channel pair) items per SM, the fp32-Y path splits
 // each item over N threads.
-constexpr long kSplitItems = 148L * 2 * 128;
+inline long split_out_items(int num_sms) { return (long)num_sms * 2 * 128; }
 
 template <int M, uint64_t MASK>
 cudaError_t launch_m(const OutputArgs& a, const TransformArgs& tf, bool src_y32, bool bf16_out, bool debug,
@@ -362,7 +362,7 @@ cudaError_t launch_m(const OutputArgs& a, const TransformArgs& tf, bool src_y32,
     if (a.ytap)
         return bf16_out ? launch_dependent(output_transform_ytap_kernel<M, MASK, true>, grid, dim3(128), 0, st, a, tf)
                         : launch_dependent(output_transform_ytap_kernel<M, MASK, false>, grid, dim3(128), 0, st, a, tf);
-    if (src_y32 && threads < kSplitItems) {   // too few items for one thread each: split them
+    if (src_y32 && threads < split_out_items(a.num_sms)) {   // too few items for one thread each: split them
         constexpr int IPW = 32 / (M + 2);
         const dim3 sgrid((unsigned)((threads + 4 * IPW - 1) / (4 * IPW)));
 #define WINO_SPLIT_LAUNCH(BF, DBG) \
