@@ -59,3 +59,19 @@ def test_reference_arm_only_rank0_prints_under_two_ranks():
     lines = [l for l in r.stdout.splitlines() if l.startswith("{")]
     assert len(lines) == 1
     assert '"impl": "reference"' in lines[0]
+
+
+def test_stage_model_matches_launches_per_call():
+    """The benchmark's per-launch byte model lists one entry per kernel the library launches,
+    for every path and reading (int8 x adds its pass in front)."""
+    import bench
+    from group_wise_int8_b200 import synth, wino
+    layer = synth.workload("resnet18")[0]
+    shape = (layer.N, layer.H, layer.W, layer.Cin, layer.Cout)
+    for y_path in (wino.YPATH_RECOMPUTE, wino.YPATH_Y32):
+        for x_int8 in (False, True):
+            plan = wino.Plan(layer.m, layer.points, None, None, layer.group, y_path=y_path, x_int8=x_int8)
+            model = bench.stage_model(layer, plan.resolved_config(*shape)[0], x_int8)
+            assert len(model) == plan.launches_per_call(*shape)
+            assert (model[0][0] == "input_quant") == x_int8
+            assert all(nbytes > 0 for _, nbytes, _ in model)
