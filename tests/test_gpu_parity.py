@@ -169,15 +169,17 @@ def test_host_entry_point_matches_device_call(cuda_dev):
     assert torch.equal(y_host, y_dev.cpu())
 
 
+@pytest.mark.parametrize("x_int8", [False, True])
 @pytest.mark.parametrize("N", [3, 5, 9])
-def test_host_entry_point_chunks_match_device_call(cuda_dev, N):
-    """The host entry point pipelines chunks of images; its bytes equal one device call."""
+def test_host_entry_point_chunks_match_device_call(cuda_dev, N, x_int8):
+    """The host entry point pipelines chunks of images; its bytes equal one device call (also
+    with the int8-x reading, whose fp32 copy of x lives in each chunk's workspace)."""
     layer = synth.random_layer(4, 6, N, 14, 13, 64, 64, 32, dtype="f32", act="relu_normal",
                                scales="loguniform", workload="host_chunks")
     x_f32, _ = synth.make_input(layer)
     w = synth.make_weights(layer)
     sb, sg = synth.make_scales(layer)
-    plan = wino.Plan(6, P6, sb, sg, 32)
+    plan = wino.Plan(6, P6, sb, sg, 32, x_int8=x_int8)
     H, W, Cin, Cout = 14, 13, 64, 64
     wt = plan.transform_weights(torch.from_numpy(w).cuda())
     x_host = torch.from_numpy(x_f32).pin_memory()
