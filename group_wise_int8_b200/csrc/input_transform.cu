@@ -23,6 +23,8 @@
 // (the two chunks of a G=64 group combine across a lane pair, G >= 128 across
 // warps in shared memory), the group scale, and 32 codes (quant4), written as
 // two 16-byte stores of the tap-major Vq.
+// Layers with few tiles per channel group run a split kernel instead (below):
+// one thread per (tile, channel pair, batch of two rows of V), same chains.
 #include <algorithm>
 
 #include "kernels.h"

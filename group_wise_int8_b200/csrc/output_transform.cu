@@ -14,6 +14,9 @@
 // the per-cout chains and their order unchanged).  Lanes run along cout
 // pairs: every tap load and output store of a warp is contiguous.  Z is built
 // one column of Y at a time, so only Z and one Y column are live.
+// Variants: per-tap Y groups (the Y_TAP reading), and, for layers with few
+// (tile, channel pair) items on the fp32-Y path, a split kernel with N threads
+// per item (one per column of Y, then one per output row).
 #include <cstring>
 
 #include "kernels.h"
