@@ -29,6 +29,10 @@ struct wino_plan_s {
     int host_dev = -1;
     cudaStream_t copy_in = nullptr, copy_out = nullptr;
     std::vector<cudaEvent_t> host_events;
+    // chunk layout of the last pipelined host call (workspace, chunks, images per chunk, bytes per
+    // image in and out): a call with the same layout orders each chunk's input copy only after the
+    // previous call's compute of that chunk, so it overlaps the previous call's tail
+    size_t host_sig[5] = {0, 0, 0, 0, 0};
 };
 
 namespace {
@@ -438,6 +442,9 @@ int wino_conv2d_int8_host(wino_plan_t p, const void* x_host, int x_dtype, int N,
     if (ws_bytes < need + stage) return WINO_ERR_WORKSPACE;
     const size_t xs = x_dtype == WINO_BF16 ? 2 : 4, ys = y_dtype == WINO_BF16 ? 2 : 4;
     const size_t xrow = xs * H * W * Cin, yrow = ys * H * W * Cout;   // bytes per image
+    size_t prev_sig[5];
+    std::memcpy(prev_sig, p->host_sig, sizeof(prev_sig));
+    std::memset(p->host_sig, 0, sizeof(p->host_sig));   // set again only when this call is fully enqueued
     unsigned char* xd = static_cast<unsigned char*>(ws) + need;
     unsigned char* yd = xd + up(xrow * N, kAlign);
     cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -465,14 +472,22 @@ int wino_conv2d_int8_host(wino_plan_t p, const void* x_host, int x_dtype, int N,
     cudaEvent_t* ev = p->host_events.data();   // [0]: start, [1 + 3k ..]: in, compute, out of chunk k
     int* err = reinterpret_cast<int*>(static_cast<unsigned char*>(ws) + L.off_err);
     if ((e = cudaMemsetAsync(err, 0, sizeof(int), st)) != cudaSuccess) return cuda_status(p, e);
-    cudaEventRecord(ev[0], st);
-    cudaStreamWaitEvent(p->copy_in, ev[0], 0);
-    cudaStreamWaitEvent(p->copy_out, ev[0], 0);
+    // The staging buffers behind the workspace are only touched by these calls.  After a call
+    // of the same layout, chunk k's input copy waits for that call's compute of chunk k (the
+    // last reader of its staging slice); otherwise every copy waits for the stream's prior work.
+    const size_t sig[5] = {reinterpret_cast<size_t>(ws), (size_t)K, (size_t)Nc, xrow, yrow};
+    const bool chained = std::memcmp(sig, prev_sig, sizeof(sig)) == 0;
+    if (!chained) {
+        cudaEventRecord(ev[0], st);
+        cudaStreamWaitEvent(p->copy_in, ev[0], 0);
+        cudaStreamWaitEvent(p->copy_out, ev[0], 0);
+    }
     const unsigned char* xh = static_cast<const unsigned char*>(x_host);
     unsigned char* yh = static_cast<unsigned char*>(y_host);
     for (int k = 0; k < K; ++k) {
         const int n0 = k * Nc, nk = std::min(Nc, N - n0);
         unsigned char* buf = static_cast<unsigned char*>(ws) + (size_t)(k & 1) * need_c;
+        if (chained) cudaStreamWaitEvent(p->copy_in, ev[2 + 3 * k], 0);   // previous call's compute of chunk k
         if ((e = cudaMemcpyAsync(xd + xrow * n0, xh + xrow * n0, xrow * nk, cudaMemcpyHostToDevice, p->copy_in)) !=
             cudaSuccess)
             return cuda_status(p, e);
@@ -490,6 +505,7 @@ int wino_conv2d_int8_host(wino_plan_t p, const void* x_host, int x_dtype, int N,
             return cuda_status(p, e);
         cudaEventRecord(ev[3 + 3 * k], p->copy_out);
     }
+    std::memcpy(p->host_sig, sig, sizeof(sig));
     return cuda_status(p, cudaStreamWaitEvent(st, ev[3 * K], 0));
 }
 

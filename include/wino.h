@@ -222,6 +222,12 @@ size_t wino_host_staging_bytes(wino_plan_t plan, int N, int H, int W, int Cin, i
  * identical to one call, every tile belonging to one image).  ws_dev must hold
  * wino_workspace_bytes() + wino_host_staging_bytes().  The caller synchronises
  * `stream` before reading y_host.  Calls on one plan must not run concurrently.
+ * Back-to-back calls of the same shape on the same workspace overlap: each
+ * chunk's input copy waits only for the previous call's convolution of that
+ * chunk, so the next batch streams in while the previous one finishes.  The
+ * staging part of ws_dev (beyond wino_workspace_bytes) must therefore be used
+ * by nothing but these calls, and x_host must not change until the call's
+ * work on `stream` has completed.
  */
 int wino_conv2d_int8_host(wino_plan_t plan, const void* x_host, int x_dtype, int N, int H, int W, int Cin,
                            const void* wt_dev, int Cout, void* y_host, int y_dtype, void* ws_dev, size_t ws_bytes,

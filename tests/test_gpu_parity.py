@@ -196,6 +196,35 @@ def test_host_entry_point_chunks_match_device_call(cuda_dev, N, x_int8):
     assert torch.equal(y_host, y_dev.cpu())
 
 
+def test_back_to_back_host_calls_overlap_safely(cuda_dev):
+    """Consecutive host calls of one shape overlap (the next batch's input copies start before
+    the previous call ends); with different inputs and outputs every call still gives the bytes
+    of its own device call."""
+    N, H, W, Cin, Cout = 8, 14, 13, 64, 64
+    plan = wino.Plan(6, P6, None, None, 32)
+    w = synth.make_weights(synth.random_layer(7, 6, N, H, W, Cin, Cout, 32, workload="host_b2b"))
+    wt = plan.transform_weights(torch.from_numpy(w).cuda())
+    ws = torch.empty(plan.workspace_bytes(N, H, W, Cin, Cout) +
+                     plan.host_staging_bytes(N, H, W, Cin, Cout, torch.bfloat16, torch.bfloat16),
+                     dtype=torch.uint8, device="cuda")
+    xs, ys = [], []
+    for seed in range(4):
+        layer = synth.random_layer(100 + seed, 6, N, H, W, Cin, Cout, 32, dtype="bf16", act="relu_normal",
+                                   workload="host_b2b")
+        _, bits = synth.make_input(layer)
+        xs.append(torch.from_numpy(bits.view(np.int16).copy()).view(torch.bfloat16).pin_memory())
+        ys.append(torch.empty((N, H, W, Cout), dtype=torch.bfloat16).pin_memory())
+    for _ in range(3):   # several rounds: later calls are chained to earlier ones
+        for x_h, y_h in zip(xs, ys):
+            plan.conv2d_host(x_h, wt, Cout, y_h, ws)
+        torch.cuda.synchronize()
+        assert plan.check_device_error(ws, N, H, W, Cin, Cout) == wino.OK
+        for x_h, y_h in zip(xs, ys):
+            y_dev = plan.conv2d(x_h.cuda(), wt, Cout, out_dtype=torch.bfloat16)
+            torch.cuda.synchronize()
+            assert torch.equal(y_h, y_dev.cpu())
+
+
 def test_repeated_calls_reuse_workspace(cuda_dev):
     """The workspace carries nothing between calls: a second call on a dirty
     workspace gives the same bits."""
