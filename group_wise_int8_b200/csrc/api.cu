@@ -146,7 +146,7 @@ int cuda_status(wino_plan_s* p, cudaError_t e) {
     return WINO_ERR_CUDA;
 }
 
-constexpr int kMaxHostChunks = 4;
+constexpr int kMaxHostChunks = 3;
 
 // The host entry point's copy streams and events, created on the current device.
 int ensure_host_streams(wino_plan_s* p) {

@@ -216,7 +216,7 @@ size_t wino_host_staging_bytes(wino_plan_t plan, int N, int H, int W, int Cin, i
  * buffers: copies x_host to the device, runs the convolution, copies the
  * result to y_host, all asynchronously with respect to stream (pinned host
  * memory gives truly asynchronous copies).  When N >= 2 the batch is cut into
- * up to 4 chunks of images, pipelined: the copy of chunk k+1 in and of chunk
+ * up to 3 chunks of images, pipelined: the copy of chunk k+1 in and of chunk
  * k-1 out overlap the convolution of chunk k (the copies run on two streams
  * the plan owns, ordered after and before `stream` by events; results are
  * identical to one call, every tile belonging to one image).  ws_dev must hold
