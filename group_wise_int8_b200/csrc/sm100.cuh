@@ -155,8 +155,6 @@ __device__ __forceinline__ void mma_commit(uint64_t* bar) {
 
 __device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
-__device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
-
 // 32 lanes x NC consecutive 32-bit columns (this warp's lane quadrant), NC = 4, 8, 16 or 32.
 #define WINO_R8(o) "=r"(r[o + 0]), "=r"(r[o + 1]), "=r"(r[o + 2]), "=r"(r[o + 3]), "=r"(r[o + 4]), "=r"(r[o + 5]), \
                    "=r"(r[o + 6]), "=r"(r[o + 7])
@@ -191,31 +189,6 @@ __device__ __forceinline__ void tmem_ld<32>(uint32_t taddr, uint32_t (&r)[32]) {
         : "r"(taddr));
 }
 #undef WINO_R8
-
-// Writes the same 32-bit value to NC consecutive columns of this warp's lanes.
-template <int NC>
-__device__ __forceinline__ void tmem_fill(uint32_t taddr, uint32_t v);
-template <>
-__device__ __forceinline__ void tmem_fill<8>(uint32_t taddr, uint32_t v) {
-    asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%1,%1,%1,%1,%1,%1,%1};" ::"r"(taddr), "r"(v)
-                 : "memory");
-}
-template <>
-__device__ __forceinline__ void tmem_fill<16>(uint32_t taddr, uint32_t v) {
-    asm volatile("tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1};" ::"r"(
-                     taddr),
-                 "r"(v)
-                 : "memory");
-}
-template <>
-__device__ __forceinline__ void tmem_fill<32>(uint32_t taddr, uint32_t v) {
-    asm volatile(
-        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
-        "{%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,"
-        "%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1};" ::"r"(taddr),
-        "r"(v)
-        : "memory");
-}
 
 // Shared-memory matrix descriptor, K-major operand, swizzle of `sw_bytes`
 // (32, 64 or 128) equal to the row pitch; 8-row groups are 8 * sw_bytes apart.
