@@ -123,7 +123,12 @@ def _dtype_code(dt: torch.dtype) -> int:
 
 
 class Plan:
-    """A wino_plan: transforms of F(m,3) for the given points and scales."""
+    """A wino_plan: transforms of F(m,3) for the given points and scales.
+
+    Options (wino_opts): y_path / gemm select the Y route and the GEMM kernel (AUTO by default);
+    debug enables the dumps; y_groups selects the Y grouping (TILE, the default reading, or TAP);
+    x_int8 and int8_transforms select the alternative input-side readings (int8 x per pixel
+    group before the transform; int8 B^T and A^T with one scale per matrix)."""
 
     def __init__(self, m: int, points: Sequence[float], S_B=None, S_G=None, group: int = 32,
                  y_path: int = YPATH_AUTO, gemm: int = GEMM_AUTO, debug: int = 0, y_groups: int = YGROUPS_TILE,
