@@ -91,6 +91,18 @@ def test_plan_int8_transforms_match_oracle(lib, m, pts, scaled):
     assert not np.array_equal(BT0, BT)
 
 
+def test_short_layers_take_the_fp32_y_path(lib):
+    """At most 32 tiles with Cout a multiple of 128: AUTO resolves to the fp32-Y path (whose GEMM
+    pass runs with swapped operands); an explicit recompute request is kept."""
+    auto = wino.Plan(6, synth.POINTS_F6, None, None, 64)
+    assert auto.resolved_config(2, 8, 8, 1280, 1280)[0] == wino.YPATH_Y32          # T = 8
+    assert auto.resolved_config(2, 16, 16, 1280, 1280)[0] == wino.YPATH_Y32        # T = 18
+    rec = wino.Plan(6, synth.POINTS_F6, None, None, 64, y_path=wino.YPATH_RECOMPUTE)
+    assert rec.resolved_config(2, 8, 8, 1280, 1280)[0] == wino.YPATH_RECOMPUTE
+    assert rec.launches_per_call(2, 8, 8, 1280, 1280) == 4
+    assert auto.launches_per_call(2, 8, 8, 1280, 1280) == 3
+
+
 def test_x_int8_option_adds_a_launch_and_workspace(lib):
     shape = (2, 20, 20, 64, 64)
     p0 = wino.Plan(6, synth.POINTS_F6, None, None, 32)
