@@ -174,7 +174,12 @@ size_t wino_workspace_bytes(wino_plan_t plan, int N, int H, int W, int Cin, int 
  *   y_dev    [N][H][W][Cout] in y_dtype (WINO_F32 or WINO_BF16, RNE), device.
  *   ws_dev   device workspace of ws_bytes >= wino_workspace_bytes().
  * Launches (with x_int8: the quantisation of x, then) the input transform, the
- * Hadamard GEMM (one or two passes) and the output transform on stream; returns after the launches (asynchronous).
+ * Hadamard GEMM (one or two passes) and the output transform on stream.
+ * Kernel variants are chosen by shape and give identical bytes: with at most
+ * 32 tiles and Cout a multiple of 128, y_path AUTO resolves to Y32 and the GEMM
+ * pass runs with swapped operands (output channels on the MMA rows); layers
+ * with few tiles per SM run split transform kernels (more threads per tile).
+ * The call returns after the launches (asynchronous).
  * A bounded device wait that expires makes a later call on the same
  * workspace return WINO_ERR_DEVICE_TIMEOUT (see wino_check_device_error).
  * Errors: INVALID_ARG, UNSUPPORTED, WORKSPACE, CUDA, DEVICE_TIMEOUT.
