@@ -584,6 +584,20 @@ int wino_resolved_config(wino_plan_t p, int N, int H, int W, int Cin, int Cout, 
     return WINO_OK;
 }
 
+int wino_resolved_variants(wino_plan_t p, int N, int H, int W, int Cin, int Cout, int* flags) {
+    int rc = check_shape(p, N, H, W, Cin, Cout);
+    if (rc) return rc;
+    if (!flags) return WINO_ERR_INVALID_ARG;
+    const Layout L = make_layout(p, N, H, W, Cin, Cout);
+    int f = 0;
+    if (L.swap) f |= WINO_VARIANT_SWAPPED_GEMM;
+    if (input_transform_split(p->mat.m, p->G, N, L.TH, L.TW, Cin, num_sms())) f |= WINO_VARIANT_SPLIT_INPUT;
+    if (output_transform_split(L.T, Cout, L.y_path == WINO_YPATH_Y32, L.ytap, num_sms()))
+        f |= WINO_VARIANT_SPLIT_OUTPUT;
+    *flags = f;
+    return WINO_OK;
+}
+
 int wino_launches_per_call(wino_plan_t p, int N, int H, int W, int Cin, int Cout) {
     if (check_shape(p, N, H, W, Cin, Cout)) return 0;
     const Layout L = make_layout(p, N, H, W, Cin, Cout);

@@ -381,6 +381,19 @@ cudaError_t launch_split_g(const InputArgs& a, const TransformArgs& tf, cudaStre
     return launch_dependent(kern, grid, dim3(Cfg::threads(TX)), smem, st, tm, a, tf, TX);
 }
 
+}  // namespace
+
+bool input_transform_split(int m, int G, int N, int TH, int TW, int Cin, int num_sms) {
+    // the choice launch_g makes: tiles per CTA as there (at most 160 threads), then the grid size
+    const int max_tx = std::min(160 / (G / 2), (256 - 2) / m);
+    const int nblk = (TW + max_tx - 1) / max_tx;
+    const int TX = (TW + nblk - 1) / nblk;
+    const long threads = (TX * (G / 2) + 31) / 32 * 32;
+    return (long)nblk * N * TH * (Cin / G) * threads < split_in_threads(num_sms);
+}
+
+namespace {
+
 template <int M, uint64_t MASK, typename Tin, int G>
 cudaError_t launch_g(const InputArgs& a, const TransformArgs& tf, cudaStream_t st) {
     using Cfg = InCfg<M, Tin, G>;
@@ -388,8 +401,8 @@ cudaError_t launch_g(const InputArgs& a, const TransformArgs& tf, cudaStream_t s
     const int max_tx = std::min(Cfg::kMaxThreads / (G / 2), (256 - 2) / M);
     const int nblk = (a.TW + max_tx - 1) / max_tx;
     const int TX = (a.TW + nblk - 1) / nblk;
-    if ((long)nblk * a.N * a.TH * (a.Cin / G) * Cfg::threads(TX) < split_in_threads(a.num_sms))
-        return launch_split_g<M, MASK, Tin, G>(a, tf, st);
+    static_assert(Cfg::kMaxThreads == 160, "input_transform_split mirrors this configuration");
+    if (input_transform_split(M, G, a.N, a.TH, a.TW, a.Cin, a.num_sms)) return launch_split_g<M, MASK, Tin, G>(a, tf, st);
     // x [N][H][W][Cin] as a 4-D tensor (Cin, W, H, N); box G x (TX*m+2) x n x 1
     CUtensorMap tm;
     const cuuint64_t es = sizeof(Tin);

@@ -62,6 +62,9 @@ struct InputArgs {
 cudaError_t launch_input_transform(const InputArgs& a, const TransformArgs& tf, int m, bool masked, bool bf16_in,
                                    cudaStream_t st);
 
+// Whether a layer of this shape runs the split input-transform kernel.
+bool input_transform_split(int m, int G, int N, int TH, int TW, int Cin, int num_sms);
+
 // Group-wise int8 on x itself: xq = s * Q(x) per G consecutive channels of a pixel
 // (elems = N*H*W*Cin values, x bf16 or fp32, xq fp32; both 16-byte aligned).
 cudaError_t launch_input_quant(const void* x, bool bf16_in, long elems, int G, float* xq, int num_sms,
@@ -110,5 +113,7 @@ struct OutputArgs {
 };
 cudaError_t launch_output_transform(const OutputArgs& a, const TransformArgs& tf, int m, bool masked, bool src_y32,
                                     bool bf16_out, cudaStream_t st);
+// Whether a layer of this shape runs the split output-transform kernel.
+bool output_transform_split(long T, int Cout, bool src_y32, bool ytap, int num_sms);
 
 }  // namespace wino

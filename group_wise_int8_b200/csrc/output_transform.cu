@@ -347,6 +347,14 @@ __global__ void __launch_bounds__(128) output_transform_split_kernel(OutputArgs 
 // each item over N threads.
 inline long split_out_items(int num_sms) { return (long)num_sms * 2 * 128; }
 
+}  // namespace
+
+bool output_transform_split(long T, int Cout, bool src_y32, bool ytap, int num_sms) {
+    return src_y32 && !ytap && T * (long)(Cout / 2) < split_out_items(num_sms);
+}
+
+namespace {
+
 template <int M, uint64_t MASK>
 cudaError_t launch_m(const OutputArgs& a, const TransformArgs& tf, bool src_y32, bool bf16_out, bool debug,
                      cudaStream_t st) {
@@ -365,7 +373,7 @@ cudaError_t launch_m(const OutputArgs& a, const TransformArgs& tf, bool src_y32,
     if (a.ytap)
         return bf16_out ? launch_dependent(output_transform_ytap_kernel<M, MASK, true>, grid, dim3(128), 0, st, a, tf)
                         : launch_dependent(output_transform_ytap_kernel<M, MASK, false>, grid, dim3(128), 0, st, a, tf);
-    if (src_y32 && threads < split_out_items(a.num_sms)) {   // too few items for one thread each: split them
+    if (output_transform_split(a.T, a.Cout, src_y32, a.ytap != 0, a.num_sms)) {   // too few items for one thread each
         constexpr int IPW = 32 / (M + 2);
         const dim3 sgrid((unsigned)((threads + 4 * IPW - 1) / (4 * IPW)));
 #define WINO_SPLIT_LAUNCH(BF, DBG) \

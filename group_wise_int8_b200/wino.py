@@ -32,6 +32,7 @@ YPATH_AUTO, YPATH_RECOMPUTE, YPATH_Y32 = 0, 1, 2
 GEMM_AUTO, GEMM_TCGEN05, GEMM_SIMT = 0, 1, 2
 DEBUG_YQ, DEBUG_ACC32, DEBUG_FORCE_TIMEOUT = 1, 2, 4
 YGROUPS_TILE, YGROUPS_TAP = 0, 1
+VARIANT_SWAPPED_GEMM, VARIANT_SPLIT_INPUT, VARIANT_SPLIT_OUTPUT = 1, 2, 4
 DUMP_VQ, DUMP_SV, DUMP_YQ, DUMP_SY, DUMP_Y32, DUMP_ACC32 = range(6)
 
 EXPORTED = [
@@ -39,7 +40,7 @@ EXPORTED = [
     "wino_transform_weights", "wino_workspace_bytes", "wino_conv2d_int8", "wino_conv2d_int8_noalloc",
     "wino_host_staging_bytes",
     "wino_conv2d_int8_host", "wino_check_device_error", "wino_debug_dump", "wino_resolved_config",
-    "wino_launches_per_call", "wino_profile_begin", "wino_profile_end", "wino_last_cuda_error",
+    "wino_resolved_variants", "wino_launches_per_call", "wino_profile_begin", "wino_profile_end", "wino_last_cuda_error",
     "wino_status_string",
 ]
 
@@ -90,6 +91,7 @@ def load_library(path: str = LIB_PATH):
     L.wino_check_device_error.argtypes = [_vp, _vp, _i, _i, _i, _i, _i, _vp]
     L.wino_debug_dump.argtypes = [_vp, _vp, _i, _i, _i, _i, _i, _i, _vp, _sz]
     L.wino_resolved_config.argtypes = [_vp, _i, _i, _i, _i, _i, ctypes.POINTER(_i), ctypes.POINTER(_i)]
+    L.wino_resolved_variants.argtypes = [_vp, _i, _i, _i, _i, _i, ctypes.POINTER(_i)]
     L.wino_launches_per_call.argtypes = [_vp, _i, _i, _i, _i, _i]
     L.wino_profile_begin.argtypes = [_vp, _i]
     L.wino_profile_end.argtypes = [_vp, ctypes.POINTER(ctypes.c_float), _i, ctypes.POINTER(_i), ctypes.POINTER(_i)]
@@ -182,6 +184,13 @@ class Plan:
         self._check(_lib.wino_resolved_config(self._h, N, H, W, Cin, Cout, ctypes.byref(yp), ctypes.byref(gm)),
                     "wino_resolved_config")
         return yp.value, gm.value
+
+    def resolved_variants(self, N, H, W, Cin, Cout) -> int:
+        """Bit set of VARIANT_* the call of this shape runs (same bytes in every variant)."""
+        f = _i()
+        self._check(_lib.wino_resolved_variants(self._h, N, H, W, Cin, Cout, ctypes.byref(f)),
+                    "wino_resolved_variants")
+        return f.value
 
     def launches_per_call(self, N, H, W, Cin, Cout) -> int:
         return int(_lib.wino_launches_per_call(self._h, N, H, W, Cin, Cout))

@@ -161,3 +161,26 @@ def test_resolved_config_cost_model(lib):
     forced = wino.Plan(6, synth.POINTS_F6, None, None, 64, y_path=wino.YPATH_RECOMPUTE, gemm=wino.GEMM_SIMT)
     assert forced.resolved_config(2, 8, 8, 1280, 1280) == (wino.YPATH_RECOMPUTE, wino.GEMM_SIMT)
     assert forced.launches_per_call(2, 8, 8, 1280, 1280) == 4
+
+
+def test_parity_cases_cover_every_kernel_variant(lib):
+    """The GPU parity cases (stagewise, both Y paths) run each shape-chosen variant -- swapped GEMM,
+    split input and split output transforms -- and also each kernel it replaces, so bit-exactness
+    is checked on both sides of every choice (SM count 148, as on the B200)."""
+    from tests.test_gpu_parity import CASES
+    seen = {}
+    for name, (m, pts, N, H, W, Cin, Cout, G, *_rest) in CASES.items():
+        for y_path in (wino.YPATH_RECOMPUTE, wino.YPATH_Y32):
+            flags = wino.Plan(m, pts, None, None, G, y_path=y_path).resolved_variants(N, H, W, Cin, Cout)
+            for bit in (wino.VARIANT_SWAPPED_GEMM, wino.VARIANT_SPLIT_INPUT, wino.VARIANT_SPLIT_OUTPUT):
+                seen.setdefault(bit, set()).add(bool(flags & bit))
+    assert all(v == {False, True} for v in seen.values()), seen
+
+
+def test_variants_follow_the_shape(lib):
+    p = wino.Plan(6, synth.POINTS_F6, None, None, 64)
+    # SD-shaped C1280 8x8, N2: 8 tiles -> all three variants
+    assert p.resolved_variants(2, 8, 8, 1280, 1280) == (wino.VARIANT_SWAPPED_GEMM | wino.VARIANT_SPLIT_INPUT |
+                                                        wino.VARIANT_SPLIT_OUTPUT)
+    q = wino.Plan(6, synth.POINTS_F6, None, None, 32)
+    assert q.resolved_variants(32, 56, 56, 64, 64) == 0          # the default layer: none
