@@ -35,7 +35,10 @@
 //
 // Parity status: pinned by the CPU tests (exact Winograd identity with
 // quantisation off, scale invariance, textbook F(4,3) special case, quantiser
-// hand cases, brute-force integer accumulators, grouping properties).
+// hand cases, brute-force integer accumulators, grouping properties, hand-written
+// codes and scales of the tile-spanning Y requantisation -- ties, a clamp after a
+// denormal scale, an all-zero group, maxima at odd taps -- and matmul bounds for
+// both output transforms).
 //
 // Build: g++ -O2 -ffp-contract=off -fopenmp -shared -fPIC (no fast-math).
 

@@ -11,7 +11,11 @@ index, a transposed operand, a wrong grouping axis -- fails at least one):
     and scale invariance of the unquantised output.
   * Textbook special case: Lavin & Gray's F(4,3) matrices (the work the pages
     cite as [15]) are a diagonal rescaling of the Vandermonde transforms.
-  * Quantiser hand cases (absmax, ties to even, zero group, clamp).
+  * Quantiser hand cases (absmax, ties to even, zero group, clamp), and for the
+    tile-spanning Y requantisation a hand-written case whose every code and
+    scale is fixed (ties that round-half-away would move, a maximum at an odd
+    tap, groups that strided couts would split) plus a clamp after a denormal
+    scale.
   * Brute-force integer accumulators and the fp32 dequantisation bound.
   * Grouping-axis properties: per-tap V/U groups make the output invariant to
     power-of-two trades between S_B and S_G; tile-spanning Y groups make it
@@ -344,6 +348,139 @@ def test_y_tap_scales_are_per_tap_group_maxima():
     q = Yq.reshape(T, n2, Cout // G, G).astype(np.float64) * sY[..., None]
     err = np.abs(q - Y.reshape(T, n2, Cout // G, G))
     assert np.all(err <= 0.5 * sY[..., None] * (1 + 1e-6) + 1e-30)
+
+
+# -------------------------------------- Y requantisation, tile-spanning groups
+# The default reading: one scale per (tile, G consecutive output channels) over
+# all n*n taps of the tile (review, "Core claim" and Fig. 3: Y's cross-shaped
+# per-tap spread is what the group must span), Q with s = absmax/127 and ties to
+# even.  The hand case below fixes every code and scale by hand; each entry
+# names the slip it catches.
+
+_DENORM = 2.0 ** -149          # the smallest positive fp32 (a denormal)
+
+
+def _y_hand_case():
+    """T = 2 tiles, n2 = 16 taps (F(2,3)), Cout = 4, G = 2 (groups {0,1} and {2,3})."""
+    T, n2, Cout = 2, 16, 4
+    Y = np.zeros((T, n2, Cout), np.float32)
+    Yq = np.zeros((T, n2, Cout), np.int8)
+    sY = np.zeros((T, 2), np.float32)
+
+    def put(t, tap, co, v, q):
+        Y[t, tap, co] = v
+        Yq[t, tap, co] = q
+
+    # tile 0, group 0: the maximum 127 sits at an odd tap (13), so s = 1 exactly; a maximum taken
+    # over even taps only would give s = 100.25/127 and different codes
+    put(0, 13, 1, -127.0, -127)
+    put(0, 0, 0, 100.25, 100)
+    put(0, 2, 0, 0.5, 0)            # tie: to even 0 (half away from zero: 1)
+    put(0, 5, 0, 1.5, 2)            # tie: 2 either way
+    put(0, 6, 1, 2.5, 2)            # tie: to even 2 (half away: 3)
+    put(0, 7, 1, -2.5, -2)          # tie: to even -2 (half away: -3)
+    put(0, 8, 0, -3.5, -4)          # tie: to even -4
+    sY[0, 0] = 1.0
+    # tile 0, group 1 (couts 2, 3): all zero -> s = 0, every code 0
+    # tile 1, group 0: maximum 63.5 at tap 3 -> s = 0.5 exactly
+    put(1, 3, 0, 63.5, 127)
+    put(1, 4, 1, 0.25, 0)           # 0.5 -> 0 (half away: 1)
+    put(1, 9, 1, 0.75, 2)           # 1.5 -> 2
+    put(1, 10, 0, -31.25, -62)      # -62.5 -> -62 (half away: -63)
+    sY[1, 0] = 0.5
+    # tile 1, group 1: maximum |-254| at tap 15, cout 3 -> s = 2 exactly.  With groups of strided
+    # couts ({0, 2}, {1, 3}) tile 0's group of couts {0, 2} would get s = 100.25/127.
+    put(1, 15, 3, -254.0, -127)
+    put(1, 1, 2, 5.0, 2)            # 2.5 -> 2 (half away: 3)
+    put(1, 14, 2, 254.0, 127)
+    put(1, 12, 3, 3.0, 2)           # 1.5 -> 2
+    sY[1, 1] = 2.0
+    return Y, Yq, sY
+
+
+def test_y_tile_requant_hand_case():
+    Y, want_q, want_s = _y_hand_case()
+    Yq, sY = oracle.y_requant(16, Y, 2)
+    assert sY.shape == (2, 2)
+    assert np.array_equal(sY, want_s)
+    assert np.array_equal(Yq, want_q)
+
+
+def test_y_tile_requant_clamps_after_a_denormal_scale():
+    """absmax = 190 * 2^-149 (a denormal): s = RN(190/127 * 2^-149) = 2^-149, so 190 * 2^-149
+    divides to 190 and is clamped to 127 (and -150 * 2^-149 to -127); 3 * 2^-149 stays 3."""
+    Y = np.zeros((1, 4, 2), np.float32)
+    Y[0, 1, 0] = np.float32(190 * _DENORM)
+    Y[0, 2, 1] = np.float32(-150 * _DENORM)
+    Y[0, 3, 1] = np.float32(3 * _DENORM)
+    Yq, sY = oracle.y_requant(4, Y, 2)
+    assert sY[0, 0] == np.float32(_DENORM)
+    assert Yq[0, 1, 0] == 127 and Yq[0, 2, 1] == -127 and Yq[0, 3, 1] == 3
+    assert np.count_nonzero(Yq) == 3
+
+
+@pytest.mark.parametrize("n2,G", [(36, 32), (64, 64)])
+def test_y_tile_scales_are_maxima_over_every_tap_and_group_channel(n2, G):
+    """sY[t][j] = RN(max over all n2 taps and the G couts j*G..j*G+G-1 of |Y| / 127).  Every
+    group's maximum is planted at a random tap (odd taps included) and a random cout of the
+    group, with the rest of the group well below it, so a partial span of taps or couts, or
+    another grouping of the couts, changes the scale."""
+    r = np.random.default_rng(41)
+    T, Cout = 5, 4 * G
+    Y = (r.standard_normal((T, n2, Cout)) * 0.25).astype(np.float32)
+    Y[:, :, :G] = 0.0
+    Y[2, :, G:2 * G] = 0.0                       # one all-zero group
+    peak_tap = np.zeros((T, Cout // G), int)
+    for t in range(T):
+        for j in range(Cout // G):
+            if (t == 2 and j == 1) or j == 0:
+                continue
+            tap, co = int(r.integers(n2)), j * G + int(r.integers(G))
+            peak_tap[t, j] = tap
+            Y[t, tap, co] = np.float32((1 if r.random() < 0.5 else -1) * (3.0 + r.random()))
+    Y[:, 5, 3] = np.float32(2.0)                 # group 0: maxima at odd tap 5 only
+    Yq, sY = oracle.y_requant(n2, Y, G)
+    amax = np.abs(Y).reshape(T, n2, Cout // G, G).max(axis=(1, 3))
+    assert np.array_equal(sY, amax / np.float32(127.0))
+    assert np.all(sY[:, 0] == np.float32(2.0) / np.float32(127.0))
+    assert sY[2, 1] == 0.0 and not Yq[2, :, G:2 * G].any()
+    assert np.any(peak_tap % 2 == 1)
+    q = Yq.reshape(T, n2, Cout // G, G).astype(np.float64)
+    s = sY[:, None, :, None].astype(np.float64)
+    assert np.all(np.abs(q * s - Y.reshape(T, n2, Cout // G, G)) <= 0.5 * s * (1 + 1e-6) + 1e-45)
+    # the planted maxima map to +-127
+    for t in range(T):
+        for j in range(1, Cout // G):
+            if sY[t, j] > 0:
+                assert np.abs(Yq[t, :, j * G:(j + 1) * G].astype(int)).max() == 127
+
+
+def test_output_transform_tap_matches_matmul():
+    """Per-tap reading: out = A^T Yd A with Yd[xi][nu] = sY[t][xi*n+nu][co/G] * Yq, within the
+    fp32 rounding bound of the two fma chains.  The scales differ by powers of two from tap to
+    tap, so using the scale of another tap (a transposed tap index, a single scale per tile)
+    breaks the bound."""
+    m, n = 4, 6
+    p = oracle.Plan(m, P4, dyadic_scales(19, n), dyadic_scales(20, n))
+    r = np.random.default_rng(21)
+    N, H, W, Cout, G = 1, 7, 6, 4, 2
+    T = N * 2 * 2
+    n2 = n * n
+    Yq = r.integers(-127, 128, (T, n2, Cout)).astype(np.int8)
+    sY = (r.uniform(0.5, 1, (T, n2, Cout // G)) * 2.0 ** r.integers(-6, 7, (T, n2, Cout // G))).astype(np.float32)
+    out = oracle.output_transform(p, Yq, sY, N, H, W, G, per_tap=True)
+    AT = p.AT_f.astype(np.float64)
+    for t in range(T):
+        ty, tx = divmod(t, 2)
+        for co in range(Cout):
+            Yd = (sY[t, :, co // G] * Yq[t, :, co].astype(np.float32)).astype(np.float64).reshape(n, n)
+            ref = AT @ Yd @ AT.T
+            bound = 4 * n * np.finfo(np.float32).eps * (abs(AT) @ abs(Yd) @ abs(AT).T)
+            for i in range(m):
+                for j in range(m):
+                    yy, xx = ty * m + i, tx * m + j
+                    if yy < H and xx < W:
+                        assert abs(out[0, yy, xx, co] - ref[i, j]) <= bound[i, j] + 1e-30
 
 
 @pytest.mark.parametrize("m,pts", [(4, P4), (6, P6)])
