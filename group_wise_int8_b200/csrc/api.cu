@@ -2,12 +2,15 @@
 // Argument checking, workspace layout and kernel orchestration; all
 // arithmetic of the convolution runs in the CUDA kernels.
 #include <cuda_runtime.h>
+#include <nvtx3/nvToolsExt.h>
 
 #include <algorithm>
 #include <cmath>
 #include <cstdint>
 #include <cstring>
+#include <mutex>
 #include <new>
+#include <unordered_map>
 #include <vector>
 
 #include "../../include/wino.h"
@@ -29,10 +32,6 @@ struct wino_plan_s {
     int host_dev = -1;
     cudaStream_t copy_in = nullptr, copy_out = nullptr;
     std::vector<cudaEvent_t> host_events;
-    // chunk layout of the last pipelined host call (workspace, chunks, images per chunk, bytes per
-    // image in and out): a call with the same layout orders each chunk's input copy only after the
-    // previous call's compute of that chunk, so it overlaps the previous call's tail
-    size_t host_sig[5] = {0, 0, 0, 0, 0};
 };
 
 namespace {
@@ -42,6 +41,12 @@ using namespace wino;
 constexpr size_t kAlign = 256;
 size_t up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
+// Guard bands (WINO_DEBUG_GUARDS): kGuardBytes of kGuardByte before every workspace region and
+// after the last one, written at the start of each call and checked by wino_check_guards.
+constexpr size_t kGuardBytes = 4096;
+constexpr unsigned char kGuardByte = 0xA5;
+constexpr int kMaxGuards = 12;
+
 struct Layout {
     int TH = 0, TW = 0, n2 = 0, ng = 0, ngo = 0;
     long T = 0, T_pad = 0;
@@ -49,6 +54,8 @@ struct Layout {
     bool dbg_yq = false, dbg_acc = false, ytap = false, xq = false, swap = false;
     size_t off_xq = 0, off_vq = 0, off_sv = 0, off_amax = 0, off_yq = 0, off_y32 = 0, off_sy = 0, off_acc = 0, off_err = 0;
     size_t total = 0;
+    int n_guards = 0;
+    size_t guard[kMaxGuards] = {};
 };
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -107,35 +114,51 @@ Layout make_layout(const wino_plan_s* p, int N, int H, int W, int Cin, int Cout)
     L.dbg_yq = (p->opts.debug & WINO_DEBUG_YQ) != 0;
     L.dbg_acc = (p->opts.debug & WINO_DEBUG_ACC32) != 0;
     L.xq = p->opts.x_int8 != 0;
+    const bool guards = (p->opts.debug & WINO_DEBUG_GUARDS) != 0;
     size_t off = 0;
+    auto guard = [&]() {
+        if (!guards) return;
+        L.guard[L.n_guards++] = off;
+        off += kGuardBytes;
+    };
     if (L.xq) {  // fp32 copy of x after its group-wise int8 round trip
+        guard();
         L.off_xq = off;
         off = up(off + sizeof(float) * (size_t)N * H * W * Cin, kAlign);
     }
+    guard();
     L.off_vq = off;
     off = up(off + (size_t)L.T_pad * L.n2 * Cin, kAlign);
+    guard();
     L.off_sv = off;
     off = up(off + sizeof(float) * (size_t)L.n2 * L.ng * L.T_pad, kAlign);
+    guard();
     L.off_amax = off;
     off = up(off + sizeof(unsigned) * (size_t)L.T_pad * L.ngo, kAlign);
     if (L.y_path == WINO_YPATH_RECOMPUTE || L.dbg_yq) {
+        guard();
         L.off_yq = off;
         off = up(off + (size_t)L.T * L.n2 * Cout, kAlign);
     }
     if (L.y_path == WINO_YPATH_Y32) {
+        guard();
         L.off_y32 = off;
         off = up(off + sizeof(float) * (size_t)L.T * L.n2 * Cout, kAlign);
     }
     if (L.dbg_yq) {
+        guard();
         L.off_sy = off;
         off = up(off + sizeof(float) * (size_t)L.T * (L.ytap ? L.n2 : 1) * L.ngo, kAlign);
     }
     if (L.dbg_acc) {
+        guard();
         L.off_acc = off;
         off = up(off + sizeof(int) * (size_t)L.n2 * L.T * Cout * L.ng, kAlign);
     }
+    guard();
     L.off_err = off;
     off = up(off + 16, kAlign);
+    guard();
     L.total = off;
     return L;
 }
@@ -147,6 +170,32 @@ int cuda_status(wino_plan_s* p, cudaError_t e) {
 }
 
 constexpr int kMaxHostChunks = 3;
+
+// The last call on each workspace, when it was a pipelined host call: its plan and its chunk
+// layout (workspace, chunks, images per chunk, bytes per image in and out).  A host call whose
+// workspace was last used by the same plan with the same layout orders each chunk's input copy
+// only after that call's compute of the chunk, so it overlaps that call's tail.  Any other call on
+// the workspace (another plan, another layout, the device-buffer entry point, whose workspace may
+// reach into the staging area) ends the chain, and so does destroying the plan.
+struct HostChain {
+    const wino_plan_s* plan;
+    size_t sig[5];
+};
+std::mutex g_chain_mutex;
+std::unordered_map<const void*, HostChain> g_chain;
+
+void chain_forget_workspace(const void* ws) {
+    std::lock_guard<std::mutex> lock(g_chain_mutex);
+    g_chain.erase(ws);
+}
+
+void chain_forget_plan(const wino_plan_s* p) {
+    std::lock_guard<std::mutex> lock(g_chain_mutex);
+    for (auto it = g_chain.begin(); it != g_chain.end();) {
+        if (it->second.plan == p) it = g_chain.erase(it);
+        else ++it;
+    }
+}
 
 // The host entry point's copy streams and events, created on the current device.
 int ensure_host_streams(wino_plan_s* p) {
@@ -211,12 +260,24 @@ int run_conv(wino_plan_s* p, const void* x, int x_dtype, int N, int H, int W, in
     const float* sU = reinterpret_cast<const float*>(static_cast<const unsigned char*>(wt) +
                                                      up((size_t)L.n2 * Cout * Cin, kAlign));
 
+    // The error word starts each call at zero.  It is cleared on the stream before the first kernel
+    // (not inside a kernel, where the clearing CTA could run after another CTA recorded a timeout).
+    cudaError_t e = cudaMemsetAsync(err, 0, sizeof(int), st);
+    if (e != cudaSuccess) return cuda_status(p, e);
+    for (int gi = 0; gi < L.n_guards; ++gi)
+        if ((e = cudaMemsetAsync(base + L.guard[gi], kGuardByte, kGuardBytes, st)) != cudaSuccess)
+            return cuda_status(p, e);
+    // element counts for the debug build's index checks (one less each under the checks' test hook)
+    const size_t sh = (p->opts.debug & WINO_DEBUG_SHRINK_BOUNDS) ? 1 : 0;
+    const size_t n_amax = (size_t)L.T_pad * L.ngo - sh, n_y = (size_t)L.T * L.n2 * Cout - sh;
     int slot = 0;
     bool x_bf16 = x_dtype == WINO_BF16;
     if (L.xq) {
         float* xq = reinterpret_cast<float*>(base + L.off_xq);
         prof_mark(p, slot++, st);
-        cudaError_t e = launch_input_quant(x, x_bf16, (long)N * H * W * Cin, p->G, xq, num_sms(), st);
+        nvtxRangePushA("wino: x quantisation");
+        e = launch_input_quant(x, x_bf16, (long)N * H * W * Cin, p->G, xq, num_sms(), st);
+        nvtxRangePop();
         if (e != cudaSuccess) return cuda_status(p, e);
         x = xq;
         x_bf16 = false;
@@ -238,8 +299,13 @@ int run_conv(wino_plan_s* p, const void* x, int x_dtype, int N, int H, int W, in
     ia.amax = amax;
     ia.err = err;
     ia.num_sms = num_sms();
+    ia.n_vq = (size_t)L.T_pad * L.n2 * Cin - sh;
+    ia.n_sv = (size_t)L.n2 * L.ng * L.T_pad - sh;
+    ia.n_amax = n_amax;
     prof_mark(p, slot++, st);
-    cudaError_t e = launch_input_transform(ia, p->tf, p->mat.m, p->bt_masked, x_bf16, st);
+    nvtxRangePushA("wino: input transform");
+    e = launch_input_transform(ia, p->tf, p->mat.m, p->bt_masked, x_bf16, st);
+    nvtxRangePop();
     if (e != cudaSuccess) return cuda_status(p, e);
 
     GemmArgs ga;
@@ -261,10 +327,20 @@ int run_conv(wino_plan_s* p, const void* x, int x_dtype, int N, int H, int W, in
     ga.err = err;
     ga.force_timeout = (p->opts.debug & WINO_DEBUG_FORCE_TIMEOUT) != 0 && L.gemm == WINO_GEMM_TCGEN05;
     ga.swap_ab = L.swap ? 1 : 0;
+    ga.n_v = (size_t)L.T_pad * L.n2 * Cin - sh;
+    ga.n_u = (size_t)L.n2 * Cout * Cin - sh;
+    ga.n_amax = n_amax;
+    ga.n_y = n_y;
+    ga.n_acc = (size_t)L.n2 * L.T * Cout * L.ng - sh;
     auto gemm = [&](int mode) -> cudaError_t {
         prof_mark(p, slot++, st);
-        if (L.gemm == WINO_GEMM_SIMT) return launch_hadamard_simt(ga, Vq, Uq, mode, st);
-        return launch_hadamard_tc(ga, Vq, Uq, mode, num_sms(), st, nullptr);
+        nvtxRangePushA(mode == kModeAbsmax ? "wino: hadamard absmax pass"
+                                           : (mode == kModeQuant ? "wino: hadamard quantising pass"
+                                                                 : "wino: hadamard fp32-Y pass"));
+        const cudaError_t ge = L.gemm == WINO_GEMM_SIMT ? launch_hadamard_simt(ga, Vq, Uq, mode, st)
+                                                        : launch_hadamard_tc(ga, Vq, Uq, mode, num_sms(), st, nullptr);
+        nvtxRangePop();
+        return ge;
     };
     if (L.y_path == WINO_YPATH_RECOMPUTE) {
         if ((e = gemm(kModeAbsmax)) != cudaSuccess) return cuda_status(p, e);
@@ -294,9 +370,15 @@ int run_conv(wino_plan_s* p, const void* x, int x_dtype, int N, int H, int W, in
     oa.ytap = L.ytap ? 1 : 0;
     oa.err = err;
     oa.num_sms = num_sms();
+    oa.n_y = n_y;
+    oa.n_out = (size_t)N * H * W * Cout - sh;
+    oa.n_amax = n_amax;
+    oa.n_sy = (size_t)L.T * (L.ytap ? L.n2 : 1) * L.ngo - sh;
     prof_mark(p, slot++, st);
+    nvtxRangePushA("wino: output transform");
     e = launch_output_transform(oa, p->tf, p->mat.m, p->at_masked, L.y_path == WINO_YPATH_Y32, y_dtype == WINO_BF16,
                                 st);
+    nvtxRangePop();
     prof_mark(p, slot, st);
     if (p->prof_calls < p->prof_max_calls) {
         p->prof_launches = slot;
@@ -317,6 +399,8 @@ const char* wino_status_string(int s) {
         case WINO_ERR_WORKSPACE: return "workspace or weight buffer too small";
         case WINO_ERR_CUDA: return "CUDA error";
         case WINO_ERR_DEVICE_TIMEOUT: return "bounded device wait expired";
+        case WINO_ERR_DEVICE_BOUNDS: return "index check failed in a kernel (debug build); the access was skipped";
+        case WINO_ERR_GUARD: return "a workspace guard band was overwritten";
         case WINO_ERR_NOT_EXACT: return "transform not exactly representable";
         default: return "unknown status";
     }
@@ -369,6 +453,7 @@ int wino_plan(wino_plan_t* out, int m, const double* points, const float* S_B, c
 
 int wino_plan_destroy(wino_plan_t p) {
     if (p) {
+        chain_forget_plan(p);
         for (cudaEvent_t ev : p->prof_events) cudaEventDestroy(ev);
         for (cudaEvent_t ev : p->host_events) cudaEventDestroy(ev);
         if (p->copy_in) cudaStreamDestroy(p->copy_in);
@@ -420,6 +505,7 @@ size_t wino_workspace_bytes(wino_plan_t p, int N, int H, int W, int Cin, int Cou
 int wino_conv2d_int8(wino_plan_t p, const void* x, int x_dtype, int N, int H, int W, int Cin, const void* wt,
                       int Cout, void* y, int y_dtype, void* ws, size_t ws_bytes, void* stream) {
     if (!p) return WINO_ERR_INVALID_ARG;
+    chain_forget_workspace(ws);
     return run_conv(p, x, x_dtype, N, H, W, Cin, wt, Cout, y, y_dtype, ws, ws_bytes,
                     static_cast<cudaStream_t>(stream));
 }
@@ -442,9 +528,15 @@ int wino_conv2d_int8_host(wino_plan_t p, const void* x_host, int x_dtype, int N,
     if (ws_bytes < need + stage) return WINO_ERR_WORKSPACE;
     const size_t xs = x_dtype == WINO_BF16 ? 2 : 4, ys = y_dtype == WINO_BF16 ? 2 : 4;
     const size_t xrow = xs * H * W * Cin, yrow = ys * H * W * Cout;   // bytes per image
-    size_t prev_sig[5];
-    std::memcpy(prev_sig, p->host_sig, sizeof(prev_sig));
-    std::memset(p->host_sig, 0, sizeof(p->host_sig));   // set again only when this call is fully enqueued
+    HostChain prev = {nullptr, {0, 0, 0, 0, 0}};
+    {   // taken out now, set again only when this call is fully enqueued
+        std::lock_guard<std::mutex> lock(g_chain_mutex);
+        auto it = g_chain.find(ws);
+        if (it != g_chain.end()) {
+            prev = it->second;
+            g_chain.erase(it);
+        }
+    }
     unsigned char* xd = static_cast<unsigned char*>(ws) + need;
     unsigned char* yd = xd + up(xrow * N, kAlign);
     cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -453,11 +545,15 @@ int wino_conv2d_int8_host(wino_plan_t p, const void* x_host, int x_dtype, int N,
     // Chunks of images: every tile, and so every result, belongs to one image, so the
     // chunks give the same bytes as one call.  Two chunk workspaces must fit below the
     // whole call's error word (which collects the chunks' errors).
+    // A chunk's workspace must hold the layout of every chunk size used (the full chunks and the
+    // last, smaller one): a smaller chunk can resolve to the fp32-Y path and need more bytes.
     int K = std::min(N, kMaxHostChunks), Nc = N;
     size_t need_c = need;
     for (; K > 1; --K) {
         Nc = (N + K - 1) / K;
-        need_c = up(make_layout(p, Nc, H, W, Cin, Cout).total, kAlign);
+        const int last = N - ((N + Nc - 1) / Nc - 1) * Nc;
+        need_c = up(std::max(make_layout(p, Nc, H, W, Cin, Cout).total, make_layout(p, last, H, W, Cin, Cout).total),
+                    kAlign);
         if (2 * need_c <= L.off_err) break;
     }
     if (K <= 1) {
@@ -476,7 +572,7 @@ int wino_conv2d_int8_host(wino_plan_t p, const void* x_host, int x_dtype, int N,
     // of the same layout, chunk k's input copy waits for that call's compute of chunk k (the
     // last reader of its staging slice); otherwise every copy waits for the stream's prior work.
     const size_t sig[5] = {reinterpret_cast<size_t>(ws), (size_t)K, (size_t)Nc, xrow, yrow};
-    const bool chained = std::memcmp(sig, prev_sig, sizeof(sig)) == 0;
+    const bool chained = prev.plan == p && std::memcmp(sig, prev.sig, sizeof(sig)) == 0;
     if (!chained) {
         cudaEventRecord(ev[0], st);
         cudaStreamWaitEvent(p->copy_in, ev[0], 0);
@@ -505,7 +601,12 @@ int wino_conv2d_int8_host(wino_plan_t p, const void* x_host, int x_dtype, int N,
             return cuda_status(p, e);
         cudaEventRecord(ev[3 + 3 * k], p->copy_out);
     }
-    std::memcpy(p->host_sig, sig, sizeof(sig));
+    {
+        std::lock_guard<std::mutex> lock(g_chain_mutex);
+        HostChain& c = g_chain[ws];
+        c.plan = p;
+        std::memcpy(c.sig, sig, sizeof(sig));
+    }
     return cuda_status(p, cudaStreamWaitEvent(st, ev[3 * K], 0));
 }
 
@@ -519,7 +620,32 @@ int wino_check_device_error(wino_plan_t p, const void* ws, int N, int H, int W, 
     int v = 0;
     e = cudaMemcpy(&v, static_cast<const unsigned char*>(ws) + L.off_err, sizeof(int), cudaMemcpyDeviceToHost);
     if (e != cudaSuccess) return cuda_status(p, e);
-    return v ? WINO_ERR_DEVICE_TIMEOUT : WINO_OK;
+    if (v == 0) return WINO_OK;
+    return v == kDevErrBounds ? WINO_ERR_DEVICE_BOUNDS : WINO_ERR_DEVICE_TIMEOUT;
+}
+
+int wino_check_guards(wino_plan_t p, const void* ws, int N, int H, int W, int Cin, int Cout, void* stream,
+                      int* bad_guard) {
+    int rc = check_shape(p, N, H, W, Cin, Cout);
+    if (rc) return rc;
+    if (!ws) return WINO_ERR_INVALID_ARG;
+    if (bad_guard) *bad_guard = -1;
+    const Layout L = make_layout(p, N, H, W, Cin, Cout);
+    if (L.n_guards == 0) return WINO_ERR_UNSUPPORTED;
+    cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_status(p, e);
+    std::vector<unsigned char> g(kGuardBytes);
+    for (int i = 0; i < L.n_guards; ++i) {
+        e = cudaMemcpy(g.data(), static_cast<const unsigned char*>(ws) + L.guard[i], kGuardBytes,
+                       cudaMemcpyDeviceToHost);
+        if (e != cudaSuccess) return cuda_status(p, e);
+        for (unsigned char b : g)
+            if (b != kGuardByte) {
+                if (bad_guard) *bad_guard = i;
+                return WINO_ERR_GUARD;
+            }
+    }
+    return WINO_OK;
 }
 
 int wino_debug_dump(wino_plan_t p, const void* ws, int N, int H, int W, int Cin, int Cout, int what, void* dst,

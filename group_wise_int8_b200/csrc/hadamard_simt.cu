@@ -20,6 +20,8 @@ __global__ void __launch_bounds__(256) hadamard_simt_kernel(GemmArgs p, const in
     const long t = i / p.Cout;
     const int co = (int)(i - t * p.Cout);
     if (t >= p.T) return;  // Cout % 32 == 0: uniform per warp
+    const size_t vrow = ((size_t)tap * p.T_pad + t) * p.Cin, urow = ((size_t)tap * p.Cout + co) * p.Cin;
+    if (!in_bounds(vrow + p.Cin - 1, p.n_v, p.err) || !in_bounds(urow + p.Cin - 1, p.n_u, p.err)) return;
     const int4* v = reinterpret_cast<const int4*>(Vq + ((size_t)tap * p.T_pad + t) * p.Cin);
     const int4* u = reinterpret_cast<const int4*>(Uq + ((size_t)tap * p.Cout + co) * p.Cin);
     float y = 0.0f;
@@ -32,12 +34,15 @@ __global__ void __launch_bounds__(256) hadamard_simt_kernel(GemmArgs p, const in
             acc = __dp4a(a.z, b.z, acc);
             acc = __dp4a(a.w, b.w, acc);
         }
-        if (DUMP) p.acc[(((size_t)tap * p.T + t) * p.Cout + co) * p.ng + j] = acc;
+        const size_t di = (((size_t)tap * p.T + t) * p.Cout + co) * p.ng + j;
+        if (DUMP && in_bounds(di, p.n_acc, p.err)) p.acc[di] = acc;
         const float pr = __fmul_rn(p.sV[((size_t)tap * p.ng + j) * p.T_pad + t], p.sU[((size_t)tap * p.ng + j) * p.Cout + co]);
         y = __fmaf_rn((float)acc, pr, y);
     }
     const size_t o = ((size_t)tap * p.T + t) * p.Cout + co;
-    unsigned* am = p.amax + (size_t)t * p.ngo + co / p.G;
+    const size_t ai = (size_t)t * p.ngo + co / p.G;
+    if (!in_bounds(o, p.n_y, p.err) || !in_bounds(ai, p.n_amax, p.err)) return;
+    unsigned* am = p.amax + ai;
     if (MODE == kModeQuant) {
         p.Yq[o] = (int8_t)quant_code(y, group_scale(__uint_as_float(*am)));
     } else {

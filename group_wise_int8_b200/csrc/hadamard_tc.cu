@@ -168,10 +168,12 @@ __device__ __forceinline__ void publish_amax(const GemmArgs& p, int row, int lan
 #pragma unroll
                 for (int off = 16; off > 0; off >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, off));
                 const int tt = colg[h] + c;
-                if (lane == 0 && tt < p.T) atomicMax(&p.amax[(size_t)tt * p.ngo + grp], __float_as_uint(v));
+                const size_t ai = (size_t)tt * p.ngo + grp;
+                if (lane == 0 && tt < p.T && in_bounds(ai, p.n_amax, p.err)) atomicMax(&p.amax[ai], __float_as_uint(v));
             }
         } else {
-            atomicMax(&p.amax[(size_t)row * p.ngo + cgrp[h]], __float_as_uint(gmax[h]));
+            const size_t ai = (size_t)row * p.ngo + cgrp[h];
+            if (in_bounds(ai, p.n_amax, p.err)) atomicMax(&p.amax[ai], __float_as_uint(gmax[h]));
         }
     }
 }
@@ -384,8 +386,9 @@ __global__ void __launch_bounds__(TcCfg<BN>::kThreads, 1)
                     gmax[h] = 0.0f;
 #pragma unroll
                     for (int c = 0; c < CPT; ++c) gcol[h][c] = 0.0f;
-                    if (MODE == kModeQuant && valid)
-                        qy[h] = make_qscale(__uint_as_float(p.amax[(size_t)row * p.ngo + cgrp[h]]));
+                    const size_t ai = (size_t)row * p.ngo + cgrp[h];
+                    if (MODE == kModeQuant && valid && in_bounds(ai, p.n_amax, p.err))
+                        qy[h] = make_qscale(__uint_as_float(p.amax[ai]));
                 }
             }
             for (int ks = 0; ok && ks < KSTAGES; ++ks) {
@@ -443,10 +446,11 @@ __global__ void __launch_bounds__(TcCfg<BN>::kThreads, 1)
 #pragma unroll
                                 for (int c = 0; c < CPT; ++c) {
                                     if (SWAP) {   // row = output channel, column = tile
-                                        if (colg[h] + c < p.T)
-                                            p.acc[(((size_t)tap * p.T + colg[h] + c) * p.Cout + row) * p.ng + jg] = (int)r[h][c];
+                                        const size_t di = (((size_t)tap * p.T + colg[h] + c) * p.Cout + row) * p.ng + jg;
+                                        if (colg[h] + c < p.T && in_bounds(di, p.n_acc, p.err)) p.acc[di] = (int)r[h][c];
                                     } else {
-                                        p.acc[(((size_t)tap * p.T + row) * p.Cout + colg[h] + c) * p.ng + jg] = (int)r[h][c];
+                                        const size_t di = (((size_t)tap * p.T + row) * p.Cout + colg[h] + c) * p.ng + jg;
+                                        if (in_bounds(di, p.n_acc, p.err)) p.acc[di] = (int)r[h][c];
                                     }
                                 }
                             }
@@ -461,10 +465,11 @@ __global__ void __launch_bounds__(TcCfg<BN>::kThreads, 1)
 #pragma unroll
                         for (int c = 0; c < CPT / 2; ++c) f2_unpack(y2[h][c], y[2 * c], y[2 * c + 1]);
                         if (MODE == kModeQuant) {
-                            if (valid) {
+                            const size_t yi = ((size_t)tap * p.T + row) * p.Cout + colg[h];
+                            if (valid && in_bounds(yi + CPT - 1, p.n_y, p.err)) {
                                 uint32_t q[CPT / 4];
                                 quant_chunk<CPT>(y, qy[h], q);
-                                int8_t* dst = p.Yq + ((size_t)tap * p.T + row) * p.Cout + colg[h];
+                                int8_t* dst = p.Yq + yi;
                                 if (CPT == 8) {
                                     *reinterpret_cast<uint2*>(dst) = make_uint2(q[0], q[1 % (CPT / 4)]);
                                 } else {
@@ -481,13 +486,15 @@ __global__ void __launch_bounds__(TcCfg<BN>::kThreads, 1)
                             for (int c = 0; c < CPT; ++c) {
                                 const int tt = colg[h] + c;
                                 gcol[h][c] = fmaxf(gcol[h][c], fabsf(y[c]));
-                                if (tt < p.T) p.Y32[((size_t)tap * p.T + tt) * p.Cout + row] = y[c];
+                                const size_t yi = ((size_t)tap * p.T + tt) * p.Cout + row;
+                                if (tt < p.T && in_bounds(yi, p.n_y, p.err)) p.Y32[yi] = y[c];
                             }
                         } else {
 #pragma unroll
                             for (int c = 0; c < CPT; c += 2) gmax[h] = max_abs3(gmax[h], y[c], y[c + 1]);
-                            if (MODE == kModeY32 && valid) {
-                                float* dst = p.Y32 + ((size_t)tap * p.T + row) * p.Cout + colg[h];
+                            const size_t yi = ((size_t)tap * p.T + row) * p.Cout + colg[h];
+                            if (MODE == kModeY32 && valid && in_bounds(yi + CPT - 1, p.n_y, p.err)) {
+                                float* dst = p.Y32 + yi;
 #pragma unroll
                                 for (int c = 0; c < CPT; c += 4)
                                     *reinterpret_cast<float4*>(dst + c) = make_float4(y[c], y[c + 1], y[c + 2], y[c + 3]);

@@ -53,7 +53,7 @@ __global__ void __launch_bounds__(256) input_quant_kernel(const Tin* __restrict_
         const long e = base + 8 * lane;
         // elems is a multiple of G (and G of 8): a group, hence a lane's 8 values, lies wholly in
         // range or wholly out; lanes past the end take part in the shuffles with zeros
-        const bool live = e < elems;
+        const bool live = e < elems && in_bounds(e + 7, elems, nullptr);
         float v[8];
         if (live) {
             load8<Tin>(x + e, v);

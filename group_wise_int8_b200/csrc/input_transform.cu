@@ -112,7 +112,8 @@ __device__ __forceinline__ void quant_batch(const float* vw, int lane, int warp,
         if (!own || ctl >= TX || tx >= p.TW) continue;
         const long t = (long)row_id * p.TW + tx;
         const QScale q = make_qscale(am);
-        if (ch == 0) p.sV[((size_t)tap * (p.Cin / G) + g) * p.T_pad + t] = q.s;
+        const size_t si = ((size_t)tap * (p.Cin / G) + g) * p.T_pad + t;
+        if (ch == 0 && in_bounds(si, p.n_sv, p.err)) p.sV[si] = q.s;
         uint32_t w[8];
 #pragma unroll
         for (int hh = 0; hh < 2; ++hh) {   // two 16-value halves of the chunk, one exactness check each
@@ -130,7 +131,9 @@ __device__ __forceinline__ void quant_batch(const float* vw, int lane, int warp,
 #pragma unroll
             for (int j = 0; j < 4; ++j) w[4 * hh + j] = wh[j];
         }
-        uint4* dst = reinterpret_cast<uint4*>(p.Vq + ((size_t)tap * p.T_pad + t) * p.Cin + g * G + ch);
+        const size_t vi = ((size_t)tap * p.T_pad + t) * p.Cin + g * G + ch;
+        if (!in_bounds(vi + 31, p.n_vq, p.err)) continue;
+        uint4* dst = reinterpret_cast<uint4*>(p.Vq + vi);
         dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
         dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
     }
@@ -165,11 +168,11 @@ __global__ void __maxnreg__(MASK == kMaskAll ? 255 : 128)
         sm100::mbar_arrive_expect_tx(&bar, (uint32_t)Cfg::patch_bytes(TX));
         sm100::tma_load_4d(smem, &tmX, &bar, g * G, tx0 * M - 1, ty * M - 1, img);
     }
-    if (blockIdx.x == 0 && blockIdx.y == 0 && g == 0 && tid == 0) *p.err = 0;
     if (g == 0)
         for (int i = tid; i < TX * p.ngo; i += blockDim.x) {
             const int tt = i / p.ngo, k = i - tt * p.ngo;
-            if (tx0 + tt < p.TW) p.amax[((size_t)row_id * p.TW + tx0 + tt) * p.ngo + k] = 0u;
+            const size_t ai = ((size_t)row_id * p.TW + tx0 + tt) * p.ngo + k;
+            if (tx0 + tt < p.TW && in_bounds(ai, p.n_amax, p.err)) p.amax[ai] = 0u;
         }
     if (tid == 0) {
         load_ok = 1;
@@ -320,11 +323,11 @@ __global__ void __launch_bounds__(InSplitCfg<M, Tin, G>::kMaxThreads)
         sm100::mbar_arrive_expect_tx(&bar, (uint32_t)Cfg::patch_bytes(TX));
         sm100::tma_load_4d(smem, &tmX, &bar, g * G, tx0 * M - 1, ty * M - 1, img);
     }
-    if (blockIdx.x == 0 && blockIdx.y == 0 && g == 0 && tid == 0) *p.err = 0;
     if (g == 0)
         for (int i = tid; i < TX * p.ngo; i += blockDim.x) {
             const int tt = i / p.ngo, k = i - tt * p.ngo;
-            if (tx0 + tt < p.TW) p.amax[((size_t)row_id * p.TW + tx0 + tt) * p.ngo + k] = 0u;
+            const size_t ai = ((size_t)row_id * p.TW + tx0 + tt) * p.ngo + k;
+            if (tx0 + tt < p.TW && in_bounds(ai, p.n_amax, p.err)) p.amax[ai] = 0u;
         }
     if (tid == 0) {
         load_ok = 1;

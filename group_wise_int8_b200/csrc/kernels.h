@@ -56,8 +56,9 @@ struct InputArgs {
     int8_t* Vq;      // [n*n][T_pad][Cin] (tap-major)
     float* sV;       // [n*n][Cin/G][T_pad]
     unsigned* amax;  // [T_pad][Cout/G], cleared here
-    int* err;        // device error word, cleared here
+    int* err;        // device error word (cleared on the stream before the call's first kernel)
     int num_sms;     // SMs of the device (sizes the choice of the split kernel)
+    size_t n_vq, n_sv, n_amax;   // element counts of Vq, sV, amax (index checks of the debug build)
 };
 cudaError_t launch_input_transform(const InputArgs& a, const TransformArgs& tf, int m, bool masked, bool bf16_in,
                                    cudaStream_t st);
@@ -86,6 +87,8 @@ struct GemmArgs {
     int force_timeout; // test hook: the MMA thread first waits 1 ms on a barrier nothing completes
     int swap_ab;       // fp32-Y mode, T <= 32, Cout % 128 == 0: the MMA rows are 128 output channels
                        // (A = Uq) and its columns the tiles (B = Vq), so no TMEM lane is padding
+    size_t n_v, n_u, n_amax, n_y, n_acc;   // element counts of Vq (and sV), Uq (and sU), amax, Yq/Y32 and acc
+                                           // (index checks of the debug build)
 };
 
 // Tensor maps and launch of the tcgen05 kernel; `Vq` is [n2][T_pad][Cin], `Uq` [n2][Cout][Cin].
@@ -110,6 +113,7 @@ struct OutputArgs {
     int ytap;              // per-tap Y groups (Y32 source; sY_dbg is then [T][n2][ngo])
     int* err;              // device error word (bounded waits)
     int num_sms;           // SMs of the device (sizes the choice of the split kernel)
+    size_t n_y, n_out, n_amax, n_sy;   // element counts of Yq/Y32, out, amax, sY (debug-build index checks)
 };
 cudaError_t launch_output_transform(const OutputArgs& a, const TransformArgs& tf, int m, bool masked, bool src_y32,
                                     bool bf16_out, cudaStream_t st);

@@ -18,7 +18,9 @@
 // All calls share the one array and it keeps whatever the previous call left
 // there.  The convolution itself clears everything that must start at zero
 // (the Y absmax table and the device error word) at the start of each call, so
-// leftover contents never change a result.  Two calls whose kernels overlap
+// leftover contents never change a result.  The error word of the last call
+// lives in the array too: wino_check_device_error_noalloc reads it (after that
+// call and before the next one, which clears it).  Two calls whose kernels overlap
 // on the GPU (different streams, or different host threads without ordering)
 // race on the array and corrupt each other's intermediates: serialise them.
 #include <cuda_runtime.h>
@@ -66,4 +68,16 @@ extern "C" int wino_conv2d_int8_noalloc(wino_plan_t plan, const void* x_dev, int
     if (rc != WINO_OK) return rc;
     return wino_conv2d_int8(plan, x_dev, x_dtype, N, H, W, Cin, wt_dev, Cout, y_dev, y_dtype, scratch,
                             kNoAllocScratchBytes, stream);
+}
+
+extern "C" int wino_check_device_error_noalloc(wino_plan_t plan, int N, int H, int W, int Cin, int Cout,
+                                               void* stream) {
+    if (!plan) return WINO_ERR_INVALID_ARG;
+    const size_t need = wino_workspace_bytes(plan, N, H, W, Cin, Cout);
+    if (need == 0) return WINO_ERR_INVALID_ARG;
+    if (need > kNoAllocScratchBytes) return WINO_ERR_WORKSPACE;
+    void* scratch = nullptr;
+    const int rc = scratch_address(&scratch);
+    if (rc != WINO_OK) return rc;
+    return wino_check_device_error(plan, scratch, N, H, W, Cin, Cout, stream);
 }

@@ -71,12 +71,17 @@ __global__ void __launch_bounds__(128, SRC_Y32 ? 6 : 4)
     const int co = 2 * (int)(i - t * cpairs);
     if (t >= p.T) return;
     const int cg = co / p.G;
+    const size_t base = (size_t)t * p.Cout + co;   // Yq / Y32 are tap-major [n2][T][Cout]
+    const size_t tstride = (size_t)p.T * p.Cout;
+    // every Y element this thread touches lies in [base, base + (N2 - 1) * tstride + 1]
+    if (!in_bounds((size_t)t * p.ngo + cg, p.n_amax, p.err) ||
+        ((SRC_Y32 || DEBUG) && !in_bounds(base + (size_t)(N2 - 1) * tstride + 1, p.n_y, p.err)) ||
+        (DEBUG && !in_bounds((size_t)t * p.ngo + cg, p.n_sy, p.err)))
+        return;
     const QScale qs = make_qscale(__uint_as_float(p.amax[(size_t)t * p.ngo + cg]));
     if (DEBUG && co % p.G == 0) p.sY_dbg[(size_t)t * p.ngo + cg] = qs.s;
     const uint64_t s2 = f2_pack(qs.s, qs.s);
 
-    const size_t base = (size_t)t * p.Cout + co;   // Yq / Y32 are tap-major [n2][T][Cout]
-    const size_t tstride = (size_t)p.T * p.Cout;
     uint64_t Z[M][N];                              // (co, co + 1) pairs
 #pragma unroll
     for (int nu = 0; nu < N; ++nu) {
@@ -131,6 +136,7 @@ __global__ void __launch_bounds__(128, SRC_Y32 ? 6 : 4)
             float o0, o1;
             f2_unpack(acc, o0, o1);
             const size_t o = (((size_t)img * p.H + yy) * p.W + xx) * p.Cout + co;
+            if (!in_bounds(o + 1, p.n_out, p.err)) continue;
             if (BF16_OUT)
                 *reinterpret_cast<__nv_bfloat162*>(reinterpret_cast<__nv_bfloat16*>(p.out) + o) =
                     __floats2bfloat162_rn(o0, o1);
@@ -158,7 +164,10 @@ __global__ void __launch_bounds__(128, 6) output_transform_ytap_kernel(OutputArg
     const int cpairs = p.Cout >> 1;
     const long t = i / cpairs;
     const int co = 2 * (int)(i - t * cpairs);
-    const bool live = t < p.T;           // a CTA covers whole groups; dead threads still join the reductions
+    // a CTA covers whole groups; dead threads (and, in the debug build, threads whose Y range fails
+    // its index check) still join the reductions with zeros
+    const bool live = t < p.T && in_bounds(((size_t)t * p.Cout + co) + (size_t)(N2 - 1) * p.T * p.Cout + 1,
+                                           p.n_y, p.err);
     const int G = p.G;
     const int cg = co / G;
     const size_t base = (size_t)(live ? t : 0) * p.Cout + co;
@@ -191,7 +200,8 @@ __global__ void __launch_bounds__(128, 6) output_transform_ytap_kernel(OutputArg
         // each lane of the segment derives the scales of every seg_w-th tap
         for (int tap = sl; tap < N2; tap += seg_w) {
             qsm[warp][seg][tap] = make_qscale(red[warp][seg][tap]);
-            if (p.sY_dbg && live) p.sY_dbg[((size_t)t * N2 + tap) * p.ngo + cg] = qsm[warp][seg][tap].s;
+            const size_t di = ((size_t)t * N2 + tap) * p.ngo + cg;
+            if (p.sY_dbg && live && in_bounds(di, p.n_sy, p.err)) p.sY_dbg[di] = qsm[warp][seg][tap].s;
         }
         __syncwarp();
     } else {
@@ -205,8 +215,8 @@ __global__ void __launch_bounds__(128, 6) output_transform_ytap_kernel(OutputArg
             qsm[gi][0][tap] = make_qscale(a);
             const long i0 = (long)blockIdx.x * blockDim.x + gi * (G / 2);   // first thread of the group
             const long tg = i0 / cpairs;
-            if (p.sY_dbg && tg < p.T)
-                p.sY_dbg[((size_t)tg * N2 + tap) * p.ngo + (int)(i0 - tg * cpairs) * 2 / G] = qsm[gi][0][tap].s;
+            const size_t di = ((size_t)tg * N2 + tap) * p.ngo + (int)(i0 - tg * cpairs) * 2 / G;
+            if (p.sY_dbg && tg < p.T && in_bounds(di, p.n_sy, p.err)) p.sY_dbg[di] = qsm[gi][0][tap].s;
         }
         __syncthreads();
     }
@@ -256,6 +266,7 @@ __global__ void __launch_bounds__(128, 6) output_transform_ytap_kernel(OutputArg
             float o0, o1;
             f2_unpack(acc, o0, o1);
             const size_t o = (((size_t)img * p.H + yy) * p.W + xx) * p.Cout + co;
+            if (!in_bounds(o + 1, p.n_out, p.err)) continue;
             if (BF16_OUT)
                 *reinterpret_cast<__nv_bfloat162*>(reinterpret_cast<__nv_bfloat16*>(p.out) + o) =
                     __floats2bfloat162_rn(o0, o1);
@@ -283,7 +294,10 @@ __global__ void __launch_bounds__(128) output_transform_split_kernel(OutputArgs 
     const int cpairs = p.Cout >> 1;
     const long t = item / cpairs;
     const int co = 2 * (int)(item - t * cpairs);
-    const bool live = slot < IPW && t < p.T;
+    const bool live = slot < IPW && t < p.T &&
+                      in_bounds((size_t)t * p.ngo + co / p.G, p.n_amax, p.err) &&
+                      in_bounds((size_t)t * p.Cout + co + (size_t)(N * N - 1) * p.T * p.Cout + 1, p.n_y, p.err) &&
+                      (!DEBUG || in_bounds((size_t)t * p.ngo + co / p.G, p.n_sy, p.err));
     if (live) {
         const int cg = co / p.G;
         const QScale qs = make_qscale(__uint_as_float(p.amax[(size_t)t * p.ngo + cg]));
@@ -335,6 +349,7 @@ __global__ void __launch_bounds__(128) output_transform_split_kernel(OutputArgs 
         float o0, o1;
         f2_unpack(acc, o0, o1);
         const size_t o = (((size_t)img * p.H + yy) * p.W + xx) * p.Cout + co;
+        if (!in_bounds(o + 1, p.n_out, p.err)) continue;
         if (BF16_OUT)
             *reinterpret_cast<__nv_bfloat162*>(reinterpret_cast<__nv_bfloat16*>(p.out) + o) =
                 __floats2bfloat162_rn(o0, o1);

@@ -16,6 +16,9 @@ import torch
 
 HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(HERE, "libwino_b200.so")
+# the same library compiled with WINO_DEBUG: index checks in every kernel (see include/wino.h)
+LIB_PATH_DEBUG = os.path.join(HERE, "libwino_b200_debug.so")
+LIB_PATHS = {"release": LIB_PATH, "debug": LIB_PATH_DEBUG}
 
 OK = 0
 ERR_INVALID_ARG = -1
@@ -24,20 +27,24 @@ ERR_WORKSPACE = -3
 ERR_CUDA = -4
 ERR_DEVICE_TIMEOUT = -5
 ERR_NOT_EXACT = -6
+ERR_DEVICE_BOUNDS = -7
+ERR_GUARD = -8
 
 F32 = 0
 BF16 = 1
 
 YPATH_AUTO, YPATH_RECOMPUTE, YPATH_Y32 = 0, 1, 2
 GEMM_AUTO, GEMM_TCGEN05, GEMM_SIMT = 0, 1, 2
-DEBUG_YQ, DEBUG_ACC32, DEBUG_FORCE_TIMEOUT = 1, 2, 4
+DEBUG_YQ, DEBUG_ACC32, DEBUG_FORCE_TIMEOUT, DEBUG_GUARDS, DEBUG_SHRINK_BOUNDS = 1, 2, 4, 8, 16
 YGROUPS_TILE, YGROUPS_TAP = 0, 1
 VARIANT_SWAPPED_GEMM, VARIANT_SPLIT_INPUT, VARIANT_SPLIT_OUTPUT = 1, 2, 4
 DUMP_VQ, DUMP_SV, DUMP_YQ, DUMP_SY, DUMP_Y32, DUMP_ACC32 = range(6)
+NOALLOC_SCRATCH_BYTES = 64 << 20   # WINO_NOALLOC_SCRATCH_BYTES
 
 EXPORTED = [
     "wino_plan", "wino_plan_destroy", "wino_plan_matrices", "wino_plan_info", "wino_weight_bytes",
     "wino_transform_weights", "wino_workspace_bytes", "wino_conv2d_int8", "wino_conv2d_int8_noalloc",
+    "wino_check_device_error_noalloc", "wino_check_guards",
     "wino_host_staging_bytes",
     "wino_conv2d_int8_host", "wino_check_device_error", "wino_debug_dump", "wino_resolved_config",
     "wino_resolved_variants", "wino_launches_per_call", "wino_profile_begin", "wino_profile_end", "wino_last_cuda_error",
@@ -58,17 +65,20 @@ class Opts(ctypes.Structure):
                 ("reserved", ctypes.c_int * 2)]
 
 
-_lib = None
+_libs = {}
+_lib = None   # the release library once loaded
 _vp = ctypes.c_void_p
 _sz = ctypes.c_size_t
 _i = ctypes.c_int
 
 
-def load_library(path: str = LIB_PATH):
-    """Load the CUDA library (raises OSError if it has not been built)."""
+def load_library(path: Optional[str] = None, variant: str = "release"):
+    """Load the CUDA library (raises OSError if it has not been built): the release build, or
+    with variant="debug" the WINO_DEBUG build whose kernels check every index."""
     global _lib
-    if _lib is not None:
-        return _lib
+    path = path or LIB_PATHS[variant]
+    if path in _libs:
+        return _libs[path]
     if not os.path.exists(path):
         raise OSError("CUDA library %s is missing: run `python -m group_wise_int8_b200.build`" % path)
     L = ctypes.CDLL(path)
@@ -85,6 +95,8 @@ def load_library(path: str = LIB_PATH):
     L.wino_workspace_bytes.restype = _sz
     L.wino_conv2d_int8.argtypes = [_vp, _vp, _i, _i, _i, _i, _i, _vp, _i, _vp, _i, _vp, _sz, _vp]
     L.wino_conv2d_int8_noalloc.argtypes = [_vp, _vp, _i, _i, _i, _i, _i, _vp, _i, _vp, _i, _vp]
+    L.wino_check_device_error_noalloc.argtypes = [_vp, _i, _i, _i, _i, _i, _vp]
+    L.wino_check_guards.argtypes = [_vp, _vp, _i, _i, _i, _i, _i, _vp, ctypes.POINTER(_i)]
     L.wino_host_staging_bytes.argtypes = [_vp, _i, _i, _i, _i, _i, _i, _i]
     L.wino_host_staging_bytes.restype = _sz
     L.wino_conv2d_int8_host.argtypes = [_vp, _vp, _i, _i, _i, _i, _i, _vp, _i, _vp, _i, _vp, _sz, _vp]
@@ -100,7 +112,9 @@ def load_library(path: str = LIB_PATH):
     L.wino_status_string.restype = ctypes.c_char_p
     for name in EXPORTED:
         getattr(L, name)  # every declared entry point must resolve
-    _lib = L
+    _libs[path] = L
+    if path == LIB_PATH:
+        _lib = L
     return L
 
 
@@ -134,8 +148,9 @@ class Plan:
 
     def __init__(self, m: int, points: Sequence[float], S_B=None, S_G=None, group: int = 32,
                  y_path: int = YPATH_AUTO, gemm: int = GEMM_AUTO, debug: int = 0, y_groups: int = YGROUPS_TILE,
-                 x_int8: bool = False, int8_transforms: bool = False):
-        L = load_library()
+                 x_int8: bool = False, int8_transforms: bool = False, variant: str = "release"):
+        L = load_library(variant=variant)
+        self._L = L
         n = m + 2
         pts = (ctypes.c_double * n)(*[float(p) for p in points])
         sb = None if S_B is None else (ctypes.c_float * n)(*[float(v) for v in S_B])
@@ -150,13 +165,14 @@ class Plan:
 
     def __del__(self):
         h = getattr(self, "_h", None)
-        if h is not None and _lib is not None:
-            _lib.wino_plan_destroy(h)
+        L = getattr(self, "_L", None)
+        if h is not None and L is not None:
+            L.wino_plan_destroy(h)
             self._h = None
 
     def _check(self, rc: int, what: str):
         if rc != OK:
-            raise WinoError(rc, what, _lib.wino_last_cuda_error(self._h))
+            raise WinoError(rc, what, self._L.wino_last_cuda_error(self._h))
 
     # -------------------------------------------------------------- queries
     def matrices(self):
@@ -164,36 +180,36 @@ class Plan:
         BT = (ctypes.c_float * (n * n))()
         G = (ctypes.c_double * (n * 3))()
         AT = (ctypes.c_float * (m * n))()
-        self._check(_lib.wino_plan_matrices(self._h, BT, G, AT), "wino_plan_matrices")
+        self._check(self._L.wino_plan_matrices(self._h, BT, G, AT), "wino_plan_matrices")
         import numpy as np
         return (np.array(BT, dtype=np.float32).reshape(n, n), np.array(G, dtype=np.float64).reshape(n, 3),
                 np.array(AT, dtype=np.float32).reshape(m, n))
 
     def weight_bytes(self, Cin: int, Cout: int) -> int:
-        return int(_lib.wino_weight_bytes(self._h, Cin, Cout))
+        return int(self._L.wino_weight_bytes(self._h, Cin, Cout))
 
     def workspace_bytes(self, N: int, H: int, W: int, Cin: int, Cout: int) -> int:
-        return int(_lib.wino_workspace_bytes(self._h, N, H, W, Cin, Cout))
+        return int(self._L.wino_workspace_bytes(self._h, N, H, W, Cin, Cout))
 
     def host_staging_bytes(self, N, H, W, Cin, Cout, x_dtype=torch.bfloat16, y_dtype=torch.bfloat16) -> int:
-        return int(_lib.wino_host_staging_bytes(self._h, N, H, W, Cin, Cout, _dtype_code(x_dtype),
+        return int(self._L.wino_host_staging_bytes(self._h, N, H, W, Cin, Cout, _dtype_code(x_dtype),
                                                 _dtype_code(y_dtype)))
 
     def resolved_config(self, N, H, W, Cin, Cout):
         yp, gm = _i(), _i()
-        self._check(_lib.wino_resolved_config(self._h, N, H, W, Cin, Cout, ctypes.byref(yp), ctypes.byref(gm)),
+        self._check(self._L.wino_resolved_config(self._h, N, H, W, Cin, Cout, ctypes.byref(yp), ctypes.byref(gm)),
                     "wino_resolved_config")
         return yp.value, gm.value
 
     def resolved_variants(self, N, H, W, Cin, Cout) -> int:
         """Bit set of VARIANT_* the call of this shape runs (same bytes in every variant)."""
         f = _i()
-        self._check(_lib.wino_resolved_variants(self._h, N, H, W, Cin, Cout, ctypes.byref(f)),
+        self._check(self._L.wino_resolved_variants(self._h, N, H, W, Cin, Cout, ctypes.byref(f)),
                     "wino_resolved_variants")
         return f.value
 
     def launches_per_call(self, N, H, W, Cin, Cout) -> int:
-        return int(_lib.wino_launches_per_call(self._h, N, H, W, Cin, Cout))
+        return int(self._L.wino_launches_per_call(self._h, N, H, W, Cin, Cout))
 
     # ---------------------------------------------------------------- calls
     def transform_weights(self, w: torch.Tensor, out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
@@ -205,7 +221,7 @@ class Plan:
             raise WinoError(ERR_INVALID_ARG, "wino_weight_bytes")
         if out is None:
             out = torch.empty(nbytes, dtype=torch.uint8, device=w.device)
-        self._check(_lib.wino_transform_weights(self._h, w.data_ptr(), Cin, Cout, out.data_ptr(), out.numel(),
+        self._check(self._L.wino_transform_weights(self._h, w.data_ptr(), Cin, Cout, out.data_ptr(), out.numel(),
                                                 _stream_handle(stream)), "wino_transform_weights")
         return out
 
@@ -222,7 +238,7 @@ class Plan:
             raise WinoError(ERR_INVALID_ARG, "wino_workspace_bytes")
         if workspace is None:
             workspace = torch.empty(need, dtype=torch.uint8, device=x.device)
-        self._check(_lib.wino_conv2d_int8(self._h, x.data_ptr(), _dtype_code(x.dtype), N, H, W, Cin, wt.data_ptr(),
+        self._check(self._L.wino_conv2d_int8(self._h, x.data_ptr(), _dtype_code(x.dtype), N, H, W, Cin, wt.data_ptr(),
                                           Cout, out.data_ptr(), _dtype_code(out.dtype), workspace.data_ptr(),
                                           workspace.numel(), _stream_handle(stream)), "wino_conv2d_int8")
         return out
@@ -231,7 +247,7 @@ class Plan:
         """wino_conv2d_int8_noalloc: no workspace argument; the library's fixed
         device scratch array is used instead (see include/wino.h)."""
         N, H, W, Cin = x.shape
-        self._check(_lib.wino_conv2d_int8_noalloc(self._h, x.data_ptr(), _dtype_code(x.dtype), N, H, W, Cin,
+        self._check(self._L.wino_conv2d_int8_noalloc(self._h, x.data_ptr(), _dtype_code(x.dtype), N, H, W, Cin,
                                                   wt.data_ptr(), Cout, out.data_ptr(), _dtype_code(out.dtype),
                                                   _stream_handle(stream)), "wino_conv2d_int8_noalloc")
         return out
@@ -240,24 +256,35 @@ class Plan:
                     workspace: torch.Tensor, stream=None):
         """Host (pinned) input and output; copies happen inside the call, asynchronously."""
         N, H, W, Cin = x_host.shape
-        self._check(_lib.wino_conv2d_int8_host(self._h, x_host.data_ptr(), _dtype_code(x_host.dtype), N, H, W, Cin,
+        self._check(self._L.wino_conv2d_int8_host(self._h, x_host.data_ptr(), _dtype_code(x_host.dtype), N, H, W, Cin,
                                                wt.data_ptr(), Cout, y_host.data_ptr(), _dtype_code(y_host.dtype),
                                                workspace.data_ptr(), workspace.numel(), _stream_handle(stream)),
                     "wino_conv2d_int8_host")
 
     def profile_begin(self, max_calls: int):
         """Record per-kernel CUDA events on the launching stream for the next max_calls calls."""
-        self._check(_lib.wino_profile_begin(self._h, max_calls), "wino_profile_begin")
+        self._check(self._L.wino_profile_begin(self._h, max_calls), "wino_profile_begin")
 
     def profile_end(self):
         """-> (summed ms per launch index, calls recorded)."""
         ms = (ctypes.c_float * 8)()
         nl, nc = _i(), _i()
-        self._check(_lib.wino_profile_end(self._h, ms, 8, ctypes.byref(nl), ctypes.byref(nc)), "wino_profile_end")
+        self._check(self._L.wino_profile_end(self._h, ms, 8, ctypes.byref(nl), ctypes.byref(nc)), "wino_profile_end")
         return [ms[i] for i in range(min(nl.value, 8))], nc.value
 
     def check_device_error(self, workspace: torch.Tensor, N, H, W, Cin, Cout, stream=None) -> int:
-        return _lib.wino_check_device_error(self._h, workspace.data_ptr(), N, H, W, Cin, Cout, _stream_handle(stream))
+        return self._L.wino_check_device_error(self._h, workspace.data_ptr(), N, H, W, Cin, Cout, _stream_handle(stream))
+
+    def check_guards(self, workspace: torch.Tensor, N, H, W, Cin, Cout, stream=None):
+        """(status, index of the first overwritten guard band or -1) after the last conv2d call."""
+        bad = _i()
+        rc = self._L.wino_check_guards(self._h, workspace.data_ptr(), N, H, W, Cin, Cout, _stream_handle(stream),
+                                       ctypes.byref(bad))
+        return rc, bad.value
+
+    def check_device_error_noalloc(self, N, H, W, Cin, Cout, stream=None) -> int:
+        """The device error word of the last conv2d_noalloc call of this shape (in the library's scratch)."""
+        return self._L.wino_check_device_error_noalloc(self._h, N, H, W, Cin, Cout, _stream_handle(stream))
 
     def debug_dump(self, workspace: torch.Tensor, N, H, W, Cin, Cout, what: int):
         """Copy one intermediate tensor of the last call (logical layout, see include/wino.h)."""
@@ -270,6 +297,6 @@ class Plan:
                   DUMP_Y32: ((T, n2, Cout), np.float32), DUMP_ACC32: ((n2, T, Cout, Cin // G), np.int32)}
         shape, dt = shapes[what]
         a = np.zeros(shape, dt)
-        self._check(_lib.wino_debug_dump(self._h, workspace.data_ptr(), N, H, W, Cin, Cout, what,
+        self._check(self._L.wino_debug_dump(self._h, workspace.data_ptr(), N, H, W, Cin, Cout, what,
                                          a.ctypes.data, a.nbytes), "wino_debug_dump")
         return a

@@ -55,6 +55,8 @@ extern "C" {
 #define WINO_ERR_CUDA (-4)           /* CUDA runtime/driver error; see wino_last_cuda_error */
 #define WINO_ERR_DEVICE_TIMEOUT (-5) /* a bounded device wait expired; the kernel returned early */
 #define WINO_ERR_NOT_EXACT (-6)      /* transform entries not exactly representable (plan) */
+#define WINO_ERR_DEVICE_BOUNDS (-7)  /* debug build: a kernel's index check failed (the access was skipped) */
+#define WINO_ERR_GUARD (-8)          /* a workspace guard band was overwritten (WINO_DEBUG_GUARDS) */
 
 /* ----------------------------------------------------------------- dtypes */
 #define WINO_F32 0
@@ -81,7 +83,16 @@ typedef struct wino_opts {
                              waits 1 ms on a barrier nothing completes, so its
                              bounded wait expires, every CTA returns early and
                              wino_check_device_error reports
-                             WINO_ERR_DEVICE_TIMEOUT (output undefined) */
+                             WINO_ERR_DEVICE_TIMEOUT (output undefined);
+                      bit 3: guard bands: 4096 bytes of 0xA5 before every
+                             workspace region and after the last (the workspace
+                             grows accordingly), written at the start of each
+                             wino_conv2d_int8 call; wino_check_guards checks them;
+                      bit 4: test hook of the debug build's index checks: every
+                             element count the kernels check against is one less
+                             than its buffer, so the last access of each buffer is
+                             skipped and reported as WINO_ERR_DEVICE_BOUNDS (no
+                             effect in the release build, which has no checks) */
     int y_groups;  /* WINO_YGROUPS_*: how Y is grouped for its requantisation */
     int x_int8;    /* 0 or 1.  1: group-wise int8 on x itself before the input transform
                       (alternative reading of the input side, Eqs. (14)-(16)): per pixel, G
@@ -106,6 +117,8 @@ typedef struct wino_opts {
 #define WINO_DEBUG_YQ 1
 #define WINO_DEBUG_ACC32 2
 #define WINO_DEBUG_FORCE_TIMEOUT 4
+#define WINO_DEBUG_GUARDS 8
+#define WINO_DEBUG_SHRINK_BOUNDS 16
 
 /* Debug dump selectors for wino_debug_dump (logical, tile-major layouts of the copy;
  * the kernels keep Vq, sV, Yq and Y tap-major in the workspace). */
@@ -180,9 +193,12 @@ size_t wino_workspace_bytes(wino_plan_t plan, int N, int H, int W, int Cin, int 
  * pass runs with swapped operands (output channels on the MMA rows); layers
  * with few tiles per SM run split transform kernels (more threads per tile).
  * The call returns after the launches (asynchronous).
- * A bounded device wait that expires makes a later call on the same
- * workspace return WINO_ERR_DEVICE_TIMEOUT (see wino_check_device_error).
- * Errors: INVALID_ARG, UNSUPPORTED, WORKSPACE, CUDA, DEVICE_TIMEOUT.
+ * A bounded device wait that expires is recorded in the workspace's device
+ * error word, and the kernels return early (output undefined).  The call
+ * cannot see that itself: call wino_check_device_error on the workspace after
+ * the call and before the next call on that workspace, which clears the word
+ * (on the stream, before its first kernel).
+ * Errors: INVALID_ARG, UNSUPPORTED, WORKSPACE, CUDA.
  */
 int wino_conv2d_int8(wino_plan_t plan, const void* x_dev, int x_dtype, int N, int H, int W, int Cin,
                       const void* wt_dev, int Cout, void* y_dev, int y_dtype, void* ws_dev, size_t ws_bytes,
@@ -205,11 +221,21 @@ int wino_conv2d_int8(wino_plan_t plan, const void* x_dev, int x_dtype, int N, in
  *   - All calls share the array, which keeps the previous call's contents;
  *     the convolution clears what must start at zero itself.  Calls whose
  *     kernels overlap on the GPU race on the array: order them.
+ *   - A bounded device wait that expires is recorded in the array's device
+ *     error word: call wino_check_device_error_noalloc after the call and
+ *     before the next call, which clears the word.
  * Errors: INVALID_ARG, WORKSPACE, CUDA, plus those of wino_conv2d_int8.
  */
 #define WINO_NOALLOC_SCRATCH_BYTES (64u << 20)
 int wino_conv2d_int8_noalloc(wino_plan_t plan, const void* x_dev, int x_dtype, int N, int H, int W, int Cin,
                              const void* wt_dev, int Cout, void* y_dev, int y_dtype, void* stream);
+
+/* wino_check_device_error for wino_conv2d_int8_noalloc: synchronises stream and
+ * reads the device error word the last call of this shape and plan left in the
+ * library's scratch array: WINO_OK, or WINO_ERR_DEVICE_TIMEOUT if a bounded wait
+ * in a kernel expired.  (No counterpart in the paper.)  Errors: INVALID_ARG,
+ * WORKSPACE (shape beyond the array), CUDA. */
+int wino_check_device_error_noalloc(wino_plan_t plan, int N, int H, int W, int Cin, int Cout, void* stream);
 
 /* Extra device bytes wino_conv2d_int8_host needs beyond wino_workspace_bytes
  * (device staging for x and y). */
@@ -227,21 +253,36 @@ size_t wino_host_staging_bytes(wino_plan_t plan, int N, int H, int W, int Cin, i
  * identical to one call, every tile belonging to one image).  ws_dev must hold
  * wino_workspace_bytes() + wino_host_staging_bytes().  The caller synchronises
  * `stream` before reading y_host.  Calls on one plan must not run concurrently.
- * Back-to-back calls of the same shape on the same workspace overlap: each
- * chunk's input copy waits only for the previous call's convolution of that
- * chunk, so the next batch streams in while the previous one finishes.  The
- * staging part of ws_dev (beyond wino_workspace_bytes) must therefore be used
- * by nothing but these calls, and x_host must not change until the call's
- * work on `stream` has completed.
+ * Back-to-back calls of the same plan and shape on the same workspace overlap:
+ * each chunk's input copy waits only for the previous call's convolution of
+ * that chunk, so the next batch streams in while the previous one finishes.
+ * Any other call on ws_dev in between (another plan or shape, or
+ * wino_conv2d_int8) ends that chaining, so the next host call waits for all
+ * prior work on `stream`.  Work outside this library must not use ws_dev, and
+ * x_host must not change until the call's work on `stream` has completed.
  */
 int wino_conv2d_int8_host(wino_plan_t plan, const void* x_host, int x_dtype, int N, int H, int W, int Cin,
                            const void* wt_dev, int Cout, void* y_host, int y_dtype, void* ws_dev, size_t ws_bytes,
                            void* stream);
 
-/* Synchronises stream and reads the workspace's device error word: WINO_OK,
- * or WINO_ERR_DEVICE_TIMEOUT if a bounded wait in a kernel expired. */
+/* Synchronises stream and reads the workspace's device error word left by the
+ * last call on ws_dev: WINO_OK, WINO_ERR_DEVICE_TIMEOUT if a bounded wait in a
+ * kernel expired, or (debug build only, libwino_b200_debug.so, compiled with
+ * WINO_DEBUG) WINO_ERR_DEVICE_BOUNDS if a kernel's index check found an
+ * element index outside its buffer and skipped the access.  The next call on
+ * the workspace clears the word, so check between calls. */
 int wino_check_device_error(wino_plan_t plan, const void* ws_dev, int N, int H, int W, int Cin, int Cout,
                             void* stream);
+
+/* Guard bands (plan option WINO_DEBUG_GUARDS): synchronises stream and checks
+ * that every guard band of the workspace layout of this shape still holds its
+ * pattern after the last wino_conv2d_int8 call on ws_dev.  Returns WINO_OK, or
+ * WINO_ERR_GUARD with *bad_guard (may be NULL) set to the index of the first
+ * overwritten band in layout order; WINO_ERR_UNSUPPORTED if the plan has no
+ * guard bands.  (A stand-in for a memory checker, which is not available where
+ * this library is tested; no counterpart in the paper.) */
+int wino_check_guards(wino_plan_t plan, const void* ws_dev, int N, int H, int W, int Cin, int Cout, void* stream,
+                      int* bad_guard);
 
 /* Synchronous copy of one intermediate tensor of the last call on ws_dev
  * into host_dst (logical layout per WINO_DUMP_*).  Errors: INVALID_ARG,

@@ -31,10 +31,27 @@ def test_header_declares_the_binding_entry_points():
     assert declared_functions() == sorted(wino.EXPORTED)
 
 
-def test_library_exports_every_declared_symbol(lib):
+def test_binding_constants_match_the_header():
+    src = open(os.path.join(ROOT, "include", "wino.h")).read()
+    m = re.search(r"#define WINO_NOALLOC_SCRATCH_BYTES \((\d+)u << (\d+)\)", src)
+    assert m and int(m.group(1)) << int(m.group(2)) == wino.NOALLOC_SCRATCH_BYTES
+
+
+def test_noalloc_error_query_checks_its_arguments(lib):
+    """wino_check_device_error_noalloc rejects a null plan, bad shapes and shapes beyond the
+    scratch array before touching the GPU."""
+    assert lib.wino_check_device_error_noalloc(None, 1, 8, 8, 32, 32, None) == wino.ERR_INVALID_ARG
+    plan = wino.Plan(6, synth.POINTS_F6, None, None, 32)
+    assert lib.wino_check_device_error_noalloc(plan._h, 1, 8, 8, 33, 32, None) == wino.ERR_INVALID_ARG
+    assert lib.wino_check_device_error_noalloc(plan._h, 128, 56, 56, 64, 64, None) == wino.ERR_WORKSPACE
+
+
+@pytest.mark.parametrize("variant", ["release", "debug"])
+def test_library_exports_every_declared_symbol(lib, variant):
+    L = wino.load_library(variant=variant)
     for name in declared_functions():
-        assert hasattr(lib, name), name
-    out = os.popen("nm -D --defined-only %s" % wino.LIB_PATH).read()
+        assert hasattr(L, name), name
+    out = os.popen("nm -D --defined-only %s" % wino.LIB_PATHS[variant]).read()
     for name in declared_functions():
         assert re.search(r"\bT %s\b" % name, out), name
 
