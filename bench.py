@@ -1,30 +1,45 @@
 """Benchmark of the group-wise fully quantized int8 Winograd convolution on B200.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload resnet18] [--impl reference]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload sd15_stack] [--impl reference]
 
-One step = one pass of the whole hot path over one batch: the input
-transform with its group-wise int8 quantisation, the Hadamard int8 GEMM(s)
-with per-K-group dequantisation and Y absmax, Y requantisation and the output
-transform (wino_conv2d_int8).  The weight transform is offline (once per
-layer) and is not part of a step.
+One step = one pass of the whole hot path over one batch of every conv of the
+workload: per conv the input transform with its group-wise int8 quantisation,
+the Hadamard int8 GEMM(s) with per-K-group dequantisation and Y absmax, Y
+requantisation and the output transform (wino_conv2d_int8).  The weight
+transform is offline (once per layer, "pre-transformed once") and is not part
+of a step.
 
-Metric: direct-convolution-equivalent TFLOP/s, 2 N H W Cin Cout 9 / time,
-whole job (all ranks).  Default workload: the ResNet-18-like layer, F(6,3),
-N32 C64 56x56 bf16, seeded synthetic inputs.  L2 is flushed (a 256 MiB write)
-before every timed step; each step is timed with CUDA events on the stream
-the kernels run on, and the run's time is the sum of the step times (max over
-ranks).  Multi-GPU: each rank runs its own batch (weak scaling, no
+Default workload: the back-to-back stack of the 44 3x3 ResNet-block convs of
+an SD-v1.5-shaped UNet (channels 320/640/1280/1280 on the down and up paths,
+latent 64x64, concatenated-skip widths Cin = 960/1920/2560 included), batch
+8, F(6,3), G = 64, bf16 Student-t(3) activations with 1 % outlier channels,
+seeded scales; every conv has its own seeded input and weights.  L2 is
+flushed (a 256 MiB write) once before every step and the 44 convs then run
+back to back on one stream, as they would inside a model.  Metric:
+direct-convolution-equivalent TFLOP/s = sum over convs of 2 N H W Cin Cout 9
+/ step time, whole job (all ranks).  Each step is timed with CUDA events on
+the stream the kernels run on; the run's time is the sum of the step times
+(max over ranks).  Multi-GPU: each rank runs its own batch (weak scaling, no
 collective on the data path).
+
+The same JSON line carries, beside the headline: the ResNet-18-like layer
+(F(6,3) N32 C64 56x56 G32) timed the same way with an L2 flush before every
+call; a per-layer table of the ResNet-34-shaped and SD-shaped layers; cuDNN
+bf16 channels-last convolution of the same shapes for context; the int8
+tensor-core peak measured in-run (a large torch._int_mm); and the CPU oracle
+on the host cores (all of them, and one thread).
 
 --impl reference times the CPU oracle (the plain C++ restatement of the
 method in oracle/) on the host cores for the same workload and metric, each
-step a bounded sample of tile rows of the layer.
+step a bounded sample of tile rows of the workload's convs.
 """
 from __future__ import annotations
 
 import argparse
+import collections
+import concurrent.futures
 import json
-import math
+import multiprocessing
 import os
 import statistics
 import subprocess
@@ -42,30 +57,27 @@ from group_wise_int8_b200 import synth  # noqa: E402
 METRIC = "direct-conv-equiv TFLOP/s per layer; % of int8 tensor-core / HBM roofline"
 UNIT = "TFLOP/s"
 
-# DRAM bytes per launch of the dominant kernel from an ncu capture
-# (dram__bytes_read.sum + dram__bytes_write.sum); the summary with its command
-# line is the named file under profiles/.  None until a capture of the
-# current kernel exists.
-NCU_TRAFFIC = {
-    # (workload, layer, kernel) -> dram read+write bytes per launch from one ncu capture of the
-    # CURRENT kernel (summarised under profiles/); entries are removed whenever that kernel changes.
-    ("resnet18", 0, "input_transform"): 12912896,
-    ("resnet18", 0, "hadamard_absmax"): 15109632,
-    ("resnet18", 0, "hadamard_quant"): 15120128,
-    ("resnet18", 0, "output_transform"): 13168896,
-}
+# DRAM bytes per launch of a kernel from one ncu capture of the CURRENT kernel
+# (dram__bytes_read.sum + dram__bytes_write.sum), keyed by (layer shape, kernel);
+# the summary with its command line is the named file under profiles/.  An
+# entry is removed whenever its kernel changes.
+NCU_TRAFFIC = {}
 
 
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=3000)
-    ap.add_argument("--warmup", type=int, default=20)
-    ap.add_argument("--workload", default="resnet18",
-                    help="resnet18 (default) | resnet34:<i> | sd15:<i> | sd15_stack:<i> | probe:<i>")
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="sd15_stack",
+                    help="sd15_stack (default: all 44 convs) | resnet18[:i] | resnet34[:i] | sd15[:i] | "
+                         "sd15_stack:<i> | probe:<i>")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--e2e-steps", type=int, default=200)
+    ap.add_argument("--no-extras", action="store_true",
+                    help="skip the ResNet-18 line, the per-layer table, cuDNN and the int8 peak")
+    ap.add_argument("--layer-steps", type=int, default=30, help="timed calls per layer in the per-layer table")
+    ap.add_argument("--e2e-steps", type=int, default=None, help="steps of the host-buffer leg (default: --steps)")
     ap.add_argument("--y-groups", default="tile", choices=["tile", "tap"],
                     help="Y quantisation groups: tile (default reading) or tap (the per-tap option)")
     ap.add_argument("--x-int8", action="store_true",
@@ -75,11 +87,27 @@ def parse():
     return ap.parse_args()
 
 
-def pick_layer(name: str) -> synth.Layer:
+def pick_layers(name: str):
+    """(label, layers): a whole workload, or one layer of it with 'workload:i'."""
     if ":" in name:
         w, i = name.split(":")
-        return synth.workload(w)[int(i)]
-    return synth.workload(name)[0]
+        layer = synth.workload(w)[int(i)]
+        return "%s[%d]: %s" % (w, layer.index, layer.describe()), [layer]
+    layers = synth.workload(name)
+    if name == "resnet18":
+        layers = layers[:1]
+    if len(layers) == 1:
+        return "%s[0]: %s" % (name, layers[0].describe()), layers
+    if name == "sd15_stack":
+        l0 = layers[0]
+        return ("sd15_stack: the 44 3x3 ResNet-block convs of an SD-v1.5-shaped UNet back to back, "
+                "F(%d,3) N%d G%d %s, Cin 320-2560, Cout 320-1280, 64x64..8x8" % (l0.m, l0.N, l0.group, l0.dtype),
+                layers)
+    return "%s: %d layers" % (name, len(layers)), layers
+
+
+def shape_key(layer: synth.Layer) -> str:
+    return "F(%d,3) N%d %d->%d %dx%d G%d" % (layer.m, layer.N, layer.Cin, layer.Cout, layer.H, layer.W, layer.group)
 
 
 def load_peaks():
@@ -192,8 +220,283 @@ def job_throughput(units_per_rank: float, world: int, max_ms: float) -> float:
     return world * units_per_rank / (max_ms * 1e-3)
 
 
+# ------------------------------------------------------ synthetic data (host)
+def _gen_layer(layer: synth.Layer):
+    """Seeded input (bf16 bits or fp32) and weights of one layer; runs in the spawn pool."""
+    x_f32, x_bits = synth.make_input(layer)
+    w = synth.make_weights(layer)
+    return (x_bits if x_bits is not None else x_f32), w
+
+
+def generate(layers):
+    """Inputs and weights of every layer, in layer order, drawn by a pool of spawned worker
+    processes (spawn, so the workers inherit no CUDA state of this process)."""
+    if len(layers) == 1:
+        return iter([_gen_layer(layers[0])])
+    ctx = multiprocessing.get_context("spawn")
+    workers = max(1, min(len(layers), (os.cpu_count() or 2) - 1, 16))
+    ex = concurrent.futures.ProcessPoolExecutor(max_workers=workers, mp_context=ctx)
+    futs = [ex.submit(_gen_layer, l) for l in layers]
+
+    def it():
+        try:
+            for f in futs:
+                yield f.result()
+        finally:
+            ex.shutdown(wait=True)
+    return it()
+
+
 # --------------------------------------------------------------- our CUDA path
-def run_ours(args, layer, rank, world):
+class DevLayer:
+    pass
+
+
+def plan_key(layer: synth.Layer):
+    return (layer.m, layer.points, layer.group, layer.workload if layer.scales != "identity" else "identity")
+
+
+def make_plan(layer: synth.Layer, args):
+    from group_wise_int8_b200 import wino
+    sb, sg = synth.make_scales(layer)
+    y_groups = wino.YGROUPS_TAP if getattr(args, "y_groups", "tile") == "tap" else wino.YGROUPS_TILE
+    return wino.Plan(layer.m, layer.points, sb, sg, layer.group, y_groups=y_groups,
+                     x_int8=getattr(args, "x_int8", False), int8_transforms=getattr(args, "int8_transforms", False))
+
+
+def prepare(layers, args, dev, keep_bf16_weights=False):
+    """Device copies of every layer: input, transformed weights, output buffer, and the plans
+    (one per distinct plan key, shared by the layers that use it)."""
+    import torch
+    plans = {}
+    dls = []
+    for layer, (xh, w) in zip(layers, generate(layers)):
+        k = plan_key(layer)
+        if k not in plans:
+            plans[k] = make_plan(layer, args)
+        d = DevLayer()
+        d.layer, d.plan = layer, plans[k]
+        if xh.dtype == np.uint16:
+            d.x = torch.from_numpy(xh.view(np.int16)).view(torch.bfloat16).to(dev)
+        else:
+            d.x = torch.from_numpy(xh).to(dev)
+        wd = torch.from_numpy(w).to(dev)
+        d.wt = d.plan.transform_weights(wd)
+        d.w_bf16 = wd.to(torch.bfloat16).permute(0, 3, 1, 2) if keep_bf16_weights else None
+        del wd
+        d.y = torch.empty((layer.N, layer.H, layer.W, layer.Cout), dtype=torch.bfloat16, device=dev)
+        d.shape = (layer.N, layer.H, layer.W, layer.Cin, layer.Cout)
+        d.y_path, d.gemm = d.plan.resolved_config(*d.shape)
+        d.variants = d.plan.resolved_variants(*d.shape)
+        d.launches = d.plan.launches_per_call(*d.shape)
+        dls.append(d)
+    torch.cuda.synchronize()
+    return dls
+
+
+def run_step(dls, ws, plan_of=None):
+    for d in dls:
+        p = plan_of(d) if plan_of else d.plan
+        p.conv2d(d.x, d.wt, d.layer.Cout, out=d.y, workspace=ws)
+
+
+def bus_id(dev):
+    import torch
+    try:
+        pr = torch.cuda.get_device_properties(dev)
+        return "%08X:%02X:%02X.0" % (int(pr.pci_domain_id), int(pr.pci_bus_id), int(pr.pci_device_id))
+    except Exception:
+        return None
+
+
+def time_steps(dls, ws, flush, stream, steps, warmup):
+    """Per-step CUDA-event times (ms) with one L2 flush before each step (outside the events)."""
+    import torch
+    for i in range(warmup):
+        flush.fill_(i & 0xff)
+        run_step(dls, ws)
+    torch.cuda.synchronize()
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    for i in range(steps):
+        flush.fill_(i & 0xff)
+        starts[i].record(stream)
+        run_step(dls, ws)
+        ends[i].record(stream)
+    torch.cuda.synchronize()
+    return [s.elapsed_time(e) for s, e in zip(starts, ends)]
+
+
+def profile_kernels(dls, ws, flush, steps, args):
+    """Average duration of every launch of every layer: a pass of `steps` steps with per-layer
+    plans whose calls record a CUDA event between kernels (kept out of the timed region: events
+    between kernels stop the next kernel's launch from overlapping the previous one's tail)."""
+    import torch
+    pplans = [make_plan(d.layer, args) for d in dls]
+    for p in pplans:
+        p.profile_begin(steps)
+    idx = {id(d): i for i, d in enumerate(dls)}
+    for i in range(steps):
+        flush.fill_(i & 0xff)
+        run_step(dls, ws, plan_of=lambda d: pplans[idx[id(d)]])
+    torch.cuda.synchronize()
+    out = []
+    for d, p in zip(dls, pplans):
+        ms, calls = p.profile_end()
+        assert calls == steps
+        model = stage_model(d.layer, d.y_path, getattr(args, "x_int8", False))
+        assert len(model) == len(ms), (len(model), len(ms))
+        out.append([(mk[0], mk[1], mk[2], t / calls) for mk, t in zip(model, ms)])
+    return out
+
+
+def roofline_of(dls, prof, peaks, int8_peak=None):
+    """Dominant (layer shape, kernel): the largest summed launch time over the step."""
+    tot = collections.defaultdict(float)
+    info = {}
+    for d, kernels in zip(dls, prof):
+        for name, nbytes, ops, ms in kernels:
+            key = (shape_key(d.layer), name)
+            tot[key] += ms
+            info.setdefault(key, []).append((nbytes, ops, ms))
+    key = max(tot, key=tot.get)
+    runs = info[key]
+    nbytes, ops = runs[0][0], runs[0][1]
+    avg_ms = sum(r[2] for r in runs) / len(runs)
+    achieved = nbytes / (avg_ms * 1e-3) / 1e9
+    step_ms = sum(tot.values())
+    r = {"kernel": "%s (%s)" % (key[1], key[0]), "bound": "hbm", "achieved": round(achieved, 1),
+         "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
+         "traffic": NCU_TRAFFIC.get(key), "algorithmic_bytes": int(nbytes), "avg_launch_us": round(avg_ms * 1e3, 2),
+         "launches_per_step": len(runs), "share_of_kernel_time": round(tot[key] / step_ms, 3),
+         "peak_source": peaks["source"] + " (hbm_gbs, copy test)",
+         "launch_timing": "CUDA events between kernels on the launching stream, in a second pass right after "
+                          "the timed region"}
+    if ops and int8_peak:
+        r["int8_tops"] = round(ops / (avg_ms * 1e-3) / 1e12, 1)
+        r["int8_frac"] = round(ops / (avg_ms * 1e-3) / 1e12 / int8_peak, 4)
+    return r
+
+
+def kernel_table(dls, prof, int8_peak=None, peaks=None):
+    """Per distinct layer shape: count, and per kernel the average us, GB/s and fractions."""
+    rows = collections.OrderedDict()
+    for d, kernels in zip(dls, prof):
+        k = shape_key(d.layer)
+        row = rows.setdefault(k, {"layer": k, "count": 0, "y_path": {1: "recompute", 2: "y32"}.get(d.y_path),
+                                  "variants": d.variants, "acc": collections.defaultdict(list)})
+        row["count"] += 1
+        for name, nbytes, ops, ms in kernels:
+            row["acc"][name].append((nbytes, ops, ms))
+    out = []
+    for row in rows.values():
+        ks = []
+        for name, runs in row.pop("acc").items():
+            ms = sum(r[2] for r in runs) / len(runs)
+            e = {"kernel": name, "avg_us": round(ms * 1e3, 2), "gbs": round(runs[0][0] / (ms * 1e-3) / 1e9, 1)}
+            if peaks:
+                e["hbm_frac"] = round(runs[0][0] / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 3)
+            if runs[0][1]:
+                e["int8_tops"] = round(runs[0][1] / (ms * 1e-3) / 1e12, 1)
+                if int8_peak:
+                    e["int8_frac"] = round(runs[0][1] / (ms * 1e-3) / 1e12 / int8_peak, 4)
+            ks.append(e)
+        row["kernels"] = ks
+        out.append(row)
+    return out
+
+
+def time_e2e(dls, steps, world, dev, stream):
+    """The host-buffer entry point: every step copies each conv's input from pinned host memory,
+    runs it and copies its output back (wino_conv2d_int8_host)."""
+    import torch
+    import torch.distributed as dist
+    hx = [d.x.cpu().pin_memory() for d in dls]
+    hy = [torch.empty(d.y.shape, dtype=torch.bfloat16).pin_memory() for d in dls]
+    need = max(d.plan.workspace_bytes(*d.shape) + d.plan.host_staging_bytes(*d.shape, d.x.dtype, torch.bfloat16)
+               for d in dls)
+    ws = torch.empty(need, dtype=torch.uint8, device=dev)
+
+    def step():
+        for d, x_h, y_h in zip(dls, hx, hy):
+            d.plan.conv2d_host(x_h, d.wt, d.layer.Cout, y_h, ws)
+    for _ in range(2):
+        step()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
+    flops = sum(d.layer.direct_flops for d in dls)
+    h2d = sum(x.numel() * x.element_size() for x in hx)
+    d2h = sum(y.numel() * y.element_size() for y in hy)
+    del ws
+    return {"value": job_throughput(steps * flops, world, e_ms) / 1e12, "unit": UNIT,
+            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "steps": steps,
+            "ms_per_step": e_ms / steps, "api": "wino_conv2d_int8_host (pinned host buffers, copies in the call)"}
+
+
+def time_cudnn(dls, flush, stream, steps, warmup=3):
+    """cuDNN bf16 convolution of the same shapes (channels-last), for context."""
+    import torch
+    import torch.nn.functional as F
+    torch.backends.cudnn.benchmark = True
+    xs = [d.x.permute(0, 3, 1, 2) if d.x.dtype == torch.bfloat16 else d.x.to(torch.bfloat16).permute(0, 3, 1, 2)
+          for d in dls]
+    ws_ = [d.w_bf16 for d in dls]
+
+    def step():
+        for x, w in zip(xs, ws_):
+            F.conv2d(x, w, padding=1)
+    for i in range(warmup):
+        flush.fill_(i & 0xff)
+        step()
+    torch.cuda.synchronize()
+    times = []
+    for i in range(steps):
+        flush.fill_(i & 0xff)
+        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s.record(stream)
+        step()
+        e.record(stream)
+        torch.cuda.synchronize()
+        times.append(s.elapsed_time(e))
+    ms = sum(times) / len(times)
+    flops = sum(d.layer.direct_flops for d in dls)
+    return {"value": flops / (ms * 1e-3) / 1e12, "unit": UNIT, "ms_per_step": ms,
+            "what": "torch.nn.functional.conv2d, bf16 NHWC (channels_last), cudnn.benchmark, same shapes"}
+
+
+def int8_peak_tops(dev, size=8192, reps=10):
+    """Dense int8 tensor-core throughput measured in-run: torch._int_mm (cuBLASLt) on size^3."""
+    import torch
+    try:
+        a = torch.randint(-127, 128, (size, size), dtype=torch.int8, device=dev)
+        b = torch.randint(-127, 128, (size, size), dtype=torch.int8, device=dev).t()
+        for _ in range(3):
+            torch._int_mm(a, b)
+        torch.cuda.synchronize()
+        best = float("inf")
+        for _ in range(reps):
+            s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            s.record()
+            torch._int_mm(a, b)
+            e.record()
+            torch.cuda.synchronize()
+            best = min(best, s.elapsed_time(e))
+        return {"int8_tops": round(2.0 * size ** 3 / (best * 1e-3) / 1e12, 1), "how":
+                "torch._int_mm int8 %d^3, best of %d (CUDA events)" % (size, reps)}
+    except Exception as ex:   # report, do not fail the benchmark
+        return {"int8_tops": None, "how": "torch._int_mm unavailable: %s" % str(ex).splitlines()[0][:120]}
+
+
+def run_ours(args, label, layers, rank, world):
     import torch
     import torch.distributed as dist
     from group_wise_int8_b200 import build, wino
@@ -201,137 +504,111 @@ def run_ours(args, layer, rank, world):
     dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
     torch.cuda.set_device(dev)
     build.build()
-    x_f32, x_bits = synth.make_input(layer)
-    w = synth.make_weights(layer)
-    sb, sg = synth.make_scales(layer)
-    y_groups = wino.YGROUPS_TAP if getattr(args, "y_groups", "tile") == "tap" else wino.YGROUPS_TILE
-    plan = wino.Plan(layer.m, layer.points, sb, sg, layer.group, y_groups=y_groups, x_int8=args.x_int8,
-                     int8_transforms=args.int8_transforms)
-    N, H, W, Cin, Cout = layer.N, layer.H, layer.W, layer.Cin, layer.Cout
-    if x_bits is not None:
-        x = torch.from_numpy(x_bits.view(np.int16).copy()).view(torch.bfloat16).to(dev)
-    else:
-        x = torch.from_numpy(x_f32).to(dev)
-    wt = plan.transform_weights(torch.from_numpy(w).to(dev))
-    ws = torch.empty(plan.workspace_bytes(N, H, W, Cin, Cout), dtype=torch.uint8, device=dev)
-    y = torch.empty((N, H, W, Cout), dtype=torch.bfloat16, device=dev)
+    extras = not args.no_extras and world == 1
+    dls = prepare(layers, args, dev, keep_bf16_weights=extras)
+    ws = torch.empty(max(d.plan.workspace_bytes(*d.shape) for d in dls), dtype=torch.uint8, device=dev)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
-    y_path, gemm = plan.resolved_config(N, H, W, Cin, Cout)
-    launches = plan.launches_per_call(N, H, W, Cin, Cout)
 
-    for _ in range(args.warmup):
-        flush.fill_(1)
-        plan.conv2d(x, wt, Cout, out=y, workspace=ws)
+    for i in range(args.warmup):
+        flush.fill_(i & 0xff)
+        run_step(dls, ws)
     torch.cuda.synchronize()
-    assert plan.check_device_error(ws, N, H, W, Cin, Cout) == wino.OK
-
-    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    bus = None
-    try:
-        pr = torch.cuda.get_device_properties(dev)
-        bus = "%08X:%02X:%02X.0" % (int(pr.pci_domain_id), int(pr.pci_bus_id), int(pr.pci_device_id))
-    except Exception:
-        pass
-    sampler = ClockSampler(bus)
+    last = dls[-1]   # the error word of the last call on the shared workspace
+    assert last.plan.check_device_error(ws, *last.shape) == wino.OK
+    sampler = ClockSampler(bus_id(dev))
     sampler.start()
     time.sleep(0.3)
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
     t_wall = time.perf_counter()
-    for i in range(args.steps):
-        flush.fill_(i & 0xff)
-        starts[i].record(stream)
-        plan.conv2d(x, wt, Cout, out=y, workspace=ws)
-        ends[i].record(stream)
-    torch.cuda.synchronize()
+    step_ms = time_steps(dls, ws, flush, stream, args.steps, 0)
     if world > 1:
         dist.barrier()
     t_wall = time.perf_counter() - t_wall
     clocks = sampler.stop()
-    assert plan.check_device_error(ws, N, H, W, Cin, Cout) == wino.OK
-    # Per-kernel breakdown: a second pass of the same steps with an event between every two
-    # kernels (events between kernels stop the next kernel's launch from overlapping the
-    # previous one's tail, so this pass is kept out of the timed region above).
-    prof_steps = min(args.steps, 500)
-    plan.profile_begin(prof_steps)
-    for i in range(prof_steps):
-        flush.fill_(i & 0xff)
-        plan.conv2d(x, wt, Cout, out=y, workspace=ws)
-    torch.cuda.synchronize()
-    stage_ms, calls = plan.profile_end()
-    assert calls == prof_steps
-    total_ms = max_over_ranks(sum(s.elapsed_time(e) for s, e in zip(starts, ends)), world, dev)
+    assert last.plan.check_device_error(ws, *last.shape) == wino.OK
+    total_ms = max_over_ranks(sum(step_ms), world, dev)
 
-    # end to end through the host-buffer entry point (H2D of x, conv, D2H of y per step)
-    e2e = None
-    if args.e2e_steps > 0:
-        xs = x.element_size()
-        x_host = x.cpu().pin_memory()
-        y_host = torch.empty((N, H, W, Cout), dtype=torch.bfloat16).pin_memory()
-        ws_h = torch.empty(plan.workspace_bytes(N, H, W, Cin, Cout) +
-                           plan.host_staging_bytes(N, H, W, Cin, Cout, x.dtype, torch.bfloat16),
-                           dtype=torch.uint8, device=dev)
-        for _ in range(3):
-            plan.conv2d_host(x_host, wt, Cout, y_host, ws_h)
-        torch.cuda.synchronize()
-        k = args.e2e_steps
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        if world > 1:
-            dist.barrier()
-        torch.cuda.synchronize()
-        e0.record(stream)
-        for _ in range(k):
-            plan.conv2d_host(x_host, wt, Cout, y_host, ws_h)
-        e1.record(stream)
-        torch.cuda.synchronize()
-        e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
-        e2e = {"value": job_throughput(k * layer.direct_flops, world, e_ms) / 1e12, "unit": UNIT,
-               "h2d_bytes_per_step": int(N * H * W * Cin * xs), "d2h_bytes_per_step": int(N * H * W * Cout * 2),
-               "steps": k, "ms_per_step": e_ms / k}
+    prof = profile_kernels(dls, ws, flush, min(args.steps, 200), args)
+    e2e = time_e2e(dls, args.e2e_steps or args.steps, world, dev, stream)
 
-    # roofline of the dominant kernel
     peaks = load_peaks()
-    model = stage_model(layer, y_path, args.x_int8)
-    avg_ms = [t / calls for t in stage_ms]
-    dom = int(np.argmax(avg_ms))
-    name, nbytes, ops = model[dom]
-    achieved_gbs = nbytes / (avg_ms[dom] * 1e-3) / 1e9
-    traffic = NCU_TRAFFIC.get((layer.workload, layer.index, name))
-    roofline = {"kernel": name, "bound": "hbm", "achieved": round(achieved_gbs, 1), "peak": peaks["hbm_gbs"],
-                "unit": "GB/s", "frac": round(achieved_gbs / peaks["hbm_gbs"], 4),
-                "traffic": traffic, "algorithmic_bytes": int(nbytes), "avg_launch_us": round(avg_ms[dom] * 1e3, 2),
-                "peak_source": peaks["source"] + " (hbm_gbs, copy test)",
-                "launch_timing": "CUDA events between kernels on the launching stream, second pass of %d steps "
-                                 "right after the timed region" % calls}
-    per_kernel = [{"kernel": m[0], "avg_us": round(a * 1e3, 2), "algorithmic_bytes": int(m[1]),
-                   "gbs": round(m[1] / (a * 1e-3) / 1e9, 1),
-                   "int8_tops": round(m[2] / (a * 1e-3) / 1e12, 2) if m[2] else None}
-                  for m, a in zip(model, avg_ms)]
-    ms_step = total_ms / args.steps
-    value = job_throughput(args.steps * layer.direct_flops, world, total_ms) / 1e12
-    return {
-        "value": value, "ms_per_step": ms_step, "e2e": e2e, "roofline": roofline, "clocks": clocks,
-        "gpu_launches": args.steps * launches, "per_kernel": per_kernel, "wall_s": t_wall,
-        "y_path": {1: "recompute", 2: "y32"}.get(y_path), "gemm": {1: "tcgen05", 2: "simt"}.get(gemm),
+    i8 = int8_peak_tops(dev) if extras else {"int8_tops": None, "how": "not measured (--no-extras)"}
+    flops = sum(d.layer.direct_flops for d in dls)
+    res = {
+        "value": job_throughput(args.steps * flops, world, total_ms) / 1e12, "ms_per_step": total_ms / args.steps,
+        "e2e": e2e, "roofline": roofline_of(dls, prof, peaks, i8["int8_tops"]), "clocks": clocks,
+        "gpu_launches": args.steps * sum(d.launches for d in dls), "wall_s": t_wall,
+        "kernels": kernel_table(dls, prof, i8["int8_tops"], peaks), "int8_peak": i8,
     }
+    if extras:
+        res["cudnn_bf16"] = time_cudnn(dls, flush, stream, args.steps)
+    del dls, ws
+    torch.cuda.empty_cache()
+    if extras:
+        res["beside"] = layer_line("resnet18", synth.workload("resnet18")[0], args, dev, flush, stream, peaks, i8)
+        res["layers"] = [layer_line(w, l, args, dev, flush, stream, peaks, i8)
+                         for w in ("resnet34", "sd15") for l in synth.workload(w)]
+    return res
+
+
+def layer_line(wname, layer, args, dev, flush, stream, peaks, i8):
+    """One layer timed on its own: L2 flushed before every call."""
+    import torch
+    dls = prepare([layer], args, dev, keep_bf16_weights=True)
+    d = dls[0]
+    ws = torch.empty(d.plan.workspace_bytes(*d.shape), dtype=torch.uint8, device=dev)
+    steps = args.layer_steps
+    ms = time_steps(dls, ws, flush, stream, steps, 3)
+    prof = profile_kernels(dls, ws, flush, steps, args)
+    cd = time_cudnn(dls, flush, stream, steps)
+    avg = sum(ms) / len(ms)
+    out = {"layer": "%s[%d]: %s" % (wname, layer.index, layer.describe()), "value": round(layer.direct_flops /
+           (avg * 1e-3) / 1e12, 1), "us": round(avg * 1e3, 1),
+           "y_path": {1: "recompute", 2: "y32"}.get(d.y_path), "variants": d.variants,
+           "kernels": kernel_table(dls, prof, i8["int8_tops"], peaks)[0]["kernels"],
+           "roofline": roofline_of(dls, prof, peaks, i8["int8_tops"]),
+           "cudnn_bf16_tflops": round(cd["value"], 1), "cudnn_bf16_us": round(cd["ms_per_step"] * 1e3, 1)}
+    del dls, ws
+    torch.cuda.empty_cache()
+    return out
 
 
 # ------------------------------------------------------------- CPU oracle timing
-def oracle_sample(layer: synth.Layer, rows: int, images: int, int8_transforms: bool = False):
-    """The layer cropped to `rows` tile rows of `images` images (same weights)."""
+_SAMPLE_CACHE = {}
+
+
+def oracle_samples(layers, rows: int, images: int, int8_transforms: bool = False, max_cout: int = 256):
+    """Per distinct layer shape: the first `images` images cropped to `rows` tile rows, and the
+    first min(Cout, max_cout) output channels, with the number of convs of that shape in the
+    workload.  The seeded streams give the first images and the first output channels of a
+    layer as a prefix, so these are exactly the workload's own values."""
+    import dataclasses
     import oracle
-    x_f32, _ = synth.make_input(layer)
-    w = synth.make_weights(layer)
-    sb, sg = synth.make_scales(layer)
-    H = min(layer.H, rows * layer.m)
-    xs = np.ascontiguousarray(x_f32[:images, :H])
-    plan = oracle.Plan(layer.m, layer.points, sb, sg, int8_transforms=int8_transforms)
-    Uq, sU, _ = oracle.weight_transform(plan, w, layer.group)
-    flops = 2.0 * images * H * layer.W * layer.Cin * layer.Cout * 9
-    return plan, xs, Uq, sU, flops
+    groups = collections.OrderedDict()
+    for l in layers:
+        groups.setdefault((l.m, l.Cin, l.Cout, l.H, l.W, l.N, l.group), []).append(l)
+    out = []
+    for ls in groups.values():
+        layer = ls[0]
+        cs = min(layer.Cout, max_cout)
+        ni = min(images, layer.N)
+        key = (layer, ni, cs, int8_transforms)
+        if key not in _SAMPLE_CACHE:
+            x_f32, _ = synth.make_input(dataclasses.replace(layer, N=ni))
+            w = synth.make_weights(dataclasses.replace(layer, Cout=cs))
+            sb, sg = synth.make_scales(layer)
+            plan = oracle.Plan(layer.m, layer.points, sb, sg, int8_transforms=int8_transforms)
+            Uq, sU, _ = oracle.weight_transform(plan, w, layer.group)
+            _SAMPLE_CACHE[key] = (plan, x_f32, Uq, sU)
+        plan, x_f32, Uq, sU = _SAMPLE_CACHE[key]
+        H = min(layer.H, rows * layer.m)
+        xs = np.ascontiguousarray(x_f32[:, :H])
+        flops = 2.0 * ni * H * layer.W * layer.Cin * cs * 9
+        out.append((len(ls), layer, plan, xs, Uq, sU, flops))
+    return out
 
 
 def oracle_step(plan, xs, Uq, sU, G, per_tap=False, x_int8=False):
@@ -346,76 +623,87 @@ def oracle_step(plan, xs, Uq, sU, G, per_tap=False, x_int8=False):
     oracle.output_transform(plan, Yq, sY, N, H, W, G, per_tap)
 
 
-def cpu_baseline(layer: synth.Layer, budget_s: float = 12.0, per_tap: bool = False, x_int8: bool = False,
-                 int8_transforms: bool = False):
+def time_samples(samples, reps, per_tap, x_int8):
+    """Workload-weighted CPU throughput: each distinct shape's sample counts as often as the
+    shape occurs in the workload."""
+    t_tot = f_tot = 0.0
+    for count, layer, plan, xs, Uq, sU, flops in samples:
+        t0 = time.perf_counter()
+        for _ in range(reps):
+            oracle_step(plan, xs, Uq, sU, layer.group, per_tap, x_int8)
+        t_tot += count * (time.perf_counter() - t0) / reps
+        f_tot += count * flops
+    return f_tot / t_tot, t_tot
+
+
+def cpu_baseline(label, layers, budget_s: float = 12.0, threads: int = 0, per_tap: bool = False,
+                 x_int8: bool = False, int8_transforms: bool = False):
     import oracle
-    threads = oracle.set_threads(0)
+    used = oracle.set_threads(threads)
     rows, images = 1, 1
-    plan, xs, Uq, sU, flops = oracle_sample(layer, rows, images, int8_transforms)
-    t0 = time.perf_counter()
-    oracle_step(plan, xs, Uq, sU, layer.group, per_tap, x_int8)
-    dt = time.perf_counter() - t0
-    # grow the sample (whole images first) while it stays within the budget
-    TH = -(-layer.H // layer.m)
-    while dt * 2 < budget_s / 2 and (rows < TH or images < layer.N):
+    samples = oracle_samples(layers, rows, images, int8_transforms)
+    _, dt = time_samples(samples, 1, per_tap, x_int8)
+    TH = max(-(-l.H // l.m) for l in layers)
+    Nmax = max(l.N for l in layers)
+    while dt * 2 < budget_s / 2 and (rows < TH or images < Nmax):
         if rows < TH:
             rows = min(TH, rows * 2)
         else:
-            images = min(layer.N, images * 2)
-        plan, xs, Uq, sU, flops = oracle_sample(layer, rows, images, int8_transforms)
-        t0 = time.perf_counter()
-        oracle_step(plan, xs, Uq, sU, layer.group, per_tap, x_int8)
-        dt = time.perf_counter() - t0
+            images = min(Nmax, images * 2)
+        samples = oracle_samples(layers, rows, images, int8_transforms)
+        _, dt = time_samples(samples, 1, per_tap, x_int8)
     reps = max(1, int(budget_s / 2 / max(dt, 1e-3)))
-    t0 = time.perf_counter()
-    for _ in range(reps):
-        oracle_step(plan, xs, Uq, sU, layer.group, per_tap, x_int8)
-    dt = (time.perf_counter() - t0) / reps
-    return {"value": flops / dt / 1e12, "unit": UNIT, "cores": threads, "kind": "oracle",
-            "sample": "%d image(s) x %d of %d tile rows of %s; input transform, Hadamard, Y requant, output "
-                      "transform (weights pre-transformed); %d rep(s)" % (images, rows, TH, layer.describe(), reps)}
+    rate, _ = time_samples(samples, reps, per_tap, x_int8)
+    oracle.set_threads(0)
+    return {"value": rate / 1e12, "unit": UNIT, "cores": used, "kind": "oracle",
+            "sample": "per distinct conv shape of %s: %d image(s) x %d tile row(s) x the first min(Cout, 256) "
+                      "output channels, weighted by the shape's count; input transform, Hadamard, Y requant, "
+                      "output transform (weights pre-transformed); %d rep(s)" % (label, images, rows, reps)}
 
 
-def run_reference(args, layer):
+def run_reference(args, label, layers):
     per_tap = args.y_groups == "tap"
     x_int8 = args.x_int8
     import oracle
     threads = oracle.set_threads(0)
-    TH = -(-layer.H // layer.m)
+    TH = max(-(-l.H // l.m) for l in layers)
     budget = 150.0 / max(1, args.steps + args.warmup)   # seconds per step: whole run within a few minutes
     rows = 1
-    plan, xs, Uq, sU, flops = oracle_sample(layer, rows, 1, args.int8_transforms)
-    t0 = time.perf_counter()
-    oracle_step(plan, xs, Uq, sU, layer.group, per_tap, x_int8)
-    dt = time.perf_counter() - t0
+    samples = oracle_samples(layers, rows, 1, args.int8_transforms)
+    _, dt = time_samples(samples, 1, per_tap, x_int8)
     while dt * 2 <= budget and rows < TH:
         rows = min(TH, rows * 2)
-        plan, xs, Uq, sU, flops = oracle_sample(layer, rows, 1, args.int8_transforms)
-        t0 = time.perf_counter()
-        oracle_step(plan, xs, Uq, sU, layer.group, per_tap, x_int8)
-        dt = time.perf_counter() - t0
+        samples = oracle_samples(layers, rows, 1, args.int8_transforms)
+        _, dt = time_samples(samples, 1, per_tap, x_int8)
     for _ in range(args.warmup):
-        oracle_step(plan, xs, Uq, sU, layer.group, per_tap, x_int8)
-    t0 = time.perf_counter()
+        time_samples(samples, 1, per_tap, x_int8)
+    ms = []
     for _ in range(args.steps):
-        oracle_step(plan, xs, Uq, sU, layer.group, per_tap, x_int8)
-    total = time.perf_counter() - t0
-    value = args.steps * flops / total / 1e12
-    sample = "1 image x %d of %d tile rows of %s per step" % (rows, TH, layer.describe())
-    return {"value": value, "ms_per_step": total / args.steps * 1e3,
+        rate, dt = time_samples(samples, 1, per_tap, x_int8)
+        ms.append(dt * 1e3)
+    flops = sum(c * f for c, _, _, _, _, _, f in samples)
+    value = args.steps * flops / (sum(ms) * 1e-3) / 1e12
+    sample = ("per distinct conv shape of %s: 1 image x %d tile row(s) x the first min(Cout, 256) output "
+              "channels, weighted by the shape's count, per step" % (label, rows))
+    return {"value": value, "ms_per_step": sum(ms) / len(ms),
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": sample}}
 
 
 def main():
     args = parse()
-    layer = pick_layer(args.workload)
+    label, layers = pick_layers(args.workload)
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
-    config = {"workload": "%s[%d]: %s" % (layer.workload, layer.index, layer.describe()), "model": layer.workload,
-              "global_batch": layer.N * world, "seq_len": None, "H": layer.H, "W": layer.W, "Cin": layer.Cin,
-              "Cout": layer.Cout, "m": layer.m, "group": layer.group, "parallelism": "dp%d" % world,
-              "l2": "flushed before every timed step (256 MiB write)", "output": "bf16 NHWC",
-              "y_groups": args.y_groups, "x_int8": args.x_int8, "int8_transforms": args.int8_transforms}
+    l0 = layers[0]
+    config = {"workload": label, "model": l0.workload, "convs_per_step": len(layers),
+              "global_batch": l0.N * world, "seq_len": None, "m": l0.m, "group": l0.group,
+              "parallelism": "dp%d" % world,
+              "l2": ("flushed once before every step (256 MiB write), convs back to back" if len(layers) > 1
+                     else "flushed before every timed step (256 MiB write)"),
+              "output": "bf16 NHWC", "y_groups": args.y_groups, "x_int8": args.x_int8,
+              "int8_transforms": args.int8_transforms}
+    if len(layers) == 1:
+        config.update(H=l0.H, W=l0.W, Cin=l0.Cin, Cout=l0.Cout, N=l0.N)
     line = {"metric": METRIC, "unit": UNIT, "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int8 (fp32 transforms)",
             "data": "synthetic (seeded)", "config": config}
@@ -423,7 +711,7 @@ def main():
     if args.impl == "reference":
         if rank != 0:
             return
-        r = run_reference(args, layer)
+        r = run_reference(args, label, layers)
         line.update(impl="reference", value=r["value"], ms_per_step=r["ms_per_step"], n_gpus=args.gpus,
                     cpu_baseline=r["cpu_baseline"],
                     e2e={"value": r["value"], "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0})
@@ -437,7 +725,7 @@ def main():
         torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", 0)))
         dist.init_process_group("nccl", timeout=timedelta(seconds=120))
     try:
-        r = run_ours(args, layer, rank, world)
+        r = run_ours(args, label, layers, rank, world)
     finally:
         if world > 1:
             import torch.distributed as dist
@@ -446,11 +734,15 @@ def main():
         return
     cpu = None
     if not args.no_cpu_baseline and world == 1:
-        cpu = cpu_baseline(layer, per_tap=args.y_groups == "tap", x_int8=args.x_int8,
-                           int8_transforms=args.int8_transforms)
+        kw = dict(per_tap=args.y_groups == "tap", x_int8=args.x_int8, int8_transforms=args.int8_transforms)
+        cpu = cpu_baseline(label, layers, 12.0, 0, **kw)
+        cpu["single_thread"] = cpu_baseline(label, layers, 6.0, 1, **kw)
     line.update(value=r["value"], ms_per_step=r["ms_per_step"], e2e=r["e2e"], roofline=r["roofline"],
-                cpu_baseline=cpu, clocks=r["clocks"], gpu_launches=r["gpu_launches"],
-                kernels=r["per_kernel"], y_path=r["y_path"], gemm=r["gemm"], impl="ours")
+                cpu_baseline=cpu, clocks=r["clocks"], gpu_launches=r["gpu_launches"], impl="ours",
+                kernels=r["kernels"], int8_peak=r["int8_peak"])
+    for k in ("cudnn_bf16", "beside", "layers"):
+        if k in r:
+            line[k] = r[k]
     print(json.dumps(line))
 
 
