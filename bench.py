@@ -84,6 +84,8 @@ def parse():
                     help="alternative reading: x group-quantised per pixel before the input transform")
     ap.add_argument("--int8-transforms", action="store_true",
                     help="alternative reading: B^T and A^T held as int8 with one scale per matrix")
+    ap.add_argument("--fused", action="store_true",
+                    help="the one-kernel path for small channel counts where it applies (off by default)")
     return ap.parse_args()
 
 
@@ -121,7 +123,7 @@ def load_peaks():
 
 
 # ----------------------------------------------------------------- byte model
-def stage_model(layer: synth.Layer, y_path: int, x_int8: bool = False):
+def stage_model(layer: synth.Layer, y_path: int, x_int8: bool = False, fused: bool = False):
     """Algorithmic bytes and int8 ops of each launch of one call, by launch index."""
     from group_wise_int8_b200 import wino
     n2 = layer.n * layer.n
@@ -135,6 +137,8 @@ def stage_model(layer: synth.Layer, y_path: int, x_int8: bool = False):
     amax = 4 * T * (layer.Cout // G)
     yq = T * n2 * layer.Cout
     ops = 2.0 * T * n2 * layer.Cin * layer.Cout
+    if fused:   # one kernel: x in, the transformed weights, the output out; both GEMM passes
+        return [("fused_layer", x + u + out, 2 * ops)]
     stages = []
     if x_int8:   # reads x, writes its fp32 round trip, which the input transform then reads
         xq = layer.N * layer.H * layer.W * layer.Cin * 4
@@ -256,12 +260,15 @@ def plan_key(layer: synth.Layer):
     return (layer.m, layer.points, layer.group, layer.workload if layer.scales != "identity" else "identity")
 
 
-def make_plan(layer: synth.Layer, args):
+def make_plan(layer: synth.Layer, args, fused=None):
     from group_wise_int8_b200 import wino
     sb, sg = synth.make_scales(layer)
     y_groups = wino.YGROUPS_TAP if getattr(args, "y_groups", "tile") == "tap" else wino.YGROUPS_TILE
+    if fused is None:
+        fused = wino.FUSED_ON if getattr(args, "fused", False) else wino.FUSED_AUTO
     return wino.Plan(layer.m, layer.points, sb, sg, layer.group, y_groups=y_groups,
-                     x_int8=getattr(args, "x_int8", False), int8_transforms=getattr(args, "int8_transforms", False))
+                     x_int8=getattr(args, "x_int8", False), int8_transforms=getattr(args, "int8_transforms", False),
+                     fused=fused)
 
 
 def prepare(layers, args, dev, keep_bf16_weights=False):
@@ -332,6 +339,7 @@ def profile_kernels(dls, ws, flush, steps, args):
     plans whose calls record a CUDA event between kernels (kept out of the timed region: events
     between kernels stop the next kernel's launch from overlapping the previous one's tail)."""
     import torch
+    from group_wise_int8_b200 import wino
     pplans = [make_plan(d.layer, args) for d in dls]
     for p in pplans:
         p.profile_begin(steps)
@@ -344,7 +352,8 @@ def profile_kernels(dls, ws, flush, steps, args):
     for d, p in zip(dls, pplans):
         ms, calls = p.profile_end()
         assert calls == steps
-        model = stage_model(d.layer, d.y_path, getattr(args, "x_int8", False))
+        model = stage_model(d.layer, d.y_path, getattr(args, "x_int8", False),
+                            bool(d.variants & wino.VARIANT_FUSED))
         assert len(model) == len(ms), (len(model), len(ms))
         out.append([(mk[0], mk[1], mk[2], t / calls) for mk, t in zip(model, ms)])
     return out
@@ -503,7 +512,7 @@ def run_ours(args, label, layers, rank, world):
 
     dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
     torch.cuda.set_device(dev)
-    build.build()
+    build.build(debug=False)
     extras = not args.no_extras and world == 1
     dls = prepare(layers, args, dev, keep_bf16_weights=extras)
     ws = torch.empty(max(d.plan.workspace_bytes(*d.shape) for d in dls), dtype=torch.uint8, device=dev)
@@ -571,6 +580,18 @@ def layer_line(wname, layer, args, dev, flush, stream, peaks, i8):
            "kernels": kernel_table(dls, prof, i8["int8_tops"], peaks)[0]["kernels"],
            "roofline": roofline_of(dls, prof, peaks, i8["int8_tops"]),
            "cudnn_bf16_tflops": round(cd["value"], 1), "cudnn_bf16_us": round(cd["ms_per_step"] * 1e3, 1)}
+    # the one-kernel path where it applies, timed the same way on the same inputs (opt-in: slower here)
+    from group_wise_int8_b200 import wino
+    fp = make_plan(layer, args, fused=wino.FUSED_ON)
+    if fp.resolved_variants(*d.shape) & wino.VARIANT_FUSED:
+        d.plan = fp
+        # (same points, scales and G: the transformed weights are the same bytes)
+        fws = torch.empty(fp.workspace_bytes(*d.shape), dtype=torch.uint8, device=dev)
+        fms = time_steps(dls, fws, flush, stream, steps, 3)
+        favg = sum(fms) / len(fms)
+        out["fused_us"] = round(favg * 1e3, 1)
+        out["fused_value"] = round(layer.direct_flops / (favg * 1e-3) / 1e12, 1)
+        del fws
     del dls, ws
     torch.cuda.empty_cache()
     return out

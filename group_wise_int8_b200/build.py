@@ -24,7 +24,7 @@ BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(HERE, "libwino_b200.so")
 LIB_DEBUG = os.path.join(HERE, "libwino_b200_debug.so")
 SOURCES = ["plan.cpp", "api.cu", "weight_transform.cu", "input_transform.cu", "hadamard_tc.cu",
-           "hadamard_simt.cu", "output_transform.cu", "input_quant.cu", "noalloc.cu"]
+           "hadamard_simt.cu", "output_transform.cu", "input_quant.cu", "noalloc.cu", "fused_small.cu"]
 HEADERS = ["plan.h", "common.cuh", "sm100.cuh", "kernels.h"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
@@ -78,9 +78,11 @@ def _build_one(lib: str, debug: bool, verbose: bool, ex) -> None:
     os.replace(tmp, lib)
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    """Builds whichever of the release and debug libraries is out of date; returns the release path."""
-    todo = [(lib, dbg) for lib, dbg in ((LIB, False), (LIB_DEBUG, True)) if force or not up_to_date(lib)]
+def build(force: bool = False, verbose: bool = False, debug: bool = True) -> str:
+    """Builds whichever of the release and (with debug) the debug library is out of date; returns
+    the release path."""
+    libs = ((LIB, False), (LIB_DEBUG, True)) if debug else ((LIB, False),)
+    todo = [(lib, dbg) for lib, dbg in libs if force or not up_to_date(lib)]
     if todo:
         with concurrent.futures.ThreadPoolExecutor(max_workers=min(16, os.cpu_count() or 1)) as ex:
             for lib, dbg in todo:

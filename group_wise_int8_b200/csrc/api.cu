@@ -51,7 +51,7 @@ struct Layout {
     int TH = 0, TW = 0, n2 = 0, ng = 0, ngo = 0;
     long T = 0, T_pad = 0;
     int y_path = 0, gemm = 0;
-    bool dbg_yq = false, dbg_acc = false, ytap = false, xq = false, swap = false;
+    bool dbg_yq = false, dbg_acc = false, ytap = false, xq = false, swap = false, fused = false;
     size_t off_xq = 0, off_vq = 0, off_sv = 0, off_amax = 0, off_yq = 0, off_y32 = 0, off_sy = 0, off_acc = 0, off_err = 0;
     size_t total = 0;
     int n_guards = 0;
@@ -114,6 +114,17 @@ Layout make_layout(const wino_plan_s* p, int N, int H, int W, int Cin, int Cout)
     L.dbg_yq = (p->opts.debug & WINO_DEBUG_YQ) != 0;
     L.dbg_acc = (p->opts.debug & WINO_DEBUG_ACC32) != 0;
     L.xq = p->opts.x_int8 != 0;
+    // the one-kernel path for small channel counts (the recompute path's arithmetic in one launch);
+    // on request only: on every configured layer it measures slower than the staged kernels
+    L.fused = p->opts.fused == WINO_FUSED_ON && fused_small_fits(Cin, Cout, p->G) && p->bt_masked &&
+              p->at_masked && !L.ytap && !L.xq &&
+              !L.dbg_acc && p->opts.gemm != WINO_GEMM_SIMT && p->opts.y_path == WINO_YPATH_AUTO &&
+              (p->opts.debug & WINO_DEBUG_FORCE_TIMEOUT) == 0;
+    if (L.fused) {
+        L.y_path = WINO_YPATH_RECOMPUTE;
+        L.gemm = WINO_GEMM_TCGEN05;
+        L.swap = false;
+    }
     const bool guards = (p->opts.debug & WINO_DEBUG_GUARDS) != 0;
     size_t off = 0;
     auto guard = [&]() {
@@ -126,16 +137,23 @@ Layout make_layout(const wino_plan_s* p, int N, int H, int W, int Cin, int Cout)
         L.off_xq = off;
         off = up(off + sizeof(float) * (size_t)N * H * W * Cin, kAlign);
     }
-    guard();
-    L.off_vq = off;
-    off = up(off + (size_t)L.T_pad * L.n2 * Cin, kAlign);
-    guard();
-    L.off_sv = off;
-    off = up(off + sizeof(float) * (size_t)L.n2 * L.ng * L.T_pad, kAlign);
-    guard();
-    L.off_amax = off;
-    off = up(off + sizeof(unsigned) * (size_t)L.T_pad * L.ngo, kAlign);
-    if (L.y_path == WINO_YPATH_RECOMPUTE || L.dbg_yq) {
+    // the fused path keeps Vq, its scales and the Y maxima on chip: they exist in the workspace
+    // only as its debug copies
+    const bool staged = !L.fused || L.dbg_yq;
+    if (staged) {
+        guard();
+        L.off_vq = off;
+        off = up(off + (size_t)L.T_pad * L.n2 * Cin, kAlign);
+        guard();
+        L.off_sv = off;
+        off = up(off + sizeof(float) * (size_t)L.n2 * L.ng * L.T_pad, kAlign);
+    }
+    if (!L.fused) {
+        guard();
+        L.off_amax = off;
+        off = up(off + sizeof(unsigned) * (size_t)L.T_pad * L.ngo, kAlign);
+    }
+    if ((L.y_path == WINO_YPATH_RECOMPUTE && !L.fused) || L.dbg_yq) {
         guard();
         L.off_yq = off;
         off = up(off + (size_t)L.T * L.n2 * Cout, kAlign);
@@ -271,6 +289,41 @@ int run_conv(wino_plan_s* p, const void* x, int x_dtype, int N, int H, int W, in
     const size_t sh = (p->opts.debug & WINO_DEBUG_SHRINK_BOUNDS) ? 1 : 0;
     const size_t n_amax = (size_t)L.T_pad * L.ngo - sh, n_y = (size_t)L.T * L.n2 * Cout - sh;
     int slot = 0;
+    if (L.fused) {
+        FusedArgs fa;
+        fa.x = x;
+        fa.N = N;
+        fa.H = H;
+        fa.W = W;
+        fa.Cin = Cin;
+        fa.Cout = Cout;
+        fa.TH = L.TH;
+        fa.TW = L.TW;
+        fa.G = p->G;
+        fa.T = L.T;
+        fa.T_pad = L.T_pad;
+        fa.Uq = static_cast<const int8_t*>(wt);
+        fa.sU = reinterpret_cast<const float*>(static_cast<const unsigned char*>(wt) +
+                                               up((size_t)L.n2 * Cout * Cin, kAlign));
+        fa.out = y;
+        fa.bf16_out = y_dtype == WINO_BF16 ? 1 : 0;
+        fa.err = err;
+        fa.n_out = (size_t)N * H * W * Cout - sh;
+        fa.Vq_dbg = L.dbg_yq ? reinterpret_cast<int8_t*>(base + L.off_vq) : nullptr;
+        fa.sV_dbg = L.dbg_yq ? reinterpret_cast<float*>(base + L.off_sv) : nullptr;
+        fa.Yq_dbg = L.dbg_yq ? reinterpret_cast<int8_t*>(base + L.off_yq) : nullptr;
+        fa.sY_dbg = L.dbg_yq ? reinterpret_cast<float*>(base + L.off_sy) : nullptr;
+        prof_mark(p, slot++, st);
+        nvtxRangePushA("wino: fused layer");
+        e = launch_fused_small(fa, p->tf, p->mat.m, x_dtype == WINO_BF16, num_sms(), st);
+        nvtxRangePop();
+        prof_mark(p, slot, st);
+        if (p->prof_calls < p->prof_max_calls) {
+            p->prof_launches = slot;
+            ++p->prof_calls;
+        }
+        return cuda_status(p, e);
+    }
     bool x_bf16 = x_dtype == WINO_BF16;
     if (L.xq) {
         float* xq = reinterpret_cast<float*>(base + L.off_xq);
@@ -423,7 +476,8 @@ int wino_plan(wino_plan_t* out, int m, const double* points, const float* S_B, c
     if (opts) p->opts = *opts;
     if (p->opts.y_path < 0 || p->opts.y_path > 2 || p->opts.gemm < 0 || p->opts.gemm > 2 || p->opts.y_groups < 0 ||
         p->opts.y_groups > 1 || (p->opts.y_groups == WINO_YGROUPS_TAP && p->opts.y_path == WINO_YPATH_RECOMPUTE) ||
-        (p->opts.x_int8 != 0 && p->opts.x_int8 != 1) || (p->opts.int8_transforms != 0 && p->opts.int8_transforms != 1)) {
+        (p->opts.x_int8 != 0 && p->opts.x_int8 != 1) || (p->opts.int8_transforms != 0 && p->opts.int8_transforms != 1) ||
+        p->opts.fused < 0 || p->opts.fused > 2) {
         delete p;
         return WINO_ERR_INVALID_ARG;
     }
@@ -656,6 +710,7 @@ int wino_debug_dump(wino_plan_t p, const void* ws, int N, int H, int W, int Cin,
     const Layout L = make_layout(p, N, H, W, Cin, Cout);
     const unsigned char* base = static_cast<const unsigned char*>(ws);
     size_t need = 0, off = 0;
+    if (L.fused && !L.dbg_yq && (what == WINO_DUMP_VQ || what == WINO_DUMP_SV)) return WINO_ERR_UNSUPPORTED;
     switch (what) {
         case WINO_DUMP_VQ: need = (size_t)L.T * L.n2 * Cin; off = L.off_vq; break;
         case WINO_DUMP_SV: need = sizeof(float) * (size_t)L.T * L.n2 * L.ng; off = L.off_sv; break;
@@ -716,6 +771,10 @@ int wino_resolved_variants(wino_plan_t p, int N, int H, int W, int Cin, int Cout
     if (!flags) return WINO_ERR_INVALID_ARG;
     const Layout L = make_layout(p, N, H, W, Cin, Cout);
     int f = 0;
+    if (L.fused) {
+        *flags = WINO_VARIANT_FUSED;
+        return WINO_OK;
+    }
     if (L.swap) f |= WINO_VARIANT_SWAPPED_GEMM;
     if (input_transform_split(p->mat.m, p->G, N, L.TH, L.TW, Cin, num_sms())) f |= WINO_VARIANT_SPLIT_INPUT;
     if (output_transform_split(L.T, Cout, L.y_path == WINO_YPATH_Y32, L.ytap, num_sms()))
@@ -727,6 +786,7 @@ int wino_resolved_variants(wino_plan_t p, int N, int H, int W, int Cin, int Cout
 int wino_launches_per_call(wino_plan_t p, int N, int H, int W, int Cin, int Cout) {
     if (check_shape(p, N, H, W, Cin, Cout)) return 0;
     const Layout L = make_layout(p, N, H, W, Cin, Cout);
+    if (L.fused) return 1;
     return (L.y_path == WINO_YPATH_RECOMPUTE ? 4 : 3) + (L.xq ? 1 : 0);
 }
 

@@ -191,7 +191,8 @@ __global__ void __launch_bounds__(TcCfg<BN>::kThreads, 1)
     const int KC = p.SK / BK;              // K chunks per stage
     const int TPS = p.tps;                 // taps per stage
     const int GPS = p.SK / p.G;            // K-groups per tap per stage = accumulator buffers per slot
-    const int KSTAGES = p.Cin / p.SK;      // stages per tap (TPS == 1 when > 1)
+    const int KSTAGES = (p.ng + GPS - 1) / GPS;   // stages per tap (TPS == 1 when > 1); the last may be ragged
+    const int GLAST = p.ng - (KSTAGES - 1) * GPS; // K-groups of the last stage (its boxes read zeros past Cin)
     const int NSLOT = NACC / GPS;          // accumulator slots (>= 2)
     const uint32_t a_tile = kBM * BK, b_tile = BN * BK;
     const uint32_t a_bytes = a_tile * KC * TPS, b_bytes = b_tile * KC * TPS;
@@ -285,7 +286,6 @@ __global__ void __launch_bounds__(TcCfg<BN>::kThreads, 1)
             const uint32_t idesc = idesc_i8(kBM, BN);
             const uint64_t a_desc0 = smem_desc_kmajor(smem_u32(smem), BK);
             const uint64_t b_desc0 = smem_desc_kmajor(smem_u32(smem) + a_bytes, BK);
-            const int ksteps = p.SK / 32;          // K-steps per tap and stage
             const int ks_per_group = p.G / 32;
             const int ks_per_chunk = BK / 32;
             Ring st{0, 0}, sl{0, 0};
@@ -300,6 +300,7 @@ __global__ void __launch_bounds__(TcCfg<BN>::kThreads, 1)
                         break;
                     }
                     const uint64_t stage_off = (uint64_t)((st.idx * stage_bytes) >> 4);
+                    const int ksteps = (ks + 1 == KSTAGES ? GLAST : GPS) * ks_per_group;   // K-steps of this stage
                     for (int t = 0; t < nt; ++t) {
                         if (!mbar_wait(&tail->acc_empty[sl.idx], sl.phase, abort_flag, p.err)) {
                             ok = false;
@@ -412,13 +413,14 @@ __global__ void __launch_bounds__(TcCfg<BN>::kThreads, 1)
                             for (int c = 0; c < CPT / 2; ++c) y2[h][c] = 0ull;
                     }
                     const uint32_t t_slot = t_lane + (uint32_t)(sl.idx * GPS * BN);
-                    for (int j = 0; j < GPS; ++j) {
+                    const int gs = ks + 1 == KSTAGES ? GLAST : GPS;   // K-groups of this stage
+                    for (int j = 0; j < gs; ++j) {
                         // one group per round, both chunks' loads in flight at once
                         uint32_t r[NP][CPT];
 #pragma unroll
                         for (int h = 0; h < NP; ++h) tmem_ld<CPT>(t_slot + (uint32_t)(j * BN + col0[h]), r[h]);
                         tmem_ld_wait();
-                        if (j + 1 == GPS) {   // the slot is read: release it
+                        if (j + 1 == gs) {   // the slot is read: release it
                             tc_fence_before();
                             __syncwarp();
                             if (lane == 0) mbar_arrive(&tail->acc_empty[sl.idx]);
@@ -608,23 +610,18 @@ int tc_block_n(int Cout, int G) {
     return 0;
 }
 
-// Stage shape: SK bytes of K (a multiple of G dividing Cin, at most NACC/2
-// groups so that at least two accumulator slots exist), swizzle width BK
-// dividing SK, and TPS taps per stage when SK == Cin and there is one column
-// block (as many as keep three
-// stages in the shared-memory budget).
+// Stage shape: SK bytes of K = GPS K-groups (at most NACC/2, so that at least two accumulator slots
+// exist, and at most 256 bytes unless one group is larger); the last stage of a tap holds the
+// remaining groups (its boxes past Cin read zeros and its MMAs and epilogue skip them).  Swizzle
+// width BK divides SK and G.  TPS taps share a stage when one stage holds a tap's whole K and there
+// is one column block (as many as keep three stages in the shared-memory budget).
 static void choose_stage(GemmArgs& a, int BN) {
     const int nacc = std::min(512 / BN, kMaxNacc);
-    const int max_groups = nacc / 2;
-    int sk = a.G;
-    for (int m = max_groups; m >= 1; --m)
-        if (a.Cin % (a.G * m) == 0 && a.G * m <= std::max(a.G, 256)) {
-            sk = a.G * m;
-            break;
-        }
+    const int max_groups = std::max(1, std::min(nacc / 2, std::max(a.G, 256) / a.G));
+    const int gps = std::min(max_groups, a.ng);
+    const int sk = gps * a.G;
     a.SK = sk;
     a.BK = sk % 128 == 0 ? 128 : (sk % 64 == 0 ? 64 : 32);
-    const int gps = sk / a.G;
     const size_t budget = 200 * 1024;
     const size_t per_tap = (size_t)sk * (kBM + BN) + (size_t)gps * (kBM + BN) * 4;
     a.tps = 1;

@@ -99,6 +99,27 @@ bool tc_swap_ok(int T, int Cout);  // the swapped-operand fp32-Y pass applies (T
 
 cudaError_t launch_hadamard_simt(const GemmArgs& a, const int8_t* Vq, const int8_t* Uq, int mode, cudaStream_t st);
 
+// --------------------------------------------- fused small-channel layer (x -> out in one kernel)
+struct FusedArgs {
+    const void* x;            // [N][H][W][Cin] bf16 or fp32
+    int N, H, W, Cin, Cout, TH, TW, G;
+    long T, T_pad;
+    const int8_t* Uq;         // [n2][Cout][Cin]
+    const float* sU;          // [n2][Cin/G][Cout]
+    void* out;                // [N][H][W][Cout] fp32 or bf16
+    int bf16_out;             // 1: bf16 output (round to nearest even), 0: fp32
+    int* err;                 // device error word
+    size_t n_out;             // elements of out (debug-build index checks)
+    int8_t* Vq_dbg;           // debug copies in the staged layouts (or null): Vq [n2][T_pad][Cin],
+    float* sV_dbg;            //   sV [n2][Cin/G][T_pad], Yq [n2][T][Cout], sY [T][Cout/G]
+    int8_t* Yq_dbg;
+    float* sY_dbg;
+};
+// Whether the fused kernel supports these channel counts and group size (the standard point orders only).
+bool fused_small_fits(int Cin, int Cout, int G);
+cudaError_t launch_fused_small(const FusedArgs& a, const TransformArgs& tf, int m, bool bf16_in, int num_sms,
+                               cudaStream_t st);
+
 // ----------------------------------------------------------- output transform
 struct OutputArgs {
     int N, H, W, Cout, TH, TW;

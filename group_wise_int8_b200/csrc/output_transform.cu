@@ -37,22 +37,25 @@ __device__ __forceinline__ uint64_t codes2_to_f2(uint32_t x) {
 }
 
 template <int M, uint64_t MASK, bool SRC_Y32, bool BF16_OUT, bool DEBUG>
-// fp32-Y source: six CTAs per SM (measured faster despite spills: the loads dominate)
-__global__ void __launch_bounds__(128, SRC_Y32 ? 6 : 4)
-    output_transform_kernel(const __grid_constant__ CUtensorMap tmYq, OutputArgs p, TransformArgs tf) {
+__global__ void __launch_bounds__(128, SRC_Y32 ? 3 : 4)
+    output_transform_kernel(const __grid_constant__ CUtensorMap tmY, OutputArgs p, TransformArgs tf) {
     constexpr int N = M + 2, N2 = N * N;
-    // int8 source: the CTA's 256 contiguous bytes of every tap, one 2-D TMA box
+    // The CTA's 128 cout pairs are 256 consecutive elements of every tap's [T][Cout] plane: one 2-D
+    // TMA box of every tap brings them to shared memory (int8 source: 256 bytes per tap, static;
+    // fp32 source: 1 KiB per tap, dynamic), so all of the CTA's Y is in flight at once.
     __shared__ __align__(128) uint8_t ysm[SRC_Y32 ? 16 : 256 * N2];
+    extern __shared__ __align__(128) unsigned char ydyn[];
     __shared__ uint64_t bar;
     __shared__ int load_ok;
     grid_dependents_launch();
     grid_dependency_wait();
-    if (!SRC_Y32) {
+    {
         if (threadIdx.x == 0) {
             sm100::mbar_init(&bar, 1);
             sm100::fence_mbar_init();
-            sm100::mbar_arrive_expect_tx(&bar, 256u * N2);
-            sm100::tma_load_2d(ysm, &tmYq, &bar, (int)(blockIdx.x * 256u), 0);
+            sm100::mbar_arrive_expect_tx(&bar, (SRC_Y32 ? 1024u : 256u) * N2);
+            sm100::tma_load_2d(SRC_Y32 ? static_cast<void*>(ydyn) : static_cast<void*>(ysm), &tmY, &bar,
+                               (int)(blockIdx.x * 256u), 0);
             load_ok = 1;
             const unsigned long long t0 = sm100::globaltimer();
             while (!sm100::mbar_try_wait(&bar, 0))
@@ -87,10 +90,11 @@ __global__ void __launch_bounds__(128, SRC_Y32 ? 6 : 4)
     for (int nu = 0; nu < N; ++nu) {
         uint64_t Yc[N];                            // column nu of Yd: taps xi * N + nu
         if (SRC_Y32) {
+            const float* ys = reinterpret_cast<const float*>(ydyn) + 2 * threadIdx.x;   // + tap * 256
 #pragma unroll
             for (int xi = 0; xi < N; xi += 2) {
-                const float2 a = *reinterpret_cast<const float2*>(p.Y32 + base + (size_t)(xi * N + nu) * tstride);
-                const float2 b = *reinterpret_cast<const float2*>(p.Y32 + base + (size_t)((xi + 1) * N + nu) * tstride);
+                const float2 a = *reinterpret_cast<const float2*>(ys + (xi * N + nu) * 256);
+                const float2 b = *reinterpret_cast<const float2*>(ys + ((xi + 1) * N + nu) * 256);
                 const Quad qd = quant4(a.x, a.y, b.x, b.y, qs);
                 Yc[xi] = f2_mul(s2, qd.k01);
                 Yc[xi + 1] = f2_mul(s2, qd.k23);
@@ -377,18 +381,21 @@ cudaError_t launch_m(const OutputArgs& a, const TransformArgs& tf, bool src_y32,
     const dim3 grid((unsigned)((threads + 127) / 128));
     CUtensorMap tm;
     std::memset(&tm, 0, sizeof(tm));
-    if (!src_y32) {   // Yq [n2][T*Cout] bytes; box 256 x n2 (a CTA's 128 cout pairs, every tap)
+    const bool split = output_transform_split(a.T, a.Cout, src_y32, a.ytap != 0, a.num_sms);
+    if (!a.ytap && !split) {   // Yq / Y32 as [n2][T*Cout]; box 256 x n2 (a CTA's 128 cout pairs, every tap)
+        const cuuint64_t es = src_y32 ? 4 : 1;
         const cuuint64_t dims[2] = {(cuuint64_t)a.T * a.Cout, (cuuint64_t)a.n2};
-        const cuuint64_t strides[1] = {(cuuint64_t)a.T * a.Cout};
+        const cuuint64_t strides[1] = {(cuuint64_t)a.T * a.Cout * es};
         const cuuint32_t box[2] = {256u, (cuuint32_t)a.n2};
-        if (!make_tensor_map(&tm, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, a.Yq, dims, strides, box,
-                             CU_TENSOR_MAP_SWIZZLE_NONE))
+        if (!make_tensor_map(&tm, src_y32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_UINT8, 2,
+                             src_y32 ? static_cast<const void*>(a.Y32) : static_cast<const void*>(a.Yq), dims,
+                             strides, box, CU_TENSOR_MAP_SWIZZLE_NONE))
             return cudaErrorInvalidValue;
     }
     if (a.ytap)
         return bf16_out ? launch_dependent(output_transform_ytap_kernel<M, MASK, true>, grid, dim3(128), 0, st, a, tf)
                         : launch_dependent(output_transform_ytap_kernel<M, MASK, false>, grid, dim3(128), 0, st, a, tf);
-    if (output_transform_split(a.T, a.Cout, src_y32, a.ytap != 0, a.num_sms)) {   // too few items for one thread each
+    if (split) {   // too few items for one thread each
         constexpr int IPW = 32 / (M + 2);
         const dim3 sgrid((unsigned)((threads + 4 * IPW - 1) / (4 * IPW)));
 #define WINO_SPLIT_LAUNCH(BF, DBG) \
@@ -400,8 +407,17 @@ cudaError_t launch_m(const OutputArgs& a, const TransformArgs& tf, bool src_y32,
         }
 #undef WINO_SPLIT_LAUNCH
     }
-#define WINO_OUT_LAUNCH(Y32, BF, DBG) \
-    return launch_dependent(output_transform_kernel<M, MASK, Y32, BF, DBG>, grid, dim3(128), 0, st, tm, a, tf)
+    const size_t dsmem = src_y32 ? (size_t)1024 * a.n2 : 0;   // fp32 source: 1 KiB per tap
+#define WINO_OUT_LAUNCH(Y32, BF, DBG)                                                                          \
+    do {                                                                                                     \
+        auto kern = output_transform_kernel<M, MASK, Y32, BF, DBG>;                                          \
+        if (Y32) {                                                                                           \
+            const cudaError_t fe = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,   \
+                                                        (int)dsmem);                                         \
+            if (fe != cudaSuccess) return fe;                                                                \
+        }                                                                                                    \
+        return launch_dependent(kern, grid, dim3(128), dsmem, st, tm, a, tf);                                \
+    } while (0)
     if (src_y32) {
         if (bf16_out) {
             if (debug) WINO_OUT_LAUNCH(true, true, true); else WINO_OUT_LAUNCH(true, true, false);

@@ -57,6 +57,19 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
     return ok != 0;
 }
 
+// Non-blocking test of the phase with the given parity (never suspends the thread).
+__device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}\n"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
 // Waits for the phase with the given parity.  Returns false if the CTA's
 // abort flag is raised or the time limit expires (then it raises the flag and
 // records the error in the global error word).
@@ -154,6 +167,14 @@ __device__ __forceinline__ void mma_commit(uint64_t* bar) {
 }
 
 __device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
+// Ties registers written by an earlier tcgen05.ld to a point after tmem_ld_wait(): every later use
+// reads the value this (empty, ordered) statement passes through, so none can move above the wait.
+template <int NC>
+__device__ __forceinline__ void tmem_regs_ready(uint32_t (&r)[NC]) {
+#pragma unroll
+    for (int i = 0; i < NC; ++i) asm volatile("" : "+r"(r[i]));
+}
 
 // 32 lanes x NC consecutive 32-bit columns (this warp's lane quadrant), NC = 4, 8, 16 or 32.
 #define WINO_R8(o) "=r"(r[o + 0]), "=r"(r[o + 1]), "=r"(r[o + 2]), "=r"(r[o + 3]), "=r"(r[o + 4]), "=r"(r[o + 5]), \

@@ -37,7 +37,8 @@ YPATH_AUTO, YPATH_RECOMPUTE, YPATH_Y32 = 0, 1, 2
 GEMM_AUTO, GEMM_TCGEN05, GEMM_SIMT = 0, 1, 2
 DEBUG_YQ, DEBUG_ACC32, DEBUG_FORCE_TIMEOUT, DEBUG_GUARDS, DEBUG_SHRINK_BOUNDS = 1, 2, 4, 8, 16
 YGROUPS_TILE, YGROUPS_TAP = 0, 1
-VARIANT_SWAPPED_GEMM, VARIANT_SPLIT_INPUT, VARIANT_SPLIT_OUTPUT = 1, 2, 4
+VARIANT_SWAPPED_GEMM, VARIANT_SPLIT_INPUT, VARIANT_SPLIT_OUTPUT, VARIANT_FUSED = 1, 2, 4, 8
+FUSED_AUTO, FUSED_OFF, FUSED_ON = 0, 1, 2
 DUMP_VQ, DUMP_SV, DUMP_YQ, DUMP_SY, DUMP_Y32, DUMP_ACC32 = range(6)
 NOALLOC_SCRATCH_BYTES = 64 << 20   # WINO_NOALLOC_SCRATCH_BYTES
 
@@ -62,7 +63,7 @@ class WinoError(RuntimeError):
 class Opts(ctypes.Structure):
     _fields_ = [("y_path", ctypes.c_int), ("gemm", ctypes.c_int), ("debug", ctypes.c_int),
                 ("y_groups", ctypes.c_int), ("x_int8", ctypes.c_int), ("int8_transforms", ctypes.c_int),
-                ("reserved", ctypes.c_int * 2)]
+                ("fused", ctypes.c_int), ("reserved", ctypes.c_int)]
 
 
 _libs = {}
@@ -148,14 +149,15 @@ class Plan:
 
     def __init__(self, m: int, points: Sequence[float], S_B=None, S_G=None, group: int = 32,
                  y_path: int = YPATH_AUTO, gemm: int = GEMM_AUTO, debug: int = 0, y_groups: int = YGROUPS_TILE,
-                 x_int8: bool = False, int8_transforms: bool = False, variant: str = "release"):
+                 x_int8: bool = False, int8_transforms: bool = False, variant: str = "release",
+                 fused: int = FUSED_AUTO):
         L = load_library(variant=variant)
         self._L = L
         n = m + 2
         pts = (ctypes.c_double * n)(*[float(p) for p in points])
         sb = None if S_B is None else (ctypes.c_float * n)(*[float(v) for v in S_B])
         sg = None if S_G is None else (ctypes.c_float * n)(*[float(v) for v in S_G])
-        opts = Opts(y_path, gemm, debug, y_groups, int(x_int8), int(int8_transforms))
+        opts = Opts(y_path, gemm, debug, y_groups, int(x_int8), int(int8_transforms), int(fused))
         h = _vp()
         rc = L.wino_plan(ctypes.byref(h), m, pts, sb, sg, group, ctypes.byref(opts))
         if rc != OK:

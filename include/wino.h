@@ -103,8 +103,23 @@ typedef struct wino_opts {
                       (same passage): each entry becomes s * clamp(rne(M/s), +-127) in fp32,
                       s = max|M|/127, at plan time; G stays fp64 (the weights are quantised
                       after their transform) */
-    int reserved[2];
+    int fused;     /* WINO_FUSED_*: the one-kernel path for small channel counts */
+    int reserved;
 } wino_opts;
+
+/* The fused path (Cin = Cout = 64 with G = 32 or 64, or Cin = Cout = G = 32; the
+ * standard point orders; tile-spanning Y groups, no int8 x, tcgen05 GEMM, automatic Y
+ * path, no accumulator dump): one kernel runs the input transform, both GEMM passes of the recompute path
+ * and the output transform on units of 16 tiles, with Vq and Yq kept in shared
+ * memory; results are identical to the staged kernels.  ON takes it wherever it
+ * applies; AUTO and OFF take the staged kernels (on the configured layers the
+ * fused kernel is slower: its units of 16 tiles run their phases one after the
+ * other, and each stage of 4 taps waits on its own TMA and accumulator
+ * handoffs).  With WINO_DEBUG_YQ the
+ * kernel also writes Vq, sV, Yq and sY to the workspace for wino_debug_dump. */
+#define WINO_FUSED_AUTO 0
+#define WINO_FUSED_OFF 1
+#define WINO_FUSED_ON 2
 
 /* Y groups (the input of the output transform).  TILE (default, the reading the
  * method needs): one scale per (tile, G consecutive couts) spanning all n*n taps.
@@ -300,6 +315,7 @@ int wino_resolved_config(wino_plan_t plan, int N, int H, int W, int Cin, int Cou
 #define WINO_VARIANT_SWAPPED_GEMM 1
 #define WINO_VARIANT_SPLIT_INPUT 2
 #define WINO_VARIANT_SPLIT_OUTPUT 4
+#define WINO_VARIANT_FUSED 8
 int wino_resolved_variants(wino_plan_t plan, int N, int H, int W, int Cin, int Cout, int* flags);
 
 /* Number of kernels one wino_conv2d_int8 call of this shape launches. */

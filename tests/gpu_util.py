@@ -27,11 +27,12 @@ def weight_dumps(plan, wt: torch.Tensor, Cin: int, Cout: int):
 
 
 def run_gpu(m, pts, sb, sg, G, x_f32, x_bits, w, out_dtype=torch.float32, y_path=wino.YPATH_AUTO,
-            gemm=wino.GEMM_AUTO, debug=0, y_groups=wino.YGROUPS_TILE, x_int8=False, int8_transforms=False):
+            gemm=wino.GEMM_AUTO, debug=0, y_groups=wino.YGROUPS_TILE, x_int8=False, int8_transforms=False,
+            fused=wino.FUSED_AUTO):
     N, H, W, Cin = x_f32.shape
     Cout = w.shape[0]
     plan = wino.Plan(m, pts, sb, sg, G, y_path=y_path, gemm=gemm, debug=debug, y_groups=y_groups,
-                     x_int8=x_int8, int8_transforms=int8_transforms)
+                     x_int8=x_int8, int8_transforms=int8_transforms, fused=fused)
     x = to_device_input(x_f32, x_bits)
     wt = plan.transform_weights(torch.from_numpy(w).cuda())
     ws = torch.empty(plan.workspace_bytes(N, H, W, Cin, Cout), dtype=torch.uint8, device="cuda")
@@ -40,10 +41,14 @@ def run_gpu(m, pts, sb, sg, G, x_f32, x_bits, w, out_dtype=torch.float32, y_path
     assert plan.check_device_error(ws, N, H, W, Cin, Cout) == wino.OK
     res = {"out": out.float().cpu().numpy(), "plan": plan}
     res["Uq"], res["sU"] = weight_dumps(plan, wt, Cin, Cout)
-    res["Vq"] = plan.debug_dump(ws, N, H, W, Cin, Cout, wino.DUMP_VQ)
-    res["sV"] = plan.debug_dump(ws, N, H, W, Cin, Cout, wino.DUMP_SV)
     yp, gm = plan.resolved_config(N, H, W, Cin, Cout)
     res["y_path"], res["gemm"] = yp, gm
+    # the fused path keeps Vq and Yq on chip: they exist only as its debug copies
+    fused = bool(plan.resolved_variants(N, H, W, Cin, Cout) & wino.VARIANT_FUSED)
+    if fused and not debug & wino.DEBUG_YQ:
+        return res
+    res["Vq"] = plan.debug_dump(ws, N, H, W, Cin, Cout, wino.DUMP_VQ)
+    res["sV"] = plan.debug_dump(ws, N, H, W, Cin, Cout, wino.DUMP_SV)
     if debug & wino.DEBUG_YQ or yp == wino.YPATH_RECOMPUTE:
         res["Yq"] = plan.debug_dump(ws, N, H, W, Cin, Cout, wino.DUMP_YQ)
     if debug & wino.DEBUG_YQ:
