@@ -104,7 +104,7 @@ Layout make_layout(const wino_plan_s* p, int N, int H, int W, int Cin, int Cout)
     L.gemm = p->opts.gemm == WINO_GEMM_AUTO ? WINO_GEMM_TCGEN05 : p->opts.gemm;
     if (L.gemm == WINO_GEMM_TCGEN05 && tc_block_n(Cout, p->G) == 0) L.gemm = WINO_GEMM_SIMT;
     L.ytap = p->opts.y_groups == WINO_YGROUPS_TAP;
-    // at most 32 tiles: the fp32-Y pass runs with swapped operands (output channels on the MMA's
+    // at most 80 tiles: the fp32-Y pass runs with swapped operands (output channels on the MMA's
     // 128 rows), unless the recompute path was asked for
     L.swap = L.gemm == WINO_GEMM_TCGEN05 && tc_swap_ok((int)std::min<long>(L.T, 1 << 30), Cout) &&
              p->opts.y_path != WINO_YPATH_RECOMPUTE;

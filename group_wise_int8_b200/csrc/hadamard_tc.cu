@@ -51,6 +51,7 @@ using namespace sm100;
 constexpr int kBM = 128;
 constexpr int kMaxStages = 8;
 constexpr int kMaxNacc = 8;
+constexpr int kSwapMaxTiles = 80;   // the swapped pass's N is 16, 32 or 80 tiles
 
 template <int BN>
 struct TcCfg {
@@ -416,29 +417,43 @@ __global__ void __launch_bounds__(TcCfg<BN>::kThreads, 1)
                     const int gs = ks + 1 == KSTAGES ? GLAST : GPS;   // K-groups of this stage
                     for (int j = 0; j < gs; ++j) {
                         // one group per round, both chunks' loads in flight at once
-                        uint32_t r[NP][CPT];
+                        // chunks of more than 16 columns are loaded one at a time (register pressure)
+                        constexpr int NR = CPT > 16 ? 1 : NP;
+                        uint32_t r[NR][CPT];
+                        if constexpr (NR == NP) {
 #pragma unroll
-                        for (int h = 0; h < NP; ++h) tmem_ld<CPT>(t_slot + (uint32_t)(j * BN + col0[h]), r[h]);
-                        tmem_ld_wait();
-                        if (j + 1 == gs) {   // the slot is read: release it
-                            tc_fence_before();
-                            __syncwarp();
-                            if (lane == 0) mbar_arrive(&tail->acc_empty[sl.idx]);
+                            for (int h = 0; h < NP; ++h) tmem_ld<CPT>(t_slot + (uint32_t)(j * BN + col0[h]), r[h]);
+                            tmem_ld_wait();
+                            if (j + 1 == gs) {   // the slot is read: release it
+                                tc_fence_before();
+                                __syncwarp();
+                                if (lane == 0) mbar_arrive(&tail->acc_empty[sl.idx]);
+                            }
                         }
                         const float sv = svs[(t * GPS + j) * kBM];
                         const uint64_t sv2 = f2_pack(sv, sv);
 #pragma unroll
                         for (int h = 0; h < NP; ++h) {
+                            const int hr = NR == NP ? h : 0;
+                            if constexpr (NR != NP) {
+                                tmem_ld<CPT>(t_slot + (uint32_t)(j * BN + col0[h]), r[0]);
+                                tmem_ld_wait();
+                                if (h + 1 == NP && j + 1 == gs) {   // the slot is read: release it
+                                    tc_fence_before();
+                                    __syncwarp();
+                                    if (lane == 0) mbar_arrive(&tail->acc_empty[sl.idx]);
+                                }
+                            }
                             const float4* su4 = reinterpret_cast<const float4*>(sus + (t * GPS + j) * BN + col0[h]);
 #pragma unroll
                             for (int c4 = 0; c4 < CPT / 4; ++c4) {
                                 const float4 uu = su4[c4];
                                 // (float)acc exactly: acc + 1.5*2^23 in the integer unit, then - 1.5*2^23 (|acc| < 2^22)
-                                const uint64_t a0 = f2_add(f2_pack(__uint_as_float(r[h][4 * c4 + 0] + kRoundMagicBits),
-                                                                   __uint_as_float(r[h][4 * c4 + 1] + kRoundMagicBits)),
+                                const uint64_t a0 = f2_add(f2_pack(__uint_as_float(r[hr][4 * c4 + 0] + kRoundMagicBits),
+                                                                   __uint_as_float(r[hr][4 * c4 + 1] + kRoundMagicBits)),
                                                            neg_magic2);
-                                const uint64_t a1 = f2_add(f2_pack(__uint_as_float(r[h][4 * c4 + 2] + kRoundMagicBits),
-                                                                   __uint_as_float(r[h][4 * c4 + 3] + kRoundMagicBits)),
+                                const uint64_t a1 = f2_add(f2_pack(__uint_as_float(r[hr][4 * c4 + 2] + kRoundMagicBits),
+                                                                   __uint_as_float(r[hr][4 * c4 + 3] + kRoundMagicBits)),
                                                            neg_magic2);
                                 y2[h][2 * c4 + 0] = f2_fma(a0, f2_mul(sv2, f2_pack(uu.x, uu.y)), y2[h][2 * c4 + 0]);
                                 y2[h][2 * c4 + 1] = f2_fma(a1, f2_mul(sv2, f2_pack(uu.z, uu.w)), y2[h][2 * c4 + 1]);
@@ -449,10 +464,10 @@ __global__ void __launch_bounds__(TcCfg<BN>::kThreads, 1)
                                 for (int c = 0; c < CPT; ++c) {
                                     if (SWAP) {   // row = output channel, column = tile
                                         const size_t di = (((size_t)tap * p.T + colg[h] + c) * p.Cout + row) * p.ng + jg;
-                                        if (colg[h] + c < p.T && in_bounds(di, p.n_acc, p.err)) p.acc[di] = (int)r[h][c];
+                                        if (colg[h] + c < p.T && in_bounds(di, p.n_acc, p.err)) p.acc[di] = (int)r[hr][c];
                                     } else {
                                         const size_t di = (((size_t)tap * p.T + row) * p.Cout + colg[h] + c) * p.ng + jg;
-                                        if (in_bounds(di, p.n_acc, p.err)) p.acc[di] = (int)r[h][c];
+                                        if (in_bounds(di, p.n_acc, p.err)) p.acc[di] = (int)r[hr][c];
                                     }
                                 }
                             }
@@ -466,7 +481,7 @@ __global__ void __launch_bounds__(TcCfg<BN>::kThreads, 1)
                         float y[CPT];
 #pragma unroll
                         for (int c = 0; c < CPT / 2; ++c) f2_unpack(y2[h][c], y[2 * c], y[2 * c + 1]);
-                        if (MODE == kModeQuant) {
+                        if constexpr (MODE == kModeQuant) {
                             const size_t yi = ((size_t)tap * p.T + row) * p.Cout + colg[h];
                             if (valid && in_bounds(yi + CPT - 1, p.n_y, p.err)) {
                                 uint32_t q[CPT / 4];
@@ -481,7 +496,7 @@ __global__ void __launch_bounds__(TcCfg<BN>::kThreads, 1)
                                             make_uint4(q[4 * c], q[4 * c + 1], q[4 * c + 2], q[4 * c + 3]);
                                 }
                             }
-                        } else if (SWAP) {
+                        } else if constexpr (SWAP) {
                             // one output channel, CPT tiles: lanes hold consecutive channels, so each
                             // store instruction writes 32 consecutive floats of one tile and tap
 #pragma unroll
@@ -635,14 +650,15 @@ static void choose_stage(GemmArgs& a, int BN) {
     a.stages = stages > kMaxStages ? kMaxStages : (stages < 2 ? 2 : stages);
 }
 
-bool tc_swap_ok(int T, int Cout) { return T <= 32 && Cout % kBM == 0; }
+bool tc_swap_ok(int T, int Cout) { return T <= kSwapMaxTiles && Cout % kBM == 0; }
 
 cudaError_t launch_hadamard_tc(GemmArgs a, const int8_t* Vq, const int8_t* Uq, int mode, int num_sms,
                                cudaStream_t st, int* launches) {
     const bool swap = a.swap_ab != 0;
     if (swap && (!tc_swap_ok(a.T, a.Cout) || mode != kModeY32)) return cudaErrorInvalidValue;
-    // swapped: 128 output channels per row block, the tiles (at most 32) as the MMA's N
-    const int BN = swap ? (a.T <= 16 ? 16 : 32) : tc_block_n(a.Cout, a.G);
+    // swapped: 128 output channels per row block, the tiles (at most 80) as the MMA's N: 16, 32 or 80
+    // (the widths in between spill registers in the epilogue)
+    const int BN = swap ? (a.T <= 16 ? 16 : (a.T <= 32 ? 32 : 80)) : tc_block_n(a.Cout, a.G);
     if (BN == 0) return cudaErrorInvalidValue;
     EncodeTiledFn enc = get_encode_fn();
     if (!enc) return cudaErrorNotSupported;
@@ -690,7 +706,14 @@ cudaError_t launch_hadamard_tc(GemmArgs a, const int8_t* Vq, const int8_t* Uq, i
             return cudaErrorInvalidValue;
     }
     if (launches) ++*launches;
-    if (swap) return BN == 16 ? launch_swap<16>(a, m, mode, num_sms, st) : launch_swap<32>(a, m, mode, num_sms, st);
+    if (swap) {
+        switch (BN) {
+            case 16: return launch_swap<16>(a, m, mode, num_sms, st);
+            case 32: return launch_swap<32>(a, m, mode, num_sms, st);
+            case 80: return launch_swap<80>(a, m, mode, num_sms, st);
+            default: return cudaErrorInvalidValue;
+        }
+    }
     if (BN == 64) return launch_bn<64>(a, m, mode, num_sms, st);
     return launch_bn<32>(a, m, mode, num_sms, st);
 }

@@ -36,51 +36,59 @@ __device__ __forceinline__ uint64_t codes2_to_f2(uint32_t x) {
     return f2_sub(f2_pack(__uint_as_float(lo), __uint_as_float(hi)), f2_pack(off, off));
 }
 
+// Bounded wait for one column's TMA box (records a timeout in the error word).
+__device__ __forceinline__ bool column_wait(uint64_t* bar, int* err) {
+    if (sm100::mbar_try_wait(bar, 0)) return true;
+    const unsigned long long t0 = sm100::globaltimer();
+    while (!sm100::mbar_try_wait(bar, 0))
+        if (sm100::globaltimer() - t0 > sm100::kWaitLimitNs) {
+            atomicCAS(err, 0, sm100::kDevErrTimeout);
+            return false;
+        }
+    return true;
+}
+
 template <int M, uint64_t MASK, bool SRC_Y32, bool BF16_OUT, bool DEBUG>
 __global__ void __launch_bounds__(128, SRC_Y32 ? 3 : 4)
     output_transform_kernel(const __grid_constant__ CUtensorMap tmY, OutputArgs p, TransformArgs tf) {
     constexpr int N = M + 2, N2 = N * N;
-    // The CTA's 128 cout pairs are 256 consecutive elements of every tap's [T][Cout] plane: one 2-D
-    // TMA box of every tap brings them to shared memory (int8 source: 256 bytes per tap, static;
-    // fp32 source: 1 KiB per tap, dynamic), so all of the CTA's Y is in flight at once.
+    // The CTA's 128 cout pairs are 256 consecutive elements of every tap's [T][Cout] plane.  One 3-D
+    // TMA box per column nu of Y (taps xi * N + nu, every xi) brings them to shared memory as
+    // [nu][xi][256] (int8 source: 256 bytes per tap, static; fp32 source: 1 KiB per tap, dynamic),
+    // each column on its own barrier, so the transform of column nu overlaps the later columns' loads.
     __shared__ __align__(128) uint8_t ysm[SRC_Y32 ? 16 : 256 * N2];
     extern __shared__ __align__(128) unsigned char ydyn[];
-    __shared__ uint64_t bar;
-    __shared__ int load_ok;
+    __shared__ uint64_t bar[N];
+    constexpr uint32_t kColBytes = (SRC_Y32 ? 1024u : 256u) * N;
     grid_dependents_launch();
     grid_dependency_wait();
-    {
-        if (threadIdx.x == 0) {
-            sm100::mbar_init(&bar, 1);
-            sm100::fence_mbar_init();
-            sm100::mbar_arrive_expect_tx(&bar, (SRC_Y32 ? 1024u : 256u) * N2);
-            sm100::tma_load_2d(SRC_Y32 ? static_cast<void*>(ydyn) : static_cast<void*>(ysm), &tmY, &bar,
-                               (int)(blockIdx.x * 256u), 0);
-            load_ok = 1;
-            const unsigned long long t0 = sm100::globaltimer();
-            while (!sm100::mbar_try_wait(&bar, 0))
-                if (sm100::globaltimer() - t0 > sm100::kWaitLimitNs) {
-                    load_ok = 0;
-                    atomicCAS(p.err, 0, sm100::kDevErrTimeout);
-                    break;
-                }
+    if (threadIdx.x == 0) {
+        for (int nu = 0; nu < N; ++nu) sm100::mbar_init(&bar[nu], 1);
+        sm100::fence_mbar_init();
+        for (int nu = 0; nu < N; ++nu) {
+            sm100::mbar_arrive_expect_tx(&bar[nu], kColBytes);
+            unsigned char* dst = (SRC_Y32 ? ydyn : ysm) + (size_t)nu * kColBytes;
+            sm100::tma_load_3d(dst, &tmY, &bar[nu], (int)(blockIdx.x * 256u), nu, 0);
         }
-        __syncthreads();
-        if (!load_ok) return;   // uniform; the host reads the error word
     }
+    __syncthreads();
     const long i = (long)blockIdx.x * blockDim.x + threadIdx.x;
     const int cpairs = p.Cout >> 1;
     const long t = i / cpairs;
     const int co = 2 * (int)(i - t * cpairs);
-    if (t >= p.T) return;
     const int cg = co / p.G;
     const size_t base = (size_t)t * p.Cout + co;   // Yq / Y32 are tap-major [n2][T][Cout]
     const size_t tstride = (size_t)p.T * p.Cout;
     // every Y element this thread touches lies in [base, base + (N2 - 1) * tstride + 1]
-    if (!in_bounds((size_t)t * p.ngo + cg, p.n_amax, p.err) ||
+    if (t >= p.T || !in_bounds((size_t)t * p.ngo + cg, p.n_amax, p.err) ||
         ((SRC_Y32 || DEBUG) && !in_bounds(base + (size_t)(N2 - 1) * tstride + 1, p.n_y, p.err)) ||
-        (DEBUG && !in_bounds((size_t)t * p.ngo + cg, p.n_sy, p.err)))
+        (DEBUG && !in_bounds((size_t)t * p.ngo + cg, p.n_sy, p.err))) {
+        // an idle thread 0 still sees every load land before the CTA's shared memory is released
+        if (threadIdx.x == 0)
+            for (int nu = 0; nu < N; ++nu)
+                if (!column_wait(&bar[nu], p.err)) break;
         return;
+    }
     const QScale qs = make_qscale(__uint_as_float(p.amax[(size_t)t * p.ngo + cg]));
     if (DEBUG && co % p.G == 0) p.sY_dbg[(size_t)t * p.ngo + cg] = qs.s;
     const uint64_t s2 = f2_pack(qs.s, qs.s);
@@ -89,12 +97,13 @@ __global__ void __launch_bounds__(128, SRC_Y32 ? 3 : 4)
 #pragma unroll
     for (int nu = 0; nu < N; ++nu) {
         uint64_t Yc[N];                            // column nu of Yd: taps xi * N + nu
+        if (!column_wait(&bar[nu], p.err)) return;   // only on a timeout (error word set)
         if (SRC_Y32) {
-            const float* ys = reinterpret_cast<const float*>(ydyn) + 2 * threadIdx.x;   // + tap * 256
+            const float* ys = reinterpret_cast<const float*>(ydyn) + 2 * threadIdx.x;   // + (nu * N + xi) * 256
 #pragma unroll
             for (int xi = 0; xi < N; xi += 2) {
-                const float2 a = *reinterpret_cast<const float2*>(ys + (xi * N + nu) * 256);
-                const float2 b = *reinterpret_cast<const float2*>(ys + ((xi + 1) * N + nu) * 256);
+                const float2 a = *reinterpret_cast<const float2*>(ys + (nu * N + xi) * 256);
+                const float2 b = *reinterpret_cast<const float2*>(ys + (nu * N + xi + 1) * 256);
                 const Quad qd = quant4(a.x, a.y, b.x, b.y, qs);
                 Yc[xi] = f2_mul(s2, qd.k01);
                 Yc[xi + 1] = f2_mul(s2, qd.k23);
@@ -108,7 +117,7 @@ __global__ void __launch_bounds__(128, SRC_Y32 ? 3 : 4)
         } else {
 #pragma unroll
             for (int xi = 0; xi < N; ++xi) {
-                const uint32_t x = *reinterpret_cast<const uint16_t*>(ysm + (xi * N + nu) * 256 + 2 * threadIdx.x);
+                const uint32_t x = *reinterpret_cast<const uint16_t*>(ysm + (nu * N + xi) * 256 + 2 * threadIdx.x);
                 Yc[xi] = f2_mul(s2, codes2_to_f2(x));
             }
         }
@@ -382,12 +391,13 @@ cudaError_t launch_m(const OutputArgs& a, const TransformArgs& tf, bool src_y32,
     CUtensorMap tm;
     std::memset(&tm, 0, sizeof(tm));
     const bool split = output_transform_split(a.T, a.Cout, src_y32, a.ytap != 0, a.num_sms);
-    if (!a.ytap && !split) {   // Yq / Y32 as [n2][T*Cout]; box 256 x n2 (a CTA's 128 cout pairs, every tap)
+    if (!a.ytap && !split) {   // Yq / Y32 as [xi][nu][T*Cout]; box 256 x 1 x N (a CTA's 128 cout pairs, one column)
         const cuuint64_t es = src_y32 ? 4 : 1;
-        const cuuint64_t dims[2] = {(cuuint64_t)a.T * a.Cout, (cuuint64_t)a.n2};
-        const cuuint64_t strides[1] = {(cuuint64_t)a.T * a.Cout * es};
-        const cuuint32_t box[2] = {256u, (cuuint32_t)a.n2};
-        if (!make_tensor_map(&tm, src_y32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_UINT8, 2,
+        const cuuint64_t n = (cuuint64_t)(M + 2);
+        const cuuint64_t dims[3] = {(cuuint64_t)a.T * a.Cout, n, n};
+        const cuuint64_t strides[2] = {(cuuint64_t)a.T * a.Cout * es, (cuuint64_t)a.T * a.Cout * es * n};
+        const cuuint32_t box[3] = {256u, 1u, (cuuint32_t)n};
+        if (!make_tensor_map(&tm, src_y32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_UINT8, 3,
                              src_y32 ? static_cast<const void*>(a.Y32) : static_cast<const void*>(a.Yq), dims,
                              strides, box, CU_TENSOR_MAP_SWIZZLE_NONE))
             return cudaErrorInvalidValue;

@@ -176,7 +176,7 @@ __device__ __forceinline__ void tmem_regs_ready(uint32_t (&r)[NC]) {
     for (int i = 0; i < NC; ++i) asm volatile("" : "+r"(r[i]));
 }
 
-// 32 lanes x NC consecutive 32-bit columns (this warp's lane quadrant), NC = 4, 8, 16 or 32.
+// 32 lanes x NC consecutive 32-bit columns (this warp's lane quadrant), NC = 4, 8, 12, 16, 20 or 32.
 #define WINO_R8(o) "=r"(r[o + 0]), "=r"(r[o + 1]), "=r"(r[o + 2]), "=r"(r[o + 3]), "=r"(r[o + 4]), "=r"(r[o + 5]), \
                    "=r"(r[o + 6]), "=r"(r[o + 7])
 template <int NC>
@@ -210,6 +210,17 @@ __device__ __forceinline__ void tmem_ld<32>(uint32_t taddr, uint32_t (&r)[32]) {
         : "r"(taddr));
 }
 #undef WINO_R8
+// Widths between the native ones, as two loads (the second at the following columns).
+template <int NA, int NB, int NC>
+__device__ __forceinline__ void tmem_ld_pair(uint32_t taddr, uint32_t (&r)[NC]) {
+    static_assert(NA + NB == NC, "split widths");
+    tmem_ld<NA>(taddr, *reinterpret_cast<uint32_t(*)[NA]>(&r[0]));
+    tmem_ld<NB>(taddr + NA, *reinterpret_cast<uint32_t(*)[NB]>(&r[NA]));
+}
+template <>
+__device__ __forceinline__ void tmem_ld<12>(uint32_t taddr, uint32_t (&r)[12]) { tmem_ld_pair<8, 4>(taddr, r); }
+template <>
+__device__ __forceinline__ void tmem_ld<20>(uint32_t taddr, uint32_t (&r)[20]) { tmem_ld_pair<16, 4>(taddr, r); }
 
 // Shared-memory matrix descriptor, K-major operand, swizzle of `sw_bytes`
 // (32, 64 or 128) equal to the row pitch; 8-row groups are 8 * sw_bytes apart.

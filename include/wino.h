@@ -204,7 +204,7 @@ size_t wino_workspace_bytes(wino_plan_t plan, int N, int H, int W, int Cin, int 
  * Launches (with x_int8: the quantisation of x, then) the input transform, the
  * Hadamard GEMM (one or two passes) and the output transform on stream.
  * Kernel variants are chosen by shape and give identical bytes: with at most
- * 32 tiles and Cout a multiple of 128, y_path AUTO resolves to Y32 and the GEMM
+ * 80 tiles and Cout a multiple of 128, y_path AUTO resolves to Y32 and the GEMM
  * pass runs with swapped operands (output channels on the MMA rows); layers
  * with few tiles per SM run split transform kernels (more threads per tile).
  * The call returns after the launches (asynchronous).

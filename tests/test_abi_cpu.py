@@ -109,11 +109,14 @@ def test_plan_int8_transforms_match_oracle(lib, m, pts, scaled):
 
 
 def test_short_layers_take_the_fp32_y_path(lib):
-    """At most 32 tiles with Cout a multiple of 128: AUTO resolves to the fp32-Y path (whose GEMM
+    """At most 80 tiles with Cout a multiple of 128: AUTO resolves to the fp32-Y path (whose GEMM
     pass runs with swapped operands); an explicit recompute request is kept."""
     auto = wino.Plan(6, synth.POINTS_F6, None, None, 64)
     assert auto.resolved_config(2, 8, 8, 1280, 1280)[0] == wino.YPATH_Y32          # T = 8
     assert auto.resolved_config(2, 16, 16, 1280, 1280)[0] == wino.YPATH_Y32        # T = 18
+    for n, swapped in ((8, True), (9, False)):                                       # T = 72, 81
+        assert bool(auto.resolved_variants(n, 16, 16, 1280, 1280) & wino.VARIANT_SWAPPED_GEMM) == swapped
+    assert auto.resolved_variants(8, 16, 16, 1280, 320) & wino.VARIANT_SWAPPED_GEMM == 0   # Cout % 128 != 0
     rec = wino.Plan(6, synth.POINTS_F6, None, None, 64, y_path=wino.YPATH_RECOMPUTE)
     assert rec.resolved_config(2, 8, 8, 1280, 1280)[0] == wino.YPATH_RECOMPUTE
     assert rec.launches_per_call(2, 8, 8, 1280, 1280) == 4

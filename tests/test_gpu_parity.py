@@ -50,6 +50,13 @@ CASES = {
     "f6_many_tiles": (6, P6, 24, 56, 56, 64, 32, 32, "bf16", "relu_normal", "loguniform"),
     # the widest concatenated-skip conv of the SD-shaped stack: 40 K-groups per tap
     "f6_cin2560_cout1280": (6, P6, 2, 16, 16, 2560, 1280, 64, "bf16", "student_t_outliers", "loguniform"),
+    # the swapped fp32-Y pass at each of its wider MMA N: 45 tiles (N 48), 64 tiles (N 64), 72 tiles
+    # of ragged images with a ragged last K stage (N 80), exactly 80 tiles, and 81 tiles (not swapped)
+    "f6_swap_n48": (6, P6, 5, 16, 16, 256, 256, 64, "bf16", "relu_normal", "loguniform"),
+    "f4_swap_n64": (4, P4, 1, 30, 30, 128, 128, 32, "f32", "normal", "loguniform"),
+    "f6_swap_n80_ragged": (6, P6, 2, 34, 35, 320, 256, 64, "bf16", "student_t_outliers", "loguniform"),
+    "f4_swap_n80_full": (4, P4, 5, 16, 16, 128, 128, 64, "bf16", "relu_normal", "loguniform"),
+    "f6_81_tiles": (6, P6, 1, 54, 54, 128, 128, 64, "bf16", "relu_normal", "loguniform"),
 }
 
 
