@@ -61,12 +61,7 @@ UNIT = "TFLOP/s"
 # (dram__bytes_read.sum + dram__bytes_write.sum), keyed by (layer shape, kernel);
 # the summary with its command line is the named file under profiles/.  An
 # entry is removed whenever its kernel changes.
-NCU_TRAFFIC = {
-    # profiles/hadamard_y32_sd15_1280x1280_16x16_full.md: 122,692,608 + 11,220,224 B
-    ("F(6,3) N8 1280->1280 16x16 G64", "hadamard_y32"): 133912832,
-    # profiles/output_transform_y32_sd15_320x320_64x64_full.md: 79,379,200 + 5,374,464 B
-    ("F(6,3) N8 320->320 64x64 G64", "output_transform"): 84753664,
-}
+NCU_TRAFFIC = {}
 
 
 def parse():

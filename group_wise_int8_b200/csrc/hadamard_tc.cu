@@ -18,16 +18,18 @@
 //   warp 0 = TMA producer;
 //   warp 1 = TMEM allocator and MMA issuer: tcgen05.mma kind::i8, M=128,
 //            N=BN, K=32 per instruction; each K-group of a tap accumulates into
-//            its own BN-column TMEM buffer (its first K-step overwrites); the
+//            its own BN-column TMEM buffer, which holds the int32 bits of
+//            1.5*2^23 before the group's first K-step (the epilogue refills it
+//            after reading it), so the result reads as that float plus acc; the
 //            buffers of one tap form a slot, a ring of at least two slots lets
 //            the MMAs run ahead of the epilogue; one wait for a free slot and
 //            one commit per tap;
 //   warps 2..9 = epilogue, 4 TMEM lane quadrants x 2 column chunks of BN/4:
 //            per tap one wait, then per group both chunks' tcgen05.ld, one
-//            wait, the slot released as soon as it is read (TMEM to register
-//            traffic is the epilogue's bottleneck, so nothing is written back),
-//            and the dequantisation in packed fp32 pairs, with (float)acc taken
-//            exactly as asfloat(acc + 0x4B400000) - 1.5*2^23.  A stage's shared
+//            wait, the buffers refilled with 1.5*2^23 (one tcgen05.st per chunk)
+//            and the slot released after its last group, and the
+//            dequantisation in packed fp32 pairs, with (float)acc taken
+//            exactly as asfloat(0x4B400000 + acc) - 1.5*2^23.  A stage's shared
 //            memory returns to the producer when every epilogue warp is done
 //            with it (which is after its MMAs completed).
 // The loops keep wrap-around ring counters (no division in the issue paths).
@@ -313,8 +315,9 @@ __global__ void __launch_bounds__(TcCfg<BN>::kThreads, 1)
                         for (int kk = 0; kk < ksteps; ++kk) {
                             const uint64_t koff = stage_off + (uint64_t)(((c * TPS + t) * a_tile + kin * 32) >> 4);
                             const uint64_t kofb = stage_off + (uint64_t)(((c * TPS + t) * b_tile + kin * 32) >> 4);
-                            // the first K-step of a group overwrites its buffer, the others accumulate
-                            mma_i8(d + (uint32_t)(g * BN), a_desc0 + koff, b_desc0 + kofb, idesc, gk != 0 ? 1u : 0u);
+                            // every K-step accumulates: the epilogue left the buffer holding the
+                            // int32 bits of 1.5*2^23, so it reads asfloat(bits + acc) = 1.5*2^23 + acc
+                            mma_i8(d + (uint32_t)(g * BN), a_desc0 + koff, b_desc0 + kofb, idesc, 1u);
                             if (++kin == ks_per_chunk) {
                                 kin = 0;
                                 ++c;
@@ -349,7 +352,14 @@ __global__ void __launch_bounds__(TcCfg<BN>::kThreads, 1)
         const uint32_t t_lane = tmem_base + ((uint32_t)(32 * quad) << 16);
         const uint64_t neg_magic2 = f2_pack(-kRoundMagic, -kRoundMagic);
 
-        // every accumulator slot starts free
+        // every accumulator buffer starts as the int32 bits of 1.5*2^23 (this warp's lanes and
+        // columns), and every slot starts free
+        for (int b = 0; b < NSLOT * GPS; ++b)
+#pragma unroll
+            for (int h = 0; h < NP; ++h) tmem_st_fill<CPT>(t_lane + (uint32_t)(b * BN + col0[h]), (uint32_t)kRoundMagicBits);
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
         if (lane == 0)
             for (int b = 0; b < NSLOT; ++b) mbar_arrive(&tail->acc_empty[b]);
 
@@ -424,7 +434,11 @@ __global__ void __launch_bounds__(TcCfg<BN>::kThreads, 1)
 #pragma unroll
                             for (int h = 0; h < NP; ++h) tmem_ld<CPT>(t_slot + (uint32_t)(j * BN + col0[h]), r[h]);
                             tmem_ld_wait();
-                            if (j + 1 == gs) {   // the slot is read: release it
+#pragma unroll
+                            for (int h = 0; h < NP; ++h)   // read: refill for the next accumulation
+                                tmem_st_fill<CPT>(t_slot + (uint32_t)(j * BN + col0[h]), (uint32_t)kRoundMagicBits);
+                            if (j + 1 == gs) {   // the slot is read and refilled: release it
+                                tmem_st_wait();
                                 tc_fence_before();
                                 __syncwarp();
                                 if (lane == 0) mbar_arrive(&tail->acc_empty[sl.idx]);
@@ -438,7 +452,9 @@ __global__ void __launch_bounds__(TcCfg<BN>::kThreads, 1)
                             if constexpr (NR != NP) {
                                 tmem_ld<CPT>(t_slot + (uint32_t)(j * BN + col0[h]), r[0]);
                                 tmem_ld_wait();
-                                if (h + 1 == NP && j + 1 == gs) {   // the slot is read: release it
+                                tmem_st_fill<CPT>(t_slot + (uint32_t)(j * BN + col0[h]), (uint32_t)kRoundMagicBits);
+                                if (h + 1 == NP && j + 1 == gs) {   // the slot is read and refilled: release it
+                                    tmem_st_wait();
                                     tc_fence_before();
                                     __syncwarp();
                                     if (lane == 0) mbar_arrive(&tail->acc_empty[sl.idx]);
@@ -448,12 +464,12 @@ __global__ void __launch_bounds__(TcCfg<BN>::kThreads, 1)
 #pragma unroll
                             for (int c4 = 0; c4 < CPT / 4; ++c4) {
                                 const float4 uu = su4[c4];
-                                // (float)acc exactly: acc + 1.5*2^23 in the integer unit, then - 1.5*2^23 (|acc| < 2^22)
-                                const uint64_t a0 = f2_add(f2_pack(__uint_as_float(r[hr][4 * c4 + 0] + kRoundMagicBits),
-                                                                   __uint_as_float(r[hr][4 * c4 + 1] + kRoundMagicBits)),
+                                // (float)acc exactly: the buffer holds the bits of 1.5*2^23 + acc (|acc| < 2^22)
+                                const uint64_t a0 = f2_add(f2_pack(__uint_as_float(r[hr][4 * c4 + 0]),
+                                                                   __uint_as_float(r[hr][4 * c4 + 1])),
                                                            neg_magic2);
-                                const uint64_t a1 = f2_add(f2_pack(__uint_as_float(r[hr][4 * c4 + 2] + kRoundMagicBits),
-                                                                   __uint_as_float(r[hr][4 * c4 + 3] + kRoundMagicBits)),
+                                const uint64_t a1 = f2_add(f2_pack(__uint_as_float(r[hr][4 * c4 + 2]),
+                                                                   __uint_as_float(r[hr][4 * c4 + 3])),
                                                            neg_magic2);
                                 y2[h][2 * c4 + 0] = f2_fma(a0, f2_mul(sv2, f2_pack(uu.x, uu.y)), y2[h][2 * c4 + 0]);
                                 y2[h][2 * c4 + 1] = f2_fma(a1, f2_mul(sv2, f2_pack(uu.z, uu.w)), y2[h][2 * c4 + 1]);
@@ -464,10 +480,10 @@ __global__ void __launch_bounds__(TcCfg<BN>::kThreads, 1)
                                 for (int c = 0; c < CPT; ++c) {
                                     if (SWAP) {   // row = output channel, column = tile
                                         const size_t di = (((size_t)tap * p.T + colg[h] + c) * p.Cout + row) * p.ng + jg;
-                                        if (colg[h] + c < p.T && in_bounds(di, p.n_acc, p.err)) p.acc[di] = (int)r[hr][c];
+                                        if (colg[h] + c < p.T && in_bounds(di, p.n_acc, p.err)) p.acc[di] = (int)(r[hr][c] - kRoundMagicBits);
                                     } else {
                                         const size_t di = (((size_t)tap * p.T + row) * p.Cout + colg[h] + c) * p.ng + jg;
-                                        if (in_bounds(di, p.n_acc, p.err)) p.acc[di] = (int)r[hr][c];
+                                        if (in_bounds(di, p.n_acc, p.err)) p.acc[di] = (int)(r[hr][c] - kRoundMagicBits);
                                     }
                                 }
                             }

@@ -210,6 +210,18 @@ __device__ __forceinline__ void tmem_ld<32>(uint32_t taddr, uint32_t (&r)[32]) {
         : "r"(taddr));
 }
 #undef WINO_R8
+// Writes v to NC consecutive 32-bit columns of this warp's 32 lanes, NC a multiple of 4, as x4
+// stores (a wider store reads a block of as many registers, all holding v).  No generic memory is
+// touched; volatile keeps the stores in order with the other tcgen05 statements.
+template <int NC>
+__device__ __forceinline__ void tmem_st_fill(uint32_t taddr, uint32_t v) {
+    static_assert(NC % 4 == 0, "x4 stores");
+#pragma unroll
+    for (int c = 0; c < NC; c += 4)
+        asm volatile("tcgen05.st.sync.aligned.32x32b.x4.b32 [%0], {%1,%1,%1,%1};" ::"r"(taddr + (uint32_t)c), "r"(v));
+}
+__device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
 // Widths between the native ones, as two loads (the second at the following columns).
 template <int NA, int NB, int NC>
 __device__ __forceinline__ void tmem_ld_pair(uint32_t taddr, uint32_t (&r)[NC]) {
