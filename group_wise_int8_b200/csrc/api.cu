@@ -776,6 +776,9 @@ int wino_resolved_variants(wino_plan_t p, int N, int H, int W, int Cin, int Cout
         return WINO_OK;
     }
     if (L.swap) f |= WINO_VARIANT_SWAPPED_GEMM;
+    if (L.gemm == WINO_GEMM_TCGEN05 &&
+        tc_a_resident((int)std::min<long>(L.T, 1 << 30), Cin, Cout, p->G, L.swap))
+        f |= WINO_VARIANT_A_RESIDENT;
     if (input_transform_split(p->mat.m, p->G, N, L.TH, L.TW, Cin, num_sms())) f |= WINO_VARIANT_SPLIT_INPUT;
     if (output_transform_split(L.T, Cout, L.y_path == WINO_YPATH_Y32, L.ytap, num_sms()))
         f |= WINO_VARIANT_SPLIT_OUTPUT;

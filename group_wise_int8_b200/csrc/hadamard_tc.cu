@@ -41,6 +41,7 @@
 // abort flag and the device error word, drains its in-flight TMA loads and
 // MMAs, frees its TMEM and returns.
 #include <algorithm>
+#include <cstring>
 
 #include "kernels.h"
 #include "sm100.cuh"
@@ -53,6 +54,7 @@ using namespace sm100;
 constexpr int kBM = 128;
 constexpr int kMaxStages = 8;
 constexpr int kMaxNacc = 8;
+constexpr int kMaxKst = 8;         // K stages of a tap kept resident (A-resident walk)
 constexpr int kSwapMaxTiles = 80;   // the swapped pass's N is 16, 32 or 80 tiles
 
 template <int BN>
@@ -69,6 +71,8 @@ struct TcCfg {
 struct SmemTail {
     uint64_t full[kMaxStages];
     uint64_t empty[kMaxStages];
+    uint64_t a_full[kMaxKst];    // A-resident walk: the tap's K stage ks of A has landed
+    uint64_t a_empty[kMaxKst];   //   ... and the MMAs of its last column block have read it
     uint64_t acc_full[kMaxNacc];
     uint64_t acc_empty[kMaxNacc];
     uint64_t done;
@@ -199,9 +203,15 @@ __global__ void __launch_bounds__(TcCfg<BN>::kThreads, 1)
     const int NSLOT = NACC / GPS;          // accumulator slots (>= 2)
     const uint32_t a_tile = kBM * BK, b_tile = BN * BK;
     const uint32_t a_bytes = a_tile * KC * TPS, b_bytes = b_tile * KC * TPS;
-    const uint32_t stage_bytes = a_bytes + b_bytes;
+    // A-resident walk: the tap's KSTAGES A stages first, then a ring of B stages; otherwise a ring
+    // of (A, B) stages
+    const bool AR = p.a_res != 0;
+    const uint32_t a_region = AR ? (uint32_t)KSTAGES * a_bytes : 0u;
+    const uint32_t stage_bytes = AR ? b_bytes : a_bytes + b_bytes;   // ring stride
+    const uint32_t b_in_stage = AR ? 0u : a_bytes;                   // B's offset within a ring stage
+    unsigned char* ring = smem + a_region;
     const int S = p.stages;
-    float* sv_ring = reinterpret_cast<float*>(smem + (size_t)S * stage_bytes);   // [S][TPS][GPS][128]
+    float* sv_ring = reinterpret_cast<float*>(ring + (size_t)S * stage_bytes);   // [S][TPS][GPS][128]
     const int su_stride = (TPS * GPS * BN + 31) / 32 * 32;                         // 128-byte stage slices
     float* su_ring = sv_ring + (size_t)S * TPS * GPS * kBM;                      // [S][su_stride]: [TPS][GPS][BN]
     SmemTail* tail = reinterpret_cast<SmemTail*>(su_ring + (size_t)S * su_stride);
@@ -220,6 +230,11 @@ __global__ void __launch_bounds__(TcCfg<BN>::kThreads, 1)
             mbar_init(&tail->acc_full[b], 1);                 // one commit per tap
             mbar_init(&tail->acc_empty[b], Cfg::kEpiWarps);
         }
+        if (AR)
+            for (int k = 0; k < KSTAGES; ++k) {
+                mbar_init(&tail->a_full[k], 1);
+                mbar_init(&tail->a_empty[k], 1);           // one commit after the last column block's MMAs
+            }
         mbar_init(&tail->done, 1);
         mbar_init(&tail->never, 1);
         tail->abort_flag = 0;
@@ -245,33 +260,50 @@ __global__ void __launch_bounds__(TcCfg<BN>::kThreads, 1)
         // ------------------------------------------------------- TMA producer
         if (lane == 0) {
             Ring st{0, 0};
-            uint32_t issued = 0;
-            bool ok = true;
+            uint32_t issued = 0, pa = 0;   // pa: phase of the resident A stages (one per tap loaded)
+            bool ok = true, a_loaded = false, first = true;
             Walk w;
             for (w.init(p); ok && w.L < w.L1;) {
                 const int nt = w.stage_taps(TPS, p.n2);
+                const bool new_a = AR && (first || w.nb == 0);   // a new (row block, tap): load its A
+                first = false;
                 for (int ks = 0; ks < KSTAGES; ++ks) {
+                    if (new_a) {
+                        if (!mbar_wait(&tail->a_empty[ks], pa ^ 1u, abort_flag, p.err)) {
+                            ok = false;
+                            break;
+                        }
+                        uint64_t* abar = &tail->a_full[ks];
+                        mbar_arrive_expect_tx(abar, a_bytes);
+                        for (int c = 0; c < KC; ++c)
+                            tma_load_3d(smem + (size_t)ks * a_bytes + (size_t)c * a_tile, &tmA, abar,
+                                        ks * p.SK + c * BK, w.mb * kBM, w.tap);
+                        a_loaded = true;
+                    }
                     if (!mbar_wait(&tail->empty[st.idx], st.phase ^ 1u, abort_flag, p.err)) {
                         ok = false;
                         break;
                     }
                     // whole boxes of TPS taps; taps past n2 read zeros and taps past the range go unused
                     uint64_t* bar = &tail->full[st.idx];
-                    unsigned char* sa = smem + (size_t)st.idx * stage_bytes;
+                    unsigned char* sa = ring + (size_t)st.idx * stage_bytes;
                     mbar_arrive_expect_tx(bar, stage_bytes + scale_bytes);
                     for (int c = 0; c < KC; ++c) {
                         const int k0 = ks * p.SK + c * BK;
-                        tma_load_3d(sa + (size_t)c * TPS * a_tile, &tmA, bar, k0, w.mb * kBM, w.tap);
-                        tma_load_3d(sa + a_bytes + (size_t)c * TPS * b_tile, &tmB, bar, k0, w.nb * BN, w.tap);
+                        if (!AR) tma_load_3d(sa + (size_t)c * TPS * a_tile, &tmA, bar, k0, w.mb * kBM, w.tap);
+                        tma_load_3d(sa + b_in_stage + (size_t)c * TPS * b_tile, &tmB, bar, k0, w.nb * BN, w.tap);
                     }
                     tma_load_3d(sv_ring + (size_t)st.idx * TPS * GPS * kBM, &tmSV, bar, w.mb * kBM, ks * GPS, w.tap);
                     tma_load_3d(su_ring + (size_t)st.idx * su_stride, &tmSU, bar, w.nb * BN, ks * GPS, w.tap);
                     ++issued;
                     st.next(S);
                 }
+                if (new_a) pa ^= 1u;
                 w.advance(nt, p);
             }
-            // drain: every issued load must land before the CTA can exit
+            // drain: every issued load must land before the CTA can exit (the last A stages too)
+            if (a_loaded)
+                for (int ks = 0; ks < KSTAGES; ++ks) mbar_wait_teardown(&tail->a_full[ks], pa ^ 1u);
             Ring dr{st.idx, st.phase};
             for (uint32_t i = 0; i < issued && i < (uint32_t)S; ++i) {
                 if (dr.idx == 0) {
@@ -287,22 +319,42 @@ __global__ void __launch_bounds__(TcCfg<BN>::kThreads, 1)
         // --------------------------------------------------------- MMA issuer
         if (lane == 0) {
             const uint32_t idesc = idesc_i8(kBM, BN);
-            const uint64_t a_desc0 = smem_desc_kmajor(smem_u32(smem), BK);
-            const uint64_t b_desc0 = smem_desc_kmajor(smem_u32(smem) + a_bytes, BK);
+            const uint64_t a_desc0 = smem_desc_kmajor(smem_u32(AR ? smem : ring), BK);
+            const uint64_t b_desc0 = smem_desc_kmajor(smem_u32(ring) + b_in_stage, BK);
             const int ks_per_group = p.G / 32;
             const int ks_per_chunk = BK / 32;
+            // per K-step of a stage (at most 8: SK <= 256 bytes for G <= 256): the descriptor offsets
+            // (16-byte units) of A and B for the stage's first tap and the TMEM column of its K-group,
+            // so that a stage's MMAs issue as straight-line code
+            uint32_t offa[8], offb[8], dcol[8];
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk) {
+                const int c = kk / ks_per_chunk, kin = kk - c * ks_per_chunk;
+                offa[kk] = (uint32_t)(c * TPS * a_tile + kin * 32) >> 4;
+                offb[kk] = (uint32_t)(c * TPS * b_tile + kin * 32) >> 4;
+                dcol[kk] = (uint32_t)((kk / ks_per_group) * BN);
+            }
             Ring st{0, 0}, sl{0, 0};
-            bool ok = true;
+            uint32_t pa = 0;
+            bool ok = true, first = true;
             if (p.force_timeout) ok = mbar_wait(&tail->never, 0, abort_flag, p.err, 1000000ull);
             Walk w;
             for (w.init(p); ok && w.L < w.L1;) {
                 const int nt = w.stage_taps(TPS, p.n2);
+                const bool new_a = AR && (first || w.nb == 0);
+                const bool last_a = AR && (w.L + 1 == w.L1 || w.nb + 1 == p.num_nb);   // A read for the last time
+                first = false;
                 for (int ks = 0; ok && ks < KSTAGES; ++ks) {
+                    if (new_a && !mbar_wait(&tail->a_full[ks], pa, abort_flag, p.err)) {
+                        ok = false;
+                        break;
+                    }
                     if (!mbar_wait(&tail->full[st.idx], st.phase, abort_flag, p.err)) {
                         ok = false;
                         break;
                     }
                     const uint64_t stage_off = (uint64_t)((st.idx * stage_bytes) >> 4);
+                    const uint64_t a_off = AR ? (uint64_t)((ks * a_bytes) >> 4) : stage_off;
                     const int ksteps = (ks + 1 == KSTAGES ? GLAST : GPS) * ks_per_group;   // K-steps of this stage
                     for (int t = 0; t < nt; ++t) {
                         if (!mbar_wait(&tail->acc_empty[sl.idx], sl.phase, abort_flag, p.err)) {
@@ -311,27 +363,20 @@ __global__ void __launch_bounds__(TcCfg<BN>::kThreads, 1)
                         }
                         tc_fence_after();
                         const uint32_t d = tmem_base + (uint32_t)(sl.idx * GPS * BN);
-                        int c = 0, kin = 0, g = 0, gk = 0;
-                        for (int kk = 0; kk < ksteps; ++kk) {
-                            const uint64_t koff = stage_off + (uint64_t)(((c * TPS + t) * a_tile + kin * 32) >> 4);
-                            const uint64_t kofb = stage_off + (uint64_t)(((c * TPS + t) * b_tile + kin * 32) >> 4);
-                            // every K-step accumulates: the epilogue left the buffer holding the
-                            // int32 bits of 1.5*2^23, so it reads asfloat(bits + acc) = 1.5*2^23 + acc
-                            mma_i8(d + (uint32_t)(g * BN), a_desc0 + koff, b_desc0 + kofb, idesc, 1u);
-                            if (++kin == ks_per_chunk) {
-                                kin = 0;
-                                ++c;
-                            }
-                            if (++gk == ks_per_group) {
-                                gk = 0;
-                                ++g;
-                            }
-                        }
+                        const uint64_t abase = a_desc0 + a_off + (uint64_t)((t * a_tile) >> 4);
+                        const uint64_t bbase = b_desc0 + stage_off + (uint64_t)((t * b_tile) >> 4);
+                        // every K-step accumulates: the epilogue left the buffer holding the
+                        // int32 bits of 1.5*2^23, so it reads asfloat(bits + acc) = 1.5*2^23 + acc
+#pragma unroll
+                        for (int kk = 0; kk < 8; ++kk)
+                            if (kk < ksteps) mma_i8(d + dcol[kk], abase + offa[kk], bbase + offb[kk], idesc, 1u);
                         mma_commit(&tail->acc_full[sl.idx]);
                         sl.next(NSLOT);
                     }
+                    if (ok && last_a) mma_commit(&tail->a_empty[ks]);   // the A stage is free once these MMAs complete
                     st.next(S);
                 }
+                if (new_a) pa ^= 1u;
                 w.advance(nt, p);
             }
             // all issued MMAs complete before TMEM is released
@@ -350,6 +395,10 @@ __global__ void __launch_bounds__(TcCfg<BN>::kThreads, 1)
 #pragma unroll
         for (int h = 0; h < NP; ++h) col0[h] = ((ew >> 2) + (4 / NP) * h) * CPT;
         const uint32_t t_lane = tmem_base + ((uint32_t)(32 * quad) << 16);
+        // a chunk's fp32 Y row segment starts at a multiple of CPT (8 or 16) floats of a row of Cout (a
+        // multiple of 32) floats, so it is 32-byte aligned whenever the Y base is (the workspace
+        // itself is only promised 16-byte alignment)
+        const bool y32_v8 = CPT % 8 == 0 && (reinterpret_cast<uintptr_t>(p.Y32) & 31u) == 0;
         const uint64_t neg_magic2 = f2_pack(-kRoundMagic, -kRoundMagic);
 
         // every accumulator buffer starts as the int32 bits of 1.5*2^23 (this warp's lanes and
@@ -528,9 +577,14 @@ __global__ void __launch_bounds__(TcCfg<BN>::kThreads, 1)
                             const size_t yi = ((size_t)tap * p.T + row) * p.Cout + colg[h];
                             if (MODE == kModeY32 && valid && in_bounds(yi + CPT - 1, p.n_y, p.err)) {
                                 float* dst = p.Y32 + yi;
+                                if (y32_v8) {   // whole 32-byte sectors per store
 #pragma unroll
-                                for (int c = 0; c < CPT; c += 4)
-                                    *reinterpret_cast<float4*>(dst + c) = make_float4(y[c], y[c + 1], y[c + 2], y[c + 3]);
+                                    for (int c = 0; c < CPT; c += 8) st_global_v8(dst + c, y + c);
+                                } else {
+#pragma unroll
+                                    for (int c = 0; c < CPT; c += 4)
+                                        *reinterpret_cast<float4*>(dst + c) = make_float4(y[c], y[c + 1], y[c + 2], y[c + 3]);
+                                }
                             }
                         }
                     }
@@ -581,9 +635,11 @@ struct Maps {
 
 size_t smem_bytes(const GemmArgs& a, int BN) {
     const size_t gps = (size_t)(a.SK / a.G);
-    const size_t per_stage = (size_t)a.tps * a.SK * (kBM + BN) + (size_t)a.tps * gps * kBM * 4 +
+    const size_t kstages = (size_t)((a.ng + (int)gps - 1) / (int)gps);
+    const size_t a_region = a.a_res ? kstages * a.SK * kBM : 0;   // the tap's resident A stages
+    const size_t per_stage = (size_t)a.tps * a.SK * ((a.a_res ? 0 : kBM) + BN) + (size_t)a.tps * gps * kBM * 4 +
                              ((size_t)a.tps * gps * BN + 31) / 32 * 32 * 4;
-    return 1024 + (size_t)a.stages * per_stage + sizeof(SmemTail);
+    return 1024 + a_region + (size_t)a.stages * per_stage + sizeof(SmemTail);
 }
 
 template <int BN, int MODE, bool DUMP, bool SWAP = false>
@@ -645,7 +701,10 @@ int tc_block_n(int Cout, int G) {
 // exist, and at most 256 bytes unless one group is larger); the last stage of a tap holds the
 // remaining groups (its boxes past Cin read zeros and its MMAs and epilogue skip them).  Swizzle
 // width BK divides SK and G.  TPS taps share a stage when one stage holds a tap's whole K and there
-// is one column block (as many as keep three stages in the shared-memory budget).
+// is one column block (as many as keep three stages in the shared-memory budget).  With several
+// column blocks (one tap per stage) a tap's whole A tile stays resident while the CTA walks that
+// tap's column blocks, when it fits beside at least three B stages: the A operand then crosses from
+// L2 once per (row block, tap) instead of once per column block.
 static void choose_stage(GemmArgs& a, int BN) {
     const int nacc = std::min(512 / BN, kMaxNacc);
     const int max_groups = std::max(1, std::min(nacc / 2, std::max(a.G, 256) / a.G));
@@ -662,11 +721,39 @@ static void choose_stage(GemmArgs& a, int BN) {
                 a.tps = t;
                 break;
             }
+    const int kstages = (a.ng + gps - 1) / gps;
+    const size_t a_region = (size_t)kstages * sk * kBM;
+    const size_t per_b = (size_t)sk * BN + (size_t)gps * (kBM + BN) * 4;
+    const size_t ar_budget = 212 * 1024;
+    a.a_res = !a.swap_ab && a.num_nb > 1 && a.tps == 1 && kstages <= kMaxKst && a_region < ar_budget &&
+              (ar_budget - a_region) / per_b >= 3;
+    if (a.a_res) {
+        const int stages = (int)((ar_budget - a_region) / per_b);
+        a.stages = stages > kMaxStages ? kMaxStages : stages;
+        return;
+    }
     const int stages = (int)(budget / (per_tap * a.tps));
     a.stages = stages > kMaxStages ? kMaxStages : (stages < 2 ? 2 : stages);
 }
 
 bool tc_swap_ok(int T, int Cout) { return T <= kSwapMaxTiles && Cout % kBM == 0; }
+
+bool tc_a_resident(int T, int Cin, int Cout, int G, bool swap) {
+    const int BN = swap ? (T <= 16 ? 16 : (T <= 32 ? 32 : 80)) : tc_block_n(Cout, G);
+    if (BN == 0 || G <= 0 || Cin % G != 0) return false;
+    GemmArgs a;
+    std::memset(&a, 0, sizeof(a));
+    a.T = T;
+    a.Cin = Cin;
+    a.Cout = Cout;
+    a.G = G;
+    a.ng = Cin / G;
+    a.n2 = 64;   // the walk's shape does not depend on the tap count beyond TPS, which is 1 here
+    a.swap_ab = swap ? 1 : 0;
+    a.num_nb = swap ? (T + BN - 1) / BN : Cout / BN;
+    choose_stage(a, BN);
+    return a.a_res != 0;
+}
 
 cudaError_t launch_hadamard_tc(GemmArgs a, const int8_t* Vq, const int8_t* Uq, int mode, int num_sms,
                                cudaStream_t st, int* launches) {

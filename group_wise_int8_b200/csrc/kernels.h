@@ -87,6 +87,8 @@ struct GemmArgs {
     int force_timeout; // test hook: the MMA thread first waits 1 ms on a barrier nothing completes
     int swap_ab;       // fp32-Y mode, T <= 80, Cout % 128 == 0: the MMA rows are 128 output channels
                        // (A = Uq) and its columns the tiles (B = Vq), so no TMEM lane is padding
+    int a_res;         // set by the launcher: a tap's whole A tile stays in shared memory while the
+                       // CTA walks that tap's column blocks (several column blocks, one tap per stage)
     size_t n_v, n_u, n_amax, n_y, n_acc;   // element counts of Vq (and sV), Uq (and sU), amax, Yq/Y32 and acc
                                            // (index checks of the debug build)
 };
@@ -96,6 +98,7 @@ cudaError_t launch_hadamard_tc(GemmArgs a, const int8_t* Vq, const int8_t* Uq, i
                                cudaStream_t st, int* launches);
 int tc_block_n(int Cout, int G);  // 0 if unsupported
 bool tc_swap_ok(int T, int Cout);  // the swapped-operand fp32-Y pass applies (T <= 80, Cout % 128 == 0)
+bool tc_a_resident(int T, int Cin, int Cout, int G, bool swap);   // the GEMM keeps a tap's A tile resident
 
 cudaError_t launch_hadamard_simt(const GemmArgs& a, const int8_t* Vq, const int8_t* Uq, int mode, cudaStream_t st);
 

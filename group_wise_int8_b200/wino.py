@@ -37,7 +37,7 @@ YPATH_AUTO, YPATH_RECOMPUTE, YPATH_Y32 = 0, 1, 2
 GEMM_AUTO, GEMM_TCGEN05, GEMM_SIMT = 0, 1, 2
 DEBUG_YQ, DEBUG_ACC32, DEBUG_FORCE_TIMEOUT, DEBUG_GUARDS, DEBUG_SHRINK_BOUNDS = 1, 2, 4, 8, 16
 YGROUPS_TILE, YGROUPS_TAP = 0, 1
-VARIANT_SWAPPED_GEMM, VARIANT_SPLIT_INPUT, VARIANT_SPLIT_OUTPUT, VARIANT_FUSED = 1, 2, 4, 8
+VARIANT_SWAPPED_GEMM, VARIANT_SPLIT_INPUT, VARIANT_SPLIT_OUTPUT, VARIANT_FUSED, VARIANT_A_RESIDENT = 1, 2, 4, 8, 16
 FUSED_AUTO, FUSED_OFF, FUSED_ON = 0, 1, 2
 DUMP_VQ, DUMP_SV, DUMP_YQ, DUMP_SY, DUMP_Y32, DUMP_ACC32 = range(6)
 NOALLOC_SCRATCH_BYTES = 64 << 20   # WINO_NOALLOC_SCRATCH_BYTES

@@ -309,13 +309,16 @@ int wino_debug_dump(wino_plan_t plan, const void* ws_dev, int N, int H, int W, i
 int wino_resolved_config(wino_plan_t plan, int N, int H, int W, int Cin, int Cout, int* y_path, int* gemm);
 
 /* Kernel variants a call of this shape runs (all give the same bytes), as a
- * bit set of WINO_VARIANT_*: the swapped-operand GEMM pass, and the split input
+ * bit set of WINO_VARIANT_*: the swapped-operand GEMM pass, the split input
  * and output transforms (more threads per tile; sized by the device's SM count,
- * 148 assumed when no device is visible).  Errors: INVALID_ARG. */
+ * 148 assumed when no device is visible), the fused small-channel kernel, and
+ * the GEMM walk that keeps a tap's A tile resident in shared memory across its
+ * column blocks.  Errors: INVALID_ARG. */
 #define WINO_VARIANT_SWAPPED_GEMM 1
 #define WINO_VARIANT_SPLIT_INPUT 2
 #define WINO_VARIANT_SPLIT_OUTPUT 4
 #define WINO_VARIANT_FUSED 8
+#define WINO_VARIANT_A_RESIDENT 16
 int wino_resolved_variants(wino_plan_t plan, int N, int H, int W, int Cin, int Cout, int* flags);
 
 /* Number of kernels one wino_conv2d_int8 call of this shape launches. */

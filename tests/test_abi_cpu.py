@@ -185,14 +185,16 @@ def test_resolved_config_cost_model(lib):
 
 def test_parity_cases_cover_every_kernel_variant(lib):
     """The GPU parity cases (stagewise, both Y paths) run each shape-chosen variant -- swapped GEMM,
-    split input and split output transforms -- and also each kernel it replaces, so bit-exactness
-    is checked on both sides of every choice (SM count 148, as on the B200)."""
+    split input and split output transforms, the A-resident GEMM walk -- and also each kernel it
+    replaces, so bit-exactness is checked on both sides of every choice (SM count 148, as on the
+    B200)."""
     from tests.test_gpu_parity import CASES
     seen = {}
     for name, (m, pts, N, H, W, Cin, Cout, G, *_rest) in CASES.items():
         for y_path in (wino.YPATH_RECOMPUTE, wino.YPATH_Y32):
             flags = wino.Plan(m, pts, None, None, G, y_path=y_path).resolved_variants(N, H, W, Cin, Cout)
-            for bit in (wino.VARIANT_SWAPPED_GEMM, wino.VARIANT_SPLIT_INPUT, wino.VARIANT_SPLIT_OUTPUT):
+            for bit in (wino.VARIANT_SWAPPED_GEMM, wino.VARIANT_SPLIT_INPUT, wino.VARIANT_SPLIT_OUTPUT,
+                        wino.VARIANT_A_RESIDENT):
                 seen.setdefault(bit, set()).add(bool(flags & bit))
     assert all(v == {False, True} for v in seen.values()), seen
 
@@ -204,3 +206,8 @@ def test_variants_follow_the_shape(lib):
                                                         wino.VARIANT_SPLIT_OUTPUT)
     q = wino.Plan(6, synth.POINTS_F6, None, None, 32)
     assert q.resolved_variants(32, 56, 56, 64, 64) == 0          # the default layer: none
+    # SD-shaped 64x64 and 32x32 layers: several column blocks, A resident up to Cin 960 (four K stages
+    # beside three B stages); Cin 1920 does not fit
+    for plan, shape, ar in ((p, (8, 64, 64, 320, 320), True), (p, (8, 64, 64, 960, 320), True),
+                            (p, (8, 32, 32, 640, 640), True), (p, (8, 32, 32, 1920, 640), False)):
+        assert bool(plan.resolved_variants(*shape) & wino.VARIANT_A_RESIDENT) == ar, shape

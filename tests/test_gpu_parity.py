@@ -57,6 +57,10 @@ CASES = {
     "f6_swap_n80_ragged": (6, P6, 2, 34, 35, 320, 256, 64, "bf16", "student_t_outliers", "loguniform"),
     "f4_swap_n80_full": (4, P4, 5, 16, 16, 128, 128, 64, "bf16", "relu_normal", "loguniform"),
     "f6_81_tiles": (6, P6, 1, 54, 54, 128, 128, 64, "bf16", "relu_normal", "loguniform"),
+    # the A-resident GEMM walk: a tap's A tile kept across three column blocks, over two K stages (the
+    # second ragged: 5 groups as 4 + 1), and over four K stages across two column blocks
+    "f6_a_resident_ragged_k": (6, P6, 2, 40, 40, 320, 192, 64, "bf16", "student_t_outliers", "loguniform"),
+    "f6_a_resident_cin960": (6, P6, 1, 60, 60, 960, 128, 64, "bf16", "relu_normal", "loguniform"),
 }
 
 
