@@ -61,7 +61,14 @@ UNIT = "TFLOP/s"
 # (dram__bytes_read.sum + dram__bytes_write.sum), keyed by (layer shape, kernel);
 # the summary with its command line is the named file under profiles/.  An
 # entry is removed whenever its kernel changes.
-NCU_TRAFFIC = {}
+NCU_TRAFFIC = {
+    # profiles/hadamard_y32_swapped_sd15_1280x1280_8x8_full.md: 114,457,344 + 4,860,160 B
+    ("F(6,3) N8 1280->1280 8x8 G64", "hadamard_y32"): 119317504,
+    # profiles/hadamard_y32_a_resident_sd15_320x320_64x64_full.md: 32,512,256 + 29,470,208 B
+    ("F(6,3) N8 320->320 64x64 G64", "hadamard_y32"): 61982464,
+    # profiles/output_transform_y32_sd15_320x320_64x64_full.md: 79,386,880 + 4,299,008 B
+    ("F(6,3) N8 320->320 64x64 G64", "output_transform"): 83685888,
+}
 
 
 def parse():
@@ -260,7 +267,7 @@ def plan_key(layer: synth.Layer):
     return (layer.m, layer.points, layer.group, layer.workload if layer.scales != "identity" else "identity")
 
 
-def make_plan(layer: synth.Layer, args, fused=None):
+def make_plan(layer: synth.Layer, args, fused=None, y_path=None):
     from group_wise_int8_b200 import wino
     sb, sg = synth.make_scales(layer)
     y_groups = wino.YGROUPS_TAP if getattr(args, "y_groups", "tile") == "tap" else wino.YGROUPS_TILE
@@ -268,7 +275,7 @@ def make_plan(layer: synth.Layer, args, fused=None):
         fused = wino.FUSED_ON if getattr(args, "fused", False) else wino.FUSED_AUTO
     return wino.Plan(layer.m, layer.points, sb, sg, layer.group, y_groups=y_groups,
                      x_int8=getattr(args, "x_int8", False), int8_transforms=getattr(args, "int8_transforms", False),
-                     fused=fused)
+                     fused=fused, y_path=wino.YPATH_AUTO if y_path is None else y_path)
 
 
 def prepare(layers, args, dev, keep_bf16_weights=False):
@@ -556,6 +563,9 @@ def run_ours(args, label, layers, rank, world):
         res["cudnn_bf16"] = time_cudnn(dls, flush, stream, args.steps)
     del dls, ws
     torch.cuda.empty_cache()
+    if extras and len(layers) > 1:
+        res["y_path_check"] = y_path_check(layers, args, dev, flush, stream, args.layer_steps)
+    torch.cuda.empty_cache()
     if extras:
         res["beside"] = layer_line("resnet18", synth.workload("resnet18")[0], args, dev, flush, stream, peaks, i8)
         res["layers"] = [layer_line(w, l, args, dev, flush, stream, peaks, i8)
@@ -580,8 +590,10 @@ def layer_line(wname, layer, args, dev, flush, stream, peaks, i8):
            "kernels": kernel_table(dls, prof, i8["int8_tops"], peaks)[0]["kernels"],
            "roofline": roofline_of(dls, prof, peaks, i8["int8_tops"]),
            "cudnn_bf16_tflops": round(cd["value"], 1), "cudnn_bf16_us": round(cd["ms_per_step"] * 1e3, 1)}
-    # the one-kernel path where it applies, timed the same way on the same inputs (opt-in: slower here)
     from group_wise_int8_b200 import wino
+    # the Y path that AUTO did not choose, timed the same way on the same inputs
+    out["other_y_path"] = other_y_path_time(d, layer, args, dev, flush, stream, steps)
+    # the one-kernel path where it applies, timed the same way on the same inputs (opt-in: slower here)
     fp = make_plan(layer, args, fused=wino.FUSED_ON)
     if fp.resolved_variants(*d.shape) & wino.VARIANT_FUSED:
         d.plan = fp
@@ -595,6 +607,52 @@ def layer_line(wname, layer, args, dev, flush, stream, peaks, i8):
     del dls, ws
     torch.cuda.empty_cache()
     return out
+
+
+def other_y_path_time(d, layer, args, dev, flush, stream, steps):
+    """Time of one call on the Y path that AUTO did not choose (the swapped GEMM
+    only exists on the fp32-Y path, so recompute there runs unswapped)."""
+    import torch
+    from group_wise_int8_b200 import wino
+    names = {wino.YPATH_RECOMPUTE: "recompute", wino.YPATH_Y32: "y32"}
+    other = wino.YPATH_Y32 if d.y_path == wino.YPATH_RECOMPUTE else wino.YPATH_RECOMPUTE
+    try:
+        op = make_plan(layer, args, y_path=other)
+    except wino.WinoError:   # e.g. per-tap Y groups exist only on the fp32-Y path
+        return None
+    if op.resolved_config(*d.shape)[0] != other:
+        return None
+    saved = d.plan
+    d.plan = op   # same points, scales and G: the transformed weights are the same bytes
+    ows = torch.empty(op.workspace_bytes(*d.shape), dtype=torch.uint8, device=dev)
+    oms = time_steps([d], ows, flush, stream, steps, 3)
+    d.plan = saved
+    del ows
+    return {"y_path": names[other], "us": round(sum(oms) / len(oms) * 1e3, 1)}
+
+
+def y_path_check(layers, args, dev, flush, stream, steps):
+    """Per distinct shape of the workload: one call on the chosen Y path and one on the other, each
+    with the L2 flushed before it, so the AUTO choice can be checked against measurement."""
+    import torch
+    rows, seen = [], set()
+    for layer in layers:
+        key = shape_key(layer)
+        if key in seen:
+            continue
+        seen.add(key)
+        d = prepare([layer], args, dev)[0]
+        ws = torch.empty(d.plan.workspace_bytes(*d.shape), dtype=torch.uint8, device=dev)
+        ms = time_steps([d], ws, flush, stream, steps, 3)
+        chosen = {1: "recompute", 2: "y32"}.get(d.y_path)
+        row = {"layer": key, "chosen": chosen, "chosen_us": round(sum(ms) / len(ms) * 1e3, 1),
+               "other": other_y_path_time(d, layer, args, dev, flush, stream, steps)}
+        if row["other"] is not None:
+            row["chosen_is_faster"] = row["chosen_us"] <= row["other"]["us"]
+        rows.append(row)
+        del d, ws
+        torch.cuda.empty_cache()
+    return rows
 
 
 # ------------------------------------------------------------- CPU oracle timing
@@ -761,7 +819,7 @@ def main():
     line.update(value=r["value"], ms_per_step=r["ms_per_step"], e2e=r["e2e"], roofline=r["roofline"],
                 cpu_baseline=cpu, clocks=r["clocks"], gpu_launches=r["gpu_launches"], impl="ours",
                 kernels=r["kernels"], int8_peak=r["int8_peak"])
-    for k in ("cudnn_bf16", "beside", "layers"):
+    for k in ("cudnn_bf16", "y_path_check", "beside", "layers"):
         if k in r:
             line[k] = r[k]
     print(json.dumps(line))

@@ -79,6 +79,9 @@ __device__ __forceinline__ void quant_batch(const float* vw, int lane, int warp,
                                             int tx0, int row_id, int g, const InputArgs& p, float (&red)[MAXW][TB]) {
     constexpr int P = kVPitch, C1 = kVChunk1;
     constexpr int CPW = G <= 64 ? 1 : G / 64;    // warps per group (G > 64)
+    // a chunk's 32 codes start at a multiple of 32 bytes of a row of Cin (a multiple of 32) bytes, so
+    // they fill one sector whenever the Vq base is 32-byte aligned (the workspace is promised 16)
+    const bool vq_v8 = (reinterpret_cast<uintptr_t>(p.Vq) & 31u) == 0;
 #pragma unroll
     for (int r0 = 0; r0 < 2 * TB; r0 += 32) {
         const int k = r0 + lane;
@@ -133,9 +136,13 @@ __device__ __forceinline__ void quant_batch(const float* vw, int lane, int warp,
         }
         const size_t vi = ((size_t)tap * p.T_pad + t) * p.Cin + g * G + ch;
         if (!in_bounds(vi + 31, p.n_vq, p.err)) continue;
-        uint4* dst = reinterpret_cast<uint4*>(p.Vq + vi);
-        dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
-        dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
+        if (vq_v8) {   // the chunk's 32 codes as one whole 32-byte sector
+            sm100::st_global_v8(reinterpret_cast<uint32_t*>(p.Vq + vi), w);
+        } else {
+            uint4* dst = reinterpret_cast<uint4*>(p.Vq + vi);
+            dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
+            dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
+        }
     }
 }
 

@@ -64,7 +64,7 @@ extern "C" {
 
 /* ----------------------------------------------------------------- options */
 /* How Y travels from the Hadamard GEMM to the output transform. */
-#define WINO_YPATH_AUTO 0      /* per layer, by a byte/ALU cost model */
+#define WINO_YPATH_AUTO 0      /* the fp32-Y path (measured faster on every configured layer) */
 #define WINO_YPATH_RECOMPUTE 1 /* GEMM pass 1: absmax only; pass 2: recompute, quantise, write int8 Yq */
 #define WINO_YPATH_Y32 2       /* one GEMM pass writes fp32 Y; the output transform requantises it */
 

@@ -171,12 +171,17 @@ def test_workspace_and_weight_sizes(lib):
     assert p.weight_bytes(C, 40) == 0
 
 
-def test_resolved_config_cost_model(lib):
+def test_resolved_config_auto_is_fp32_y(lib):
+    """AUTO resolves to the single-pass fp32-Y path on every shape (measured faster than the
+    two-pass recompute path on each configured layer); recompute runs on request."""
     p = wino.Plan(6, synth.POINTS_F6, None, None, 64)
-    # many tiles, few channels: recompute the GEMM rather than round-trip fp32 Y
-    assert p.resolved_config(32, 56, 56, 64, 64)[0] in (wino.YPATH_RECOMPUTE, wino.YPATH_Y32)
-    # few tiles, many channels: re-reading the transformed weights dominates -> fp32 Y
-    assert p.resolved_config(2, 8, 8, 1280, 1280)[0] == wino.YPATH_Y32
+    for shape in ((32, 56, 56, 64, 64), (64, 28, 28, 128, 128), (2, 64, 64, 320, 320), (8, 32, 32, 1920, 640),
+                  (2, 8, 8, 1280, 1280)):
+        assert p.resolved_config(*shape)[0] == wino.YPATH_Y32, shape
+        assert p.launches_per_call(*shape) == 3
+    rec = wino.Plan(6, synth.POINTS_F6, None, None, 64, y_path=wino.YPATH_RECOMPUTE)
+    assert rec.resolved_config(32, 56, 56, 64, 64)[0] == wino.YPATH_RECOMPUTE
+    assert rec.launches_per_call(32, 56, 56, 64, 64) == 4
     assert p.resolved_config(2, 8, 8, 1280, 1280)[1] == wino.GEMM_TCGEN05
     forced = wino.Plan(6, synth.POINTS_F6, None, None, 64, y_path=wino.YPATH_RECOMPUTE, gemm=wino.GEMM_SIMT)
     assert forced.resolved_config(2, 8, 8, 1280, 1280) == (wino.YPATH_RECOMPUTE, wino.GEMM_SIMT)

@@ -215,17 +215,17 @@ def test_host_entry_point_chunks_match_device_call(cuda_dev, N, x_int8):
     assert torch.equal(y_host, y_dev.cpu())
 
 
-def test_host_entry_point_last_chunk_on_another_y_path(cuda_dev):
+def test_host_entry_point_last_chunk_on_another_kernel(cuda_dev):
     """N = 8 in chunks of 3, 3 and 2 images: on this SD-shaped layer (320 -> 640, 32x32, G = 64)
-    the 3-image chunks take the recompute path and the 2-image chunk the fp32-Y path, whose
-    workspace is twice as large; the chunk workspaces are sized for both."""
+    the 3-image chunks (108 tiles) run the GEMM with tiles on the MMA rows and the 2-image chunk
+    (72 tiles) the swapped GEMM; the chunk workspaces are carved for every chunk size."""
     N, H, W, Cin, Cout = 8, 32, 32, 320, 640
     layer = synth.random_layer(11, 6, N, H, W, Cin, Cout, 64, dtype="bf16", act="student_t_outliers",
                                w_var_num=1.0, workload="host_chunk_paths")
     sb, sg = synth.make_scales(layer)
     plan = wino.Plan(6, P6, sb, sg, 64)
-    assert plan.resolved_config(3, H, W, Cin, Cout)[0] == wino.YPATH_RECOMPUTE
-    assert plan.resolved_config(2, H, W, Cin, Cout)[0] == wino.YPATH_Y32
+    assert not plan.resolved_variants(3, H, W, Cin, Cout) & wino.VARIANT_SWAPPED_GEMM
+    assert plan.resolved_variants(2, H, W, Cin, Cout) & wino.VARIANT_SWAPPED_GEMM
     wt = plan.transform_weights(torch.from_numpy(synth.make_weights(layer)).cuda())
     _, bits = synth.make_input(layer)
     x_host = torch.from_numpy(bits.view(np.int16).copy()).view(torch.bfloat16).pin_memory()
