@@ -182,29 +182,38 @@ int cuda_status(wino_plan_s* p, cudaError_t e) {
 
 constexpr int kMaxHostChunks = 3;
 
-// The last call on each workspace, when it was a pipelined host call: its plan and its chunk
-// layout (workspace, chunks, images per chunk, bytes per image in and out).  A host call whose
-// workspace was last used by the same plan with the same layout orders each chunk's input copy
-// only after that call's compute of the chunk, so it overlaps that call's tail.  Any other call on
-// the workspace (another plan, another layout, the device-buffer entry point, whose workspace may
-// reach into the staging area) ends the chain, and so does destroying the plan.
+// The last host call on each workspace: its plan, the bytes its convolution used from the
+// workspace's start (need) and its staging range [lo, hi), and an event recorded on its stream
+// when it began (so it fires once every call before it is complete).  The next host call on the
+// workspace puts its staging where it touches neither of those ranges, when that fits, and then
+// orders its input copies only after that event: they overlap the previous call's convolution
+// and output copies.  Any other use of the workspace (the device-buffer entry point) ends the
+// chain, and so does destroying the plan.
 struct HostChain {
     const wino_plan_s* plan;
-    size_t sig[5];
+    size_t need, lo, hi;
+    cudaEvent_t start;
 };
 std::mutex g_chain_mutex;
 std::unordered_map<const void*, HostChain> g_chain;
 
+void chain_erase(std::unordered_map<const void*, HostChain>::iterator it) {
+    if (it->second.start) cudaEventDestroy(it->second.start);
+    g_chain.erase(it);
+}
+
 void chain_forget_workspace(const void* ws) {
     std::lock_guard<std::mutex> lock(g_chain_mutex);
-    g_chain.erase(ws);
+    auto it = g_chain.find(ws);
+    if (it != g_chain.end()) chain_erase(it);
 }
 
 void chain_forget_plan(const wino_plan_s* p) {
     std::lock_guard<std::mutex> lock(g_chain_mutex);
     for (auto it = g_chain.begin(); it != g_chain.end();) {
-        if (it->second.plan == p) it = g_chain.erase(it);
-        else ++it;
+        auto next = std::next(it);
+        if (it->second.plan == p) chain_erase(it);
+        it = next;
     }
 }
 
@@ -557,10 +566,15 @@ int wino_conv2d_int8(wino_plan_t p, const void* x, int x_dtype, int N, int H, in
                     static_cast<cudaStream_t>(stream));
 }
 
-size_t wino_host_staging_bytes(wino_plan_t p, int N, int H, int W, int Cin, int Cout, int x_dtype, int y_dtype) {
-    if (check_shape(p, N, H, W, Cin, Cout)) return 0;
+// One call's device staging for x and y.
+size_t staging_one(int N, int H, int W, int Cin, int Cout, int x_dtype, int y_dtype) {
     const size_t xs = x_dtype == WINO_BF16 ? 2 : 4, ys = y_dtype == WINO_BF16 ? 2 : 4;
     return up(xs * N * H * W * Cin, kAlign) + up(ys * N * H * W * Cout, kAlign);
+}
+
+size_t wino_host_staging_bytes(wino_plan_t p, int N, int H, int W, int Cin, int Cout, int x_dtype, int y_dtype) {
+    if (check_shape(p, N, H, W, Cin, Cout)) return 0;
+    return 2 * staging_one(N, H, W, Cin, Cout, x_dtype, y_dtype);   // two calls' staging: consecutive calls overlap
 }
 
 int wino_conv2d_int8_host(wino_plan_t p, const void* x_host, int x_dtype, int N, int H, int W, int Cin,
@@ -571,29 +585,61 @@ int wino_conv2d_int8_host(wino_plan_t p, const void* x_host, int x_dtype, int N,
     if (rc) return rc;
     const Layout L = make_layout(p, N, H, W, Cin, Cout);
     const size_t need = L.total;
-    const size_t stage = wino_host_staging_bytes(p, N, H, W, Cin, Cout, x_dtype, y_dtype);
-    if (ws_bytes < need + stage) return WINO_ERR_WORKSPACE;
+    const size_t stage = staging_one(N, H, W, Cin, Cout, x_dtype, y_dtype);
+    if (ws_bytes < need + wino_host_staging_bytes(p, N, H, W, Cin, Cout, x_dtype, y_dtype)) return WINO_ERR_WORKSPACE;
     const size_t xs = x_dtype == WINO_BF16 ? 2 : 4, ys = y_dtype == WINO_BF16 ? 2 : 4;
     const size_t xrow = xs * H * W * Cin, yrow = ys * H * W * Cout;   // bytes per image
-    HostChain prev = {nullptr, {0, 0, 0, 0, 0}};
+    HostChain prev = {nullptr, 0, 0, 0, nullptr};
     {   // taken out now, set again only when this call is fully enqueued
         std::lock_guard<std::mutex> lock(g_chain_mutex);
         auto it = g_chain.find(ws);
         if (it != g_chain.end()) {
             prev = it->second;
-            g_chain.erase(it);
+            g_chain.erase(it);   // (the event moves to this call)
         }
     }
-    unsigned char* xd = static_cast<unsigned char*>(ws) + need;
+    // Staging: above this call's convolution workspace, and, to overlap the previous host call on
+    // the workspace, above its convolution workspace too and clear of its staging (the top of the
+    // workspace, or just below the previous staging); otherwise right after this call's workspace.
+    size_t s0 = need;
+    bool overlap = false;
+    if (prev.start) {
+        const size_t floor = std::max(need, prev.need);
+        auto clear = [&](size_t a) { return a >= floor && (a + stage <= prev.lo || a >= prev.hi); };
+        const size_t top = (ws_bytes - stage) / kAlign * kAlign;
+        const size_t below = prev.lo >= stage ? (prev.lo - stage) / kAlign * kAlign : 0;
+        if (clear(top)) {
+            s0 = top;
+            overlap = true;
+        } else if (prev.lo >= stage && clear(below)) {
+            s0 = below;
+            overlap = true;
+        }
+    }
+    unsigned char* xd = static_cast<unsigned char*>(ws) + s0;
     unsigned char* yd = xd + up(xrow * N, kAlign);
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     cudaError_t e;
+    cudaEvent_t start = prev.start;
+    if (!start && (e = cudaEventCreateWithFlags(&start, cudaEventDisableTiming)) != cudaSuccess) return cuda_status(p, e);
+    bool recorded = false;   // the start event marks this call on `stream`
+    auto finish = [&](int status) {   // record this call as the workspace's last host call
+        std::lock_guard<std::mutex> lock(g_chain_mutex);
+        auto it = g_chain.find(ws);
+        if (it != g_chain.end()) chain_erase(it);
+        if (!recorded) {   // (an error before the event was recorded: the next call waits for everything)
+            cudaEventDestroy(start);
+            start = nullptr;
+        }
+        g_chain[ws] = HostChain{p, need, s0, s0 + stage, start};
+        return status;
+    };
 
     // Chunks of images: every tile, and so every result, belongs to one image, so the
     // chunks give the same bytes as one call.  Two chunk workspaces must fit below the
     // whole call's error word (which collects the chunks' errors).
     // A chunk's workspace must hold the layout of every chunk size used (the full chunks and the
-    // last, smaller one): a smaller chunk can resolve to the fp32-Y path and need more bytes.
+    // last, smaller one): a smaller chunk can resolve to another kernel variant and need more bytes.
     int K = std::min(N, kMaxHostChunks), Nc = N;
     size_t need_c = need;
     for (; K > 1; --K) {
@@ -603,58 +649,56 @@ int wino_conv2d_int8_host(wino_plan_t p, const void* x_host, int x_dtype, int N,
                     kAlign);
         if (2 * need_c <= L.off_err) break;
     }
-    if (K <= 1) {
+    if (K <= 1) {   // one stream: every step follows all prior work on it
+        if ((e = cudaEventRecord(start, st)) != cudaSuccess) return finish(cuda_status(p, e));
+        recorded = true;
         if ((e = cudaMemcpyAsync(xd, x_host, xrow * N, cudaMemcpyHostToDevice, st)) != cudaSuccess)
-            return cuda_status(p, e);
+            return finish(cuda_status(p, e));
         rc = run_conv(p, xd, x_dtype, N, H, W, Cin, wt, Cout, yd, y_dtype, ws, need, st);
-        if (rc) return rc;
-        return cuda_status(p, cudaMemcpyAsync(y_host, yd, yrow * N, cudaMemcpyDeviceToHost, st));
+        if (rc) return finish(rc);
+        return finish(cuda_status(p, cudaMemcpyAsync(y_host, yd, yrow * N, cudaMemcpyDeviceToHost, st)));
     }
     K = (N + Nc - 1) / Nc;
-    if ((rc = ensure_host_streams(p)) != WINO_OK) return rc;
+    if ((rc = ensure_host_streams(p)) != WINO_OK) return finish(rc);
     cudaEvent_t* ev = p->host_events.data();   // [0]: start, [1 + 3k ..]: in, compute, out of chunk k
     int* err = reinterpret_cast<int*>(static_cast<unsigned char*>(ws) + L.off_err);
-    if ((e = cudaMemsetAsync(err, 0, sizeof(int), st)) != cudaSuccess) return cuda_status(p, e);
-    // The staging buffers behind the workspace are only touched by these calls.  After a call
-    // of the same layout, chunk k's input copy waits for that call's compute of chunk k (the
-    // last reader of its staging slice); otherwise every copy waits for the stream's prior work.
-    const size_t sig[5] = {reinterpret_cast<size_t>(ws), (size_t)K, (size_t)Nc, xrow, yrow};
-    const bool chained = prev.plan == p && std::memcmp(sig, prev.sig, sizeof(sig)) == 0;
-    if (!chained) {
+    // The input copies write only this call's staging.  When it is clear of everything the previous
+    // host call on the workspace uses, they wait for that call's start event (every call before it
+    // is complete, including the last one to use this staging range); otherwise for all prior work
+    // on `stream`.  The output copies wait for this call's convolution of their chunk.
+    if (overlap) {
+        if ((e = cudaStreamWaitEvent(p->copy_in, start, 0)) != cudaSuccess) return finish(cuda_status(p, e));
+    } else {
         cudaEventRecord(ev[0], st);
         cudaStreamWaitEvent(p->copy_in, ev[0], 0);
-        cudaStreamWaitEvent(p->copy_out, ev[0], 0);
     }
+    // this call's start on `stream` (re-recorded after the wait above captured the previous one)
+    if ((e = cudaEventRecord(start, st)) != cudaSuccess) return finish(cuda_status(p, e));
+    recorded = true;
+    if ((e = cudaMemsetAsync(err, 0, sizeof(int), st)) != cudaSuccess) return finish(cuda_status(p, e));
     const unsigned char* xh = static_cast<const unsigned char*>(x_host);
     unsigned char* yh = static_cast<unsigned char*>(y_host);
     for (int k = 0; k < K; ++k) {
         const int n0 = k * Nc, nk = std::min(Nc, N - n0);
         unsigned char* buf = static_cast<unsigned char*>(ws) + (size_t)(k & 1) * need_c;
-        if (chained) cudaStreamWaitEvent(p->copy_in, ev[2 + 3 * k], 0);   // previous call's compute of chunk k
         if ((e = cudaMemcpyAsync(xd + xrow * n0, xh + xrow * n0, xrow * nk, cudaMemcpyHostToDevice, p->copy_in)) !=
             cudaSuccess)
-            return cuda_status(p, e);
+            return finish(cuda_status(p, e));
         cudaEventRecord(ev[1 + 3 * k], p->copy_in);
         cudaStreamWaitEvent(st, ev[1 + 3 * k], 0);
         rc = run_conv(p, xd + xrow * n0, x_dtype, nk, H, W, Cin, wt, Cout, yd + yrow * n0, y_dtype, buf, need_c, st);
-        if (rc) return rc;
+        if (rc) return finish(rc);
         const Layout Lk = make_layout(p, nk, H, W, Cin, Cout);
         if ((e = launch_error_merge(err, reinterpret_cast<const int*>(buf + Lk.off_err), st)) != cudaSuccess)
-            return cuda_status(p, e);
+            return finish(cuda_status(p, e));
         cudaEventRecord(ev[2 + 3 * k], st);
         cudaStreamWaitEvent(p->copy_out, ev[2 + 3 * k], 0);
         if ((e = cudaMemcpyAsync(yh + yrow * n0, yd + yrow * n0, yrow * nk, cudaMemcpyDeviceToHost, p->copy_out)) !=
             cudaSuccess)
-            return cuda_status(p, e);
+            return finish(cuda_status(p, e));
         cudaEventRecord(ev[3 + 3 * k], p->copy_out);
     }
-    {
-        std::lock_guard<std::mutex> lock(g_chain_mutex);
-        HostChain& c = g_chain[ws];
-        c.plan = p;
-        std::memcpy(c.sig, sig, sizeof(sig));
-    }
-    return cuda_status(p, cudaStreamWaitEvent(st, ev[3 * K], 0));
+    return finish(cuda_status(p, cudaStreamWaitEvent(st, ev[3 * K], 0)));
 }
 
 int wino_check_device_error(wino_plan_t p, const void* ws, int N, int H, int W, int Cin, int Cout, void* stream) {

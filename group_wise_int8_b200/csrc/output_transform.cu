@@ -12,11 +12,14 @@
 // One thread per (tile, pair of adjacent couts): the pair shares its Y group,
 // so every step runs on packed fp32 pairs (one two-lane instruction per pair,
 // the per-cout chains and their order unchanged).  Lanes run along cout
-// pairs: every tap load and output store of a warp is contiguous.  Z is built
-// one column of Y at a time, so only Z and one Y column are live.
+// pairs: every tap load and output store of a warp is contiguous.  Column nu
+// of Z is formed from column nu of Y and at once added into every output
+// o[i][j] (whose chain over nu stays in ascending order), so only the output
+// tile and one column are live.
 // Variants: per-tap Y groups (the Y_TAP reading), and, for layers with few
 // (tile, channel pair) items on the fp32-Y path, a split kernel with N threads
 // per item (one per column of Y, then one per output row).
+#include <algorithm>
 #include <cstring>
 
 #include "kernels.h"
@@ -36,11 +39,11 @@ __device__ __forceinline__ uint64_t codes2_to_f2(uint32_t x) {
     return f2_sub(f2_pack(__uint_as_float(lo), __uint_as_float(hi)), f2_pack(off, off));
 }
 
-// Bounded wait for one column's TMA box (records a timeout in the error word).
-__device__ __forceinline__ bool column_wait(uint64_t* bar, int* err) {
-    if (sm100::mbar_try_wait(bar, 0)) return true;
+// Bounded wait for a phase of one column slot's TMA barrier (records a timeout in the error word).
+__device__ __forceinline__ bool column_wait(uint64_t* bar, uint32_t parity, int* err) {
+    if (sm100::mbar_try_wait(bar, parity)) return true;
     const unsigned long long t0 = sm100::globaltimer();
-    while (!sm100::mbar_try_wait(bar, 0))
+    while (!sm100::mbar_try_wait(bar, parity))
         if (sm100::globaltimer() - t0 > sm100::kWaitLimitNs) {
             atomicCAS(err, 0, sm100::kDevErrTimeout);
             return false;
@@ -48,27 +51,32 @@ __device__ __forceinline__ bool column_wait(uint64_t* bar, int* err) {
     return true;
 }
 
+constexpr int kYRing = 4;   // column slots of the fp32 source: 4 x 8 KiB for F(6,3), four CTAs per SM
+
 template <int M, uint64_t MASK, bool SRC_Y32, bool BF16_OUT, bool DEBUG>
-__global__ void __launch_bounds__(128, SRC_Y32 ? 3 : 4)
+__global__ void __launch_bounds__(128, 4)
     output_transform_kernel(const __grid_constant__ CUtensorMap tmY, OutputArgs p, TransformArgs tf) {
     constexpr int N = M + 2, N2 = N * N;
     // The CTA's 128 cout pairs are 256 consecutive elements of every tap's [T][Cout] plane.  One 3-D
     // TMA box per column nu of Y (taps xi * N + nu, every xi) brings them to shared memory as
-    // [nu][xi][256] (int8 source: 256 bytes per tap, static; fp32 source: 1 KiB per tap, dynamic),
-    // each column on its own barrier, so the transform of column nu overlaps the later columns' loads.
+    // [xi][256], each column slot on its own barrier.  The int8 source keeps every column (256 bytes
+    // per tap, static); the fp32 source cycles R = kYRing slots (1 KiB per tap, dynamic): once every
+    // thread has read column nu, its slot is refilled with column nu + R, so the transform of the
+    // first columns overlaps the later columns' loads and a CTA holds 4 columns instead of N.
+    constexpr int R = (SRC_Y32 && kYRing < N) ? kYRing : N;
+    constexpr uint32_t kColBytes = (SRC_Y32 ? 1024u : 256u) * N;
     __shared__ __align__(128) uint8_t ysm[SRC_Y32 ? 16 : 256 * N2];
     extern __shared__ __align__(128) unsigned char ydyn[];
-    __shared__ uint64_t bar[N];
-    constexpr uint32_t kColBytes = (SRC_Y32 ? 1024u : 256u) * N;
+    unsigned char* ybuf = SRC_Y32 ? ydyn : ysm;
+    __shared__ uint64_t bar[R];
     grid_dependents_launch();
     grid_dependency_wait();
     if (threadIdx.x == 0) {
-        for (int nu = 0; nu < N; ++nu) sm100::mbar_init(&bar[nu], 1);
+        for (int s = 0; s < R; ++s) sm100::mbar_init(&bar[s], 1);
         sm100::fence_mbar_init();
-        for (int nu = 0; nu < N; ++nu) {
+        for (int nu = 0; nu < R; ++nu) {
             sm100::mbar_arrive_expect_tx(&bar[nu], kColBytes);
-            unsigned char* dst = (SRC_Y32 ? ydyn : ysm) + (size_t)nu * kColBytes;
-            sm100::tma_load_3d(dst, &tmY, &bar[nu], (int)(blockIdx.x * 256u), nu, 0);
+            sm100::tma_load_3d(ybuf + (size_t)nu * kColBytes, &tmY, &bar[nu], (int)(blockIdx.x * 256u), nu, 0);
         }
     }
     __syncthreads();
@@ -79,57 +87,74 @@ __global__ void __launch_bounds__(128, SRC_Y32 ? 3 : 4)
     const int cg = co / p.G;
     const size_t base = (size_t)t * p.Cout + co;   // Yq / Y32 are tap-major [n2][T][Cout]
     const size_t tstride = (size_t)p.T * p.Cout;
-    // every Y element this thread touches lies in [base, base + (N2 - 1) * tstride + 1]
-    if (t >= p.T || !in_bounds((size_t)t * p.ngo + cg, p.n_amax, p.err) ||
-        ((SRC_Y32 || DEBUG) && !in_bounds(base + (size_t)(N2 - 1) * tstride + 1, p.n_y, p.err)) ||
-        (DEBUG && !in_bounds((size_t)t * p.ngo + cg, p.n_sy, p.err))) {
-        // an idle thread 0 still sees every load land before the CTA's shared memory is released
-        if (threadIdx.x == 0)
-            for (int nu = 0; nu < N; ++nu)
-                if (!column_wait(&bar[nu], p.err)) break;
-        return;
-    }
-    const QScale qs = make_qscale(__uint_as_float(p.amax[(size_t)t * p.ngo + cg]));
-    if (DEBUG && co % p.G == 0) p.sY_dbg[(size_t)t * p.ngo + cg] = qs.s;
+    // every Y element this thread touches lies in [base, base + (N2 - 1) * tstride + 1]; a thread
+    // past the last tile (or failing a debug-build index check) still takes part in the ring
+    const bool active = t < p.T && in_bounds((size_t)t * p.ngo + cg, p.n_amax, p.err) &&
+                        (!(SRC_Y32 || DEBUG) || in_bounds(base + (size_t)(N2 - 1) * tstride + 1, p.n_y, p.err)) &&
+                        (!DEBUG || in_bounds((size_t)t * p.ngo + cg, p.n_sy, p.err));
+    const QScale qs = make_qscale(active ? __uint_as_float(p.amax[(size_t)t * p.ngo + cg]) : 0.0f);
+    if (DEBUG && active && co % p.G == 0) p.sY_dbg[(size_t)t * p.ngo + cg] = qs.s;
     const uint64_t s2 = f2_pack(qs.s, qs.s);
 
-    uint64_t Z[M][N];                              // (co, co + 1) pairs
+    // o[r][c] = fma chain over ascending nu of Z[r][nu] * AT[c][nu], with Z[r][nu] = fma chain over
+    // ascending xi of AT[r][xi] * Yd[xi][nu]: column nu of Z is formed and used at once, so only the
+    // output tile (M x M pairs) and one column stay live
+    uint64_t o[M][M];
+#pragma unroll
+    for (int r = 0; r < M; ++r)
+#pragma unroll
+        for (int c = 0; c < M; ++c) o[r][c] = 0ull;
+    bool ok = true;
 #pragma unroll
     for (int nu = 0; nu < N; ++nu) {
+        const int slot = nu % R;
+        if (ok && !column_wait(&bar[slot], (uint32_t)((nu / R) & 1), p.err)) ok = false;
         uint64_t Yc[N];                            // column nu of Yd: taps xi * N + nu
-        if (!column_wait(&bar[nu], p.err)) return;   // only on a timeout (error word set)
         if (SRC_Y32) {
-            const float* ys = reinterpret_cast<const float*>(ydyn) + 2 * threadIdx.x;   // + (nu * N + xi) * 256
+            const float* ys = reinterpret_cast<const float*>(ybuf + (size_t)slot * kColBytes) + 2 * threadIdx.x;
 #pragma unroll
             for (int xi = 0; xi < N; xi += 2) {
-                const float2 a = *reinterpret_cast<const float2*>(ys + (nu * N + xi) * 256);
-                const float2 b = *reinterpret_cast<const float2*>(ys + (nu * N + xi + 1) * 256);
+                const float2 a = *reinterpret_cast<const float2*>(ys + xi * 256);
+                const float2 b = *reinterpret_cast<const float2*>(ys + (xi + 1) * 256);
                 const Quad qd = quant4(a.x, a.y, b.x, b.y, qs);
                 Yc[xi] = f2_mul(s2, qd.k01);
                 Yc[xi + 1] = f2_mul(s2, qd.k23);
-                if (DEBUG) {
+                if (DEBUG && active) {
                     *reinterpret_cast<uint16_t*>(p.Yq_dbg + base + (size_t)(xi * N + nu) * tstride) =
                         (uint16_t)(qd.packed & 0xffffu);
                     *reinterpret_cast<uint16_t*>(p.Yq_dbg + base + (size_t)((xi + 1) * N + nu) * tstride) =
                         (uint16_t)(qd.packed >> 16);
                 }
             }
+            if (nu + R < N) {   // every thread has read the slot: refill it with column nu + R
+                __syncthreads();
+                if (threadIdx.x == 0 && ok) {
+                    sm100::fence_proxy_async_smem();
+                    sm100::mbar_arrive_expect_tx(&bar[slot], kColBytes);
+                    sm100::tma_load_3d(ybuf + (size_t)slot * kColBytes, &tmY, &bar[slot], (int)(blockIdx.x * 256u),
+                                       nu + R, 0);
+                }
+            }
         } else {
 #pragma unroll
             for (int xi = 0; xi < N; ++xi) {
-                const uint32_t x = *reinterpret_cast<const uint16_t*>(ysm + (nu * N + xi) * 256 + 2 * threadIdx.x);
+                const uint32_t x = *reinterpret_cast<const uint16_t*>(ybuf + (size_t)slot * kColBytes + xi * 256 +
+                                                                       2 * threadIdx.x);
                 Yc[xi] = f2_mul(s2, codes2_to_f2(x));
             }
         }
 #pragma unroll
         for (int r = 0; r < M; ++r) {
-            uint64_t acc = 0ull;
+            uint64_t z = 0ull;
 #pragma unroll
             for (int xi = 0; xi < N; ++xi)
-                if ((MASK >> (r * N + xi)) & 1ull) acc = f2_fma(tf.ATd[r * N + xi], Yc[xi], acc);
-            Z[r][nu] = acc;
+                if ((MASK >> (r * N + xi)) & 1ull) z = f2_fma(tf.ATd[r * N + xi], Yc[xi], z);
+#pragma unroll
+            for (int c = 0; c < M; ++c)
+                if ((MASK >> (c * N + nu)) & 1ull) o[r][c] = f2_fma(z, tf.ATd[c * N + nu], o[r][c]);
         }
     }
+    if (!active || !ok) return;
     const int TT = p.TH * p.TW;
     const int img = (int)(t / TT);
     const int rem = (int)(t - (long)img * TT);
@@ -142,19 +167,15 @@ __global__ void __launch_bounds__(128, SRC_Y32 ? 3 : 4)
         for (int c = 0; c < M; ++c) {
             const int xx = tx * M + c;
             if (xx >= p.W) break;
-            uint64_t acc = 0ull;
-#pragma unroll
-            for (int nu = 0; nu < N; ++nu)
-                if ((MASK >> (c * N + nu)) & 1ull) acc = f2_fma(Z[r][nu], tf.ATd[c * N + nu], acc);
             float o0, o1;
-            f2_unpack(acc, o0, o1);
-            const size_t o = (((size_t)img * p.H + yy) * p.W + xx) * p.Cout + co;
-            if (!in_bounds(o + 1, p.n_out, p.err)) continue;
+            f2_unpack(o[r][c], o0, o1);
+            const size_t oi = (((size_t)img * p.H + yy) * p.W + xx) * p.Cout + co;
+            if (!in_bounds(oi + 1, p.n_out, p.err)) continue;
             if (BF16_OUT)
-                *reinterpret_cast<__nv_bfloat162*>(reinterpret_cast<__nv_bfloat16*>(p.out) + o) =
+                *reinterpret_cast<__nv_bfloat162*>(reinterpret_cast<__nv_bfloat16*>(p.out) + oi) =
                     __floats2bfloat162_rn(o0, o1);
             else
-                *reinterpret_cast<float2*>(reinterpret_cast<float*>(p.out) + o) = make_float2(o0, o1);
+                *reinterpret_cast<float2*>(reinterpret_cast<float*>(p.out) + oi) = make_float2(o0, o1);
         }
     }
 }
@@ -417,7 +438,8 @@ cudaError_t launch_m(const OutputArgs& a, const TransformArgs& tf, bool src_y32,
         }
 #undef WINO_SPLIT_LAUNCH
     }
-    const size_t dsmem = src_y32 ? (size_t)1024 * a.n2 : 0;   // fp32 source: 1 KiB per tap
+    // fp32 source: a ring of kYRing column slots of 1 KiB per tap (every column when there are fewer)
+    const size_t dsmem = src_y32 ? (size_t)1024 * std::min(kYRing, M + 2) * (M + 2) : 0;
 #define WINO_OUT_LAUNCH(Y32, BF, DBG)                                                                          \
     do {                                                                                                     \
         auto kern = output_transform_kernel<M, MASK, Y32, BF, DBG>;                                          \

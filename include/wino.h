@@ -252,8 +252,9 @@ int wino_conv2d_int8_noalloc(wino_plan_t plan, const void* x_dev, int x_dtype, i
  * WORKSPACE (shape beyond the array), CUDA. */
 int wino_check_device_error_noalloc(wino_plan_t plan, int N, int H, int W, int Cin, int Cout, void* stream);
 
-/* Extra device bytes wino_conv2d_int8_host needs beyond wino_workspace_bytes
- * (device staging for x and y). */
+/* Extra device bytes wino_conv2d_int8_host needs beyond wino_workspace_bytes:
+ * device staging for x and y, twice (room for two calls' staging, so that
+ * consecutive host calls on one workspace overlap; see below). */
 size_t wino_host_staging_bytes(wino_plan_t plan, int N, int H, int W, int Cin, int Cout, int x_dtype,
                                int y_dtype);
 
@@ -266,15 +267,19 @@ size_t wino_host_staging_bytes(wino_plan_t plan, int N, int H, int W, int Cin, i
  * k-1 out overlap the convolution of chunk k (the copies run on two streams
  * the plan owns, ordered after and before `stream` by events; results are
  * identical to one call, every tile belonging to one image).  ws_dev must hold
- * wino_workspace_bytes() + wino_host_staging_bytes().  The caller synchronises
- * `stream` before reading y_host.  Calls on one plan must not run concurrently.
- * Back-to-back calls of the same plan and shape on the same workspace overlap:
- * each chunk's input copy waits only for the previous call's convolution of
- * that chunk, so the next batch streams in while the previous one finishes.
- * Any other call on ws_dev in between (another plan or shape, or
- * wino_conv2d_int8) ends that chaining, so the next host call waits for all
- * prior work on `stream`.  Work outside this library must not use ws_dev, and
- * x_host must not change until the call's work on `stream` has completed.
+ * wino_workspace_bytes() + wino_host_staging_bytes() (else WINO_ERR_WORKSPACE).
+ * The caller synchronises `stream` before reading y_host.  Calls on one plan
+ * must not run concurrently.  Consecutive host calls on one workspace (any
+ * plans and shapes, issued on one stream) overlap: a call stages x and y where
+ * they touch neither the previous host call's convolution workspace nor its
+ * staging (the top of ws_dev, or just below the previous staging), and its
+ * input copies then wait only until every call before the previous one is
+ * complete, so they stream in during the previous call's convolution and
+ * output copies.  When no such place fits in ws_bytes (a workspace sized for a
+ * smaller shape), the call waits for all prior work on `stream`, and so does
+ * the first host call after a wino_conv2d_int8 call on ws_dev.  Work outside
+ * this library must not use ws_dev, and x_host must not change until the
+ * call's work on `stream` has completed.
  */
 int wino_conv2d_int8_host(wino_plan_t plan, const void* x_host, int x_dtype, int N, int H, int W, int Cin,
                            const void* wt_dev, int Cout, void* y_host, int y_dtype, void* ws_dev, size_t ws_bytes,

@@ -299,6 +299,43 @@ def test_host_calls_of_two_plans_sharing_a_workspace(cuda_dev):
         assert torch.equal(ys[k], want[k]), k
 
 
+@pytest.mark.parametrize("room", ["overlap", "tight"])
+def test_host_calls_of_several_shapes_on_one_workspace(cuda_dev, room):
+    """Back-to-back host calls cycling through three layers of different shapes and plans on one
+    workspace, each call with its own input and output buffers and no synchronisation between
+    calls: with room for two stagings above the largest convolution workspace every call's input
+    copies overlap the previous call; on a workspace sized for the largest single call some calls
+    find no clear staging and wait.  Every output equals the device entry point's."""
+    shapes = [(6, 14, 13, 64, 64, 32), (4, 20, 20, 128, 64, 64), (3, 9, 10, 64, 128, 32)]
+    plans, wts, need, stage = [], [], [], []
+    for k, (N, H, W, Cin, Cout, G) in enumerate(shapes):
+        layer = synth.random_layer(300 + k, 6, N, H, W, Cin, Cout, G, dtype="bf16", act="relu_normal",
+                                   workload="host_shapes")
+        sb, sg = synth.make_scales(layer)
+        plan = wino.Plan(6, P6, sb, sg, G)
+        plans.append(plan)
+        wts.append(plan.transform_weights(torch.from_numpy(synth.make_weights(layer)).cuda()))
+        need.append(plan.workspace_bytes(N, H, W, Cin, Cout))
+        stage.append(plan.host_staging_bytes(N, H, W, Cin, Cout, torch.bfloat16, torch.bfloat16))
+    size = max(need) + max(stage) if room == "overlap" else max(n + st for n, st in zip(need, stage))
+    ws = torch.empty(size, dtype=torch.uint8, device="cuda")
+    calls = []
+    for rep in range(3):
+        for k, (N, H, W, Cin, Cout, G) in enumerate(shapes):
+            g = torch.Generator().manual_seed(1000 * rep + k)
+            x = (torch.randn((N, H, W, Cin), generator=g) * (1 + rep)).to(torch.bfloat16).pin_memory()
+            y = torch.full((N, H, W, Cout), float("nan"), dtype=torch.bfloat16).pin_memory()
+            calls.append((k, x, y))
+    for k, x, y in calls:
+        plans[k].conv2d_host(x, wts[k], shapes[k][4], y, ws)
+    torch.cuda.synchronize()
+    k_last = calls[-1][0]   # the error word belongs to the last call's layout
+    assert plans[k_last].check_device_error(ws, *shapes[k_last][:5]) == wino.OK
+    for i, (k, x, y) in enumerate(calls):
+        want = plans[k].conv2d(x.cuda(), wts[k], shapes[k][4], out_dtype=torch.bfloat16).cpu()
+        assert torch.equal(y.view(torch.int16), want.view(torch.int16)), i
+
+
 def test_repeated_calls_reuse_workspace(cuda_dev):
     """The workspace carries nothing between calls: a second call on a dirty
     workspace gives the same bits."""
