@@ -640,6 +640,29 @@ int wino_conv2d_int8_host(wino_plan_t p, const void* x_host, int x_dtype, int N,
     // whole call's error word (which collects the chunks' errors).
     // A chunk's workspace must hold the layout of every chunk size used (the full chunks and the
     // last, smaller one): a smaller chunk can resolve to another kernel variant and need more bytes.
+    if (overlap) {
+        // The previous host call on this workspace covers this one's input copy: the whole batch
+        // is copied in on the copy stream while that call computes and copies out, then runs as
+        // one convolution on `stream` (its weights read once) and is copied out.
+        if ((rc = ensure_host_streams(p)) != WINO_OK) return finish(rc);
+        cudaEvent_t* ev = p->host_events.data();
+        if ((e = cudaStreamWaitEvent(p->copy_in, start, 0)) != cudaSuccess) return finish(cuda_status(p, e));
+        if ((e = cudaEventRecord(start, st)) != cudaSuccess) return finish(cuda_status(p, e));
+        recorded = true;
+        if ((e = cudaMemcpyAsync(xd, x_host, xrow * N, cudaMemcpyHostToDevice, p->copy_in)) != cudaSuccess)
+            return finish(cuda_status(p, e));
+        cudaEventRecord(ev[1], p->copy_in);
+        cudaStreamWaitEvent(st, ev[1], 0);
+        rc = run_conv(p, xd, x_dtype, N, H, W, Cin, wt, Cout, yd, y_dtype, ws, need, st);
+        if (rc) return finish(rc);
+        cudaEventRecord(ev[2], st);
+        cudaStreamWaitEvent(p->copy_out, ev[2], 0);
+        if ((e = cudaMemcpyAsync(y_host, yd, yrow * N, cudaMemcpyDeviceToHost, p->copy_out)) != cudaSuccess)
+            return finish(cuda_status(p, e));
+        cudaEventRecord(ev[3], p->copy_out);
+        return finish(cuda_status(p, cudaStreamWaitEvent(st, ev[3], 0)));
+    }
+
     int K = std::min(N, kMaxHostChunks), Nc = N;
     size_t need_c = need;
     for (; K > 1; --K) {
@@ -662,17 +685,12 @@ int wino_conv2d_int8_host(wino_plan_t p, const void* x_host, int x_dtype, int N,
     if ((rc = ensure_host_streams(p)) != WINO_OK) return finish(rc);
     cudaEvent_t* ev = p->host_events.data();   // [0]: start, [1 + 3k ..]: in, compute, out of chunk k
     int* err = reinterpret_cast<int*>(static_cast<unsigned char*>(ws) + L.off_err);
-    // The input copies write only this call's staging.  When it is clear of everything the previous
-    // host call on the workspace uses, they wait for that call's start event (every call before it
-    // is complete, including the last one to use this staging range); otherwise for all prior work
-    // on `stream`.  The output copies wait for this call's convolution of their chunk.
-    if (overlap) {
-        if ((e = cudaStreamWaitEvent(p->copy_in, start, 0)) != cudaSuccess) return finish(cuda_status(p, e));
-    } else {
-        cudaEventRecord(ev[0], st);
-        cudaStreamWaitEvent(p->copy_in, ev[0], 0);
-    }
-    // this call's start on `stream` (re-recorded after the wait above captured the previous one)
+    // Without a previous host call to overlap, the input copies wait for all prior work on `stream`
+    // (the staging may hold what earlier work still reads); the output copies wait for this call's
+    // convolution of their chunk.
+    cudaEventRecord(ev[0], st);
+    cudaStreamWaitEvent(p->copy_in, ev[0], 0);
+    // this call's start on `stream`: the next host call's input copies wait for it
     if ((e = cudaEventRecord(start, st)) != cudaSuccess) return finish(cuda_status(p, e));
     recorded = true;
     if ((e = cudaMemsetAsync(err, 0, sizeof(int), st)) != cudaSuccess) return finish(cuda_status(p, e));

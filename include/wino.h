@@ -272,10 +272,11 @@ size_t wino_host_staging_bytes(wino_plan_t plan, int N, int H, int W, int Cin, i
  * must not run concurrently.  Consecutive host calls on one workspace (any
  * plans and shapes, issued on one stream) overlap: a call stages x and y where
  * they touch neither the previous host call's convolution workspace nor its
- * staging (the top of ws_dev, or just below the previous staging), and its
- * input copies then wait only until every call before the previous one is
- * complete, so they stream in during the previous call's convolution and
- * output copies.  When no such place fits in ws_bytes (a workspace sized for a
+ * staging (the top of ws_dev, or just below the previous staging), its input
+ * copy then waits only until every call before the previous one is complete,
+ * so it streams in during the previous call's convolution and output copy, and
+ * the batch runs as one convolution (its weights read once).  When no such
+ * place fits in ws_bytes (a workspace sized for a
  * smaller shape), the call waits for all prior work on `stream`, and so does
  * the first host call after a wino_conv2d_int8 call on ws_dev.  Work outside
  * this library must not use ws_dev, and x_host must not change until the
