@@ -182,23 +182,27 @@ int cuda_status(wino_plan_s* p, cudaError_t e) {
 
 constexpr int kMaxHostChunks = 3;
 
-// The last host call on each workspace: its plan, the bytes its convolution used from the
-// workspace's start (need) and its staging range [lo, hi), and an event recorded on its stream
-// when it began (so it fires once every call before it is complete).  The next host call on the
-// workspace puts its staging where it touches neither of those ranges, when that fits, and then
-// orders its input copies only after that event: they overlap the previous call's convolution
-// and output copies.  Any other use of the workspace (the device-buffer entry point) ends the
-// chain, and so does destroying the plan.
+// The last two host calls on each workspace ([0] the latest): their plan, the bytes each one's
+// convolution used from the workspace's start (need) and its staging range [lo, hi), and an event
+// recorded on its stream when it began (so it fires once every call before it is complete).  The
+// next host call on the workspace puts its staging where it touches none of those ranges, when
+// that fits, and then orders its input copy only after the older call's event: it streams in
+// during both calls' convolutions and output copies.  Any other use of the workspace (the
+// device-buffer entry point) ends the chain, and so does destroying a plan of either call.
+struct HostCall {
+    size_t need = 0, lo = 0, hi = 0;
+    cudaEvent_t start = nullptr;
+};
 struct HostChain {
-    const wino_plan_s* plan;
-    size_t need, lo, hi;
-    cudaEvent_t start;
+    const wino_plan_s* plan[2] = {nullptr, nullptr};
+    HostCall call[2];
 };
 std::mutex g_chain_mutex;
 std::unordered_map<const void*, HostChain> g_chain;
 
 void chain_erase(std::unordered_map<const void*, HostChain>::iterator it) {
-    if (it->second.start) cudaEventDestroy(it->second.start);
+    for (HostCall& c : it->second.call)
+        if (c.start) cudaEventDestroy(c.start);
     g_chain.erase(it);
 }
 
@@ -212,7 +216,7 @@ void chain_forget_plan(const wino_plan_s* p) {
     std::lock_guard<std::mutex> lock(g_chain_mutex);
     for (auto it = g_chain.begin(); it != g_chain.end();) {
         auto next = std::next(it);
-        if (it->second.plan == p) chain_erase(it);
+        if (it->second.plan[0] == p || it->second.plan[1] == p) chain_erase(it);
         it = next;
     }
 }
@@ -574,7 +578,7 @@ size_t staging_one(int N, int H, int W, int Cin, int Cout, int x_dtype, int y_dt
 
 size_t wino_host_staging_bytes(wino_plan_t p, int N, int H, int W, int Cin, int Cout, int x_dtype, int y_dtype) {
     if (check_shape(p, N, H, W, Cin, Cout)) return 0;
-    return 2 * staging_one(N, H, W, Cin, Cout, x_dtype, y_dtype);   // two calls' staging: consecutive calls overlap
+    return 3 * staging_one(N, H, W, Cin, Cout, x_dtype, y_dtype);   // three calls' staging: consecutive calls overlap
 }
 
 int wino_conv2d_int8_host(wino_plan_t p, const void* x_host, int x_dtype, int N, int H, int W, int Cin,
@@ -589,49 +593,70 @@ int wino_conv2d_int8_host(wino_plan_t p, const void* x_host, int x_dtype, int N,
     if (ws_bytes < need + wino_host_staging_bytes(p, N, H, W, Cin, Cout, x_dtype, y_dtype)) return WINO_ERR_WORKSPACE;
     const size_t xs = x_dtype == WINO_BF16 ? 2 : 4, ys = y_dtype == WINO_BF16 ? 2 : 4;
     const size_t xrow = xs * H * W * Cin, yrow = ys * H * W * Cout;   // bytes per image
-    HostChain prev = {nullptr, 0, 0, 0, nullptr};
+    HostChain prev;
     {   // taken out now, set again only when this call is fully enqueued
         std::lock_guard<std::mutex> lock(g_chain_mutex);
         auto it = g_chain.find(ws);
         if (it != g_chain.end()) {
             prev = it->second;
-            g_chain.erase(it);   // (the event moves to this call)
+            g_chain.erase(it);   // (its events move to this call's record)
         }
     }
-    // Staging: above this call's convolution workspace, and, to overlap the previous host call on
-    // the workspace, above its convolution workspace too and clear of its staging (the top of the
-    // workspace, or just below the previous staging); otherwise right after this call's workspace.
+    // Staging: above this call's convolution workspace and, to overlap the last host calls on the
+    // workspace (the latest, and the one before it when there is one), above theirs and clear of
+    // their staging ranges: the top of the workspace, just below one of their stagings, or right
+    // above the highest convolution workspace.  Otherwise right after this call's workspace.
+    const int nprev = prev.call[0].start ? (prev.call[1].start ? 2 : 1) : 0;
     size_t s0 = need;
     bool overlap = false;
-    if (prev.start) {
-        const size_t floor = std::max(need, prev.need);
-        auto clear = [&](size_t a) { return a >= floor && (a + stage <= prev.lo || a >= prev.hi); };
-        const size_t top = (ws_bytes - stage) / kAlign * kAlign;
-        const size_t below = prev.lo >= stage ? (prev.lo - stage) / kAlign * kAlign : 0;
-        if (clear(top)) {
-            s0 = top;
-            overlap = true;
-        } else if (prev.lo >= stage && clear(below)) {
-            s0 = below;
-            overlap = true;
-        }
+    if (nprev > 0) {
+        size_t floor = need;
+        for (int i = 0; i < nprev; ++i) floor = std::max(floor, prev.call[i].need);
+        auto clear = [&](size_t a) {
+            if (a < floor || a + stage > ws_bytes) return false;
+            for (int i = 0; i < nprev; ++i)
+                if (a + stage > prev.call[i].lo && a < prev.call[i].hi) return false;
+            return true;
+        };
+        size_t cand[4];
+        int nc = 0;
+        cand[nc++] = (ws_bytes - stage) / kAlign * kAlign;
+        for (int i = 0; i < nprev; ++i)
+            if (prev.call[i].lo >= stage) cand[nc++] = (prev.call[i].lo - stage) / kAlign * kAlign;
+        cand[nc++] = up(floor, kAlign);
+        for (int i = 0; i < nc && !overlap; ++i)
+            if (clear(cand[i])) {
+                s0 = cand[i];
+                overlap = true;
+            }
     }
     unsigned char* xd = static_cast<unsigned char*>(ws) + s0;
     unsigned char* yd = xd + up(xrow * N, kAlign);
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     cudaError_t e;
-    cudaEvent_t start = prev.start;
+    // The input copy of an overlapping call waits for the start of the oldest call it overlaps
+    // (every call before that one is complete, including the last one to use this staging range).
+    cudaEvent_t wait_ev = nprev > 0 ? prev.call[nprev - 1].start : nullptr;
+    // This call's start event: the object of the call that drops out of the record (two back),
+    // after the wait above has captured its last record, or a new one.
+    cudaEvent_t start = nprev == 2 ? prev.call[1].start : nullptr;
     if (!start && (e = cudaEventCreateWithFlags(&start, cudaEventDisableTiming)) != cudaSuccess) return cuda_status(p, e);
     bool recorded = false;   // the start event marks this call on `stream`
-    auto finish = [&](int status) {   // record this call as the workspace's last host call
+    auto finish = [&](int status) {   // record this call as the workspace's latest host call
         std::lock_guard<std::mutex> lock(g_chain_mutex);
         auto it = g_chain.find(ws);
         if (it != g_chain.end()) chain_erase(it);
-        if (!recorded) {   // (an error before the event was recorded: the next call waits for everything)
+        HostChain c;
+        if (recorded) {
+            c.plan[0] = p;
+            c.call[0] = HostCall{need, s0, s0 + stage, start};
+            c.plan[1] = prev.plan[0];
+            c.call[1] = prev.call[0];
+        } else {   // (an error before the event was recorded: the next call waits for everything)
             cudaEventDestroy(start);
-            start = nullptr;
+            if (prev.call[0].start) cudaEventDestroy(prev.call[0].start);
         }
-        g_chain[ws] = HostChain{p, need, s0, s0 + stage, start};
+        g_chain[ws] = c;
         return status;
     };
 
@@ -646,7 +671,7 @@ int wino_conv2d_int8_host(wino_plan_t p, const void* x_host, int x_dtype, int N,
         // one convolution on `stream` (its weights read once) and is copied out.
         if ((rc = ensure_host_streams(p)) != WINO_OK) return finish(rc);
         cudaEvent_t* ev = p->host_events.data();
-        if ((e = cudaStreamWaitEvent(p->copy_in, start, 0)) != cudaSuccess) return finish(cuda_status(p, e));
+        if ((e = cudaStreamWaitEvent(p->copy_in, wait_ev, 0)) != cudaSuccess) return finish(cuda_status(p, e));
         if ((e = cudaEventRecord(start, st)) != cudaSuccess) return finish(cuda_status(p, e));
         recorded = true;
         if ((e = cudaMemcpyAsync(xd, x_host, xrow * N, cudaMemcpyHostToDevice, p->copy_in)) != cudaSuccess)

@@ -253,8 +253,8 @@ int wino_conv2d_int8_noalloc(wino_plan_t plan, const void* x_dev, int x_dtype, i
 int wino_check_device_error_noalloc(wino_plan_t plan, int N, int H, int W, int Cin, int Cout, void* stream);
 
 /* Extra device bytes wino_conv2d_int8_host needs beyond wino_workspace_bytes:
- * device staging for x and y, twice (room for two calls' staging, so that
- * consecutive host calls on one workspace overlap; see below). */
+ * device staging for x and y, three times (room for three calls' staging, so
+ * that consecutive host calls on one workspace overlap; see below). */
 size_t wino_host_staging_bytes(wino_plan_t plan, int N, int H, int W, int Cin, int Cout, int x_dtype,
                                int y_dtype);
 
@@ -271,11 +271,12 @@ size_t wino_host_staging_bytes(wino_plan_t plan, int N, int H, int W, int Cin, i
  * The caller synchronises `stream` before reading y_host.  Calls on one plan
  * must not run concurrently.  Consecutive host calls on one workspace (any
  * plans and shapes, issued on one stream) overlap: a call stages x and y where
- * they touch neither the previous host call's convolution workspace nor its
- * staging (the top of ws_dev, or just below the previous staging), its input
- * copy then waits only until every call before the previous one is complete,
- * so it streams in during the previous call's convolution and output copy, and
- * the batch runs as one convolution (its weights read once).  When no such
+ * they touch neither the last two host calls' convolution workspaces nor their
+ * staging (the top of ws_dev, just below one of their stagings, or above the
+ * largest of the three convolution workspaces), its input copy then waits only
+ * until every call before those two is complete, so it streams in during their
+ * convolutions and output copies, and the batch runs as one convolution (its
+ * weights read once).  When no such
  * place fits in ws_bytes (a workspace sized for a
  * smaller shape), the call waits for all prior work on `stream`, and so does
  * the first host call after a wino_conv2d_int8 call on ws_dev.  Work outside
