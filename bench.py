@@ -68,6 +68,10 @@ NCU_TRAFFIC = {
     ("F(6,3) N8 320->320 64x64 G64", "hadamard_y32"): 61982464,
     # profiles/output_transform_y32_sd15_320x320_64x64_full.md: 79,385,600 + 3,409,920 B
     ("F(6,3) N8 320->320 64x64 G64", "output_transform"): 82795520,
+    # profiles/input_transform_sd15_320x320_64x64_full.md: 21,031,168 + 85,760 B
+    ("F(6,3) N8 320->320 64x64 G64", "input_transform"): 21116928,
+    # profiles/hadamard_y32_probe_T2048_C2560_full.md: 6.022703 GB + 1.330437 GB (ncu rounds to 1 kB)
+    ("F(6,3) N2 2560->2560 192x192 G64", "hadamard_y32"): 7353140000,
 }
 
 
