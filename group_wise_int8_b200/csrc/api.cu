@@ -640,7 +640,10 @@ int wino_conv2d_int8_host(wino_plan_t p, const void* x_host, int x_dtype, int N,
     // This call's start event: the object of the call that drops out of the record (two back),
     // after the wait above has captured its last record, or a new one.
     cudaEvent_t start = nprev == 2 ? prev.call[1].start : nullptr;
-    if (!start && (e = cudaEventCreateWithFlags(&start, cudaEventDisableTiming)) != cudaSuccess) return cuda_status(p, e);
+    if (!start && (e = cudaEventCreateWithFlags(&start, cudaEventDisableTiming)) != cudaSuccess) {
+        if (prev.call[0].start) cudaEventDestroy(prev.call[0].start);   // (the record is dropped)
+        return cuda_status(p, e);
+    }
     bool recorded = false;   // the start event marks this call on `stream`
     auto finish = [&](int status) {   // record this call as the workspace's latest host call
         std::lock_guard<std::mutex> lock(g_chain_mutex);
@@ -660,15 +663,10 @@ int wino_conv2d_int8_host(wino_plan_t p, const void* x_host, int x_dtype, int N,
         return status;
     };
 
-    // Chunks of images: every tile, and so every result, belongs to one image, so the
-    // chunks give the same bytes as one call.  Two chunk workspaces must fit below the
-    // whole call's error word (which collects the chunks' errors).
-    // A chunk's workspace must hold the layout of every chunk size used (the full chunks and the
-    // last, smaller one): a smaller chunk can resolve to another kernel variant and need more bytes.
     if (overlap) {
-        // The previous host call on this workspace covers this one's input copy: the whole batch
-        // is copied in on the copy stream while that call computes and copies out, then runs as
-        // one convolution on `stream` (its weights read once) and is copied out.
+        // The last host calls on this workspace cover this one's input copy: the whole batch is
+        // copied in on the copy stream while they compute and copy out, then runs as one
+        // convolution on `stream` (its weights read once) and is copied out.
         if ((rc = ensure_host_streams(p)) != WINO_OK) return finish(rc);
         cudaEvent_t* ev = p->host_events.data();
         if ((e = cudaStreamWaitEvent(p->copy_in, wait_ev, 0)) != cudaSuccess) return finish(cuda_status(p, e));
@@ -688,6 +686,11 @@ int wino_conv2d_int8_host(wino_plan_t p, const void* x_host, int x_dtype, int N,
         return finish(cuda_status(p, cudaStreamWaitEvent(st, ev[3], 0)));
     }
 
+    // Otherwise, chunks of images: every tile, and so every result, belongs to one image, so the
+    // chunks give the same bytes as one call.  Two chunk workspaces must fit below the whole
+    // call's error word (which collects the chunks' errors).  A chunk's workspace must hold the
+    // layout of every chunk size used (the full chunks and the last, smaller one): a smaller chunk
+    // can resolve to another kernel variant and need more bytes.
     int K = std::min(N, kMaxHostChunks), Nc = N;
     size_t need_c = need;
     for (; K > 1; --K) {
