@@ -226,8 +226,6 @@ __device__ __forceinline__ void warp_max_scatter64(float (&a)[64], int lane) {
     }
 }
 
-__device__ __forceinline__ float bf16_bits_to_float(uint16_t b) { return __uint_as_float(((uint32_t)b) << 16); }
-
 // Index checks of the debug build (compiled with -DWINO_DEBUG): an access whose
 // element index i lies outside its buffer of n elements is skipped and recorded
 // in the device error word as kDevErrBounds (first error wins); nothing traps.

@@ -57,19 +57,6 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
     return ok != 0;
 }
 
-// Non-blocking test of the phase with the given parity (never suspends the thread).
-__device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}\n"
-        : "=r"(ok)
-        : "r"(smem_u32(bar)), "r"(parity)
-        : "memory");
-    return ok != 0;
-}
-
 // Waits for the phase with the given parity.  Returns false if the CTA's
 // abort flag is raised or the time limit expires (then it raises the flag and
 // records the error in the global error word).
@@ -104,15 +91,6 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, u
         "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(
             smem_u32(dst)),
         "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(smem_u32(bar))
-        : "memory");
-}
-
-// TMA: 2-D tiled global -> shared load completing on an mbarrier (no multicast).
-__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, uint64_t* bar, int c0, int c1) {
-    asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
-            smem_u32(dst)),
-        "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(smem_u32(bar))
         : "memory");
 }
 
@@ -188,7 +166,7 @@ __device__ __forceinline__ void tmem_regs_ready(uint32_t (&r)[NC]) {
     for (int i = 0; i < NC; ++i) asm volatile("" : "+r"(r[i]));
 }
 
-// 32 lanes x NC consecutive 32-bit columns (this warp's lane quadrant), NC = 4, 8, 12, 16, 20 or 32.
+// 32 lanes x NC consecutive 32-bit columns (this warp's lane quadrant), NC = 4, 8, 16, 20 or 32.
 #define WINO_R8(o) "=r"(r[o + 0]), "=r"(r[o + 1]), "=r"(r[o + 2]), "=r"(r[o + 3]), "=r"(r[o + 4]), "=r"(r[o + 5]), \
                    "=r"(r[o + 6]), "=r"(r[o + 7])
 template <int NC>
@@ -241,8 +219,6 @@ __device__ __forceinline__ void tmem_ld_pair(uint32_t taddr, uint32_t (&r)[NC]) 
     tmem_ld<NA>(taddr, *reinterpret_cast<uint32_t(*)[NA]>(&r[0]));
     tmem_ld<NB>(taddr + NA, *reinterpret_cast<uint32_t(*)[NB]>(&r[NA]));
 }
-template <>
-__device__ __forceinline__ void tmem_ld<12>(uint32_t taddr, uint32_t (&r)[12]) { tmem_ld_pair<8, 4>(taddr, r); }
 template <>
 __device__ __forceinline__ void tmem_ld<20>(uint32_t taddr, uint32_t (&r)[20]) { tmem_ld_pair<16, 4>(taddr, r); }
 
