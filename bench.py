@@ -64,6 +64,8 @@ UNIT = "TFLOP/s"
 NCU_TRAFFIC = {
     # profiles/hadamard_y32_swapped_sd15_1280x1280_8x8_full.md: 114,457,344 + 4,860,160 B
     ("F(6,3) N8 1280->1280 8x8 G64", "hadamard_y32"): 119317504,
+    # profiles/hadamard_y32_swapped_n80_sd15_1280x1280_16x16_full.md: 120,098,048 + 10,921,472 B
+    ("F(6,3) N8 1280->1280 16x16 G64", "hadamard_y32"): 131019520,
     # profiles/hadamard_y32_a_resident_sd15_320x320_64x64_full.md: 32,512,256 + 29,470,208 B
     ("F(6,3) N8 320->320 64x64 G64", "hadamard_y32"): 61982464,
     # profiles/output_transform_y32_sd15_320x320_64x64_full.md: 79,385,600 + 3,409,920 B
